@@ -1,0 +1,200 @@
+/*
+ * tp.h - C ABI of libtp, the B200 (sm_100a) tensor-parallel layer-pair library.
+ *
+ * What the library computes is defined on the Diffusers documentation page
+ * "Tensor parallelism" (Portuguese "main" edition; Chinese v0.43.0 edition):
+ *
+ *   - opening paragraph: each device holds a column-wise ("colwise") or
+ *     row-wise ("rowwise") slice of a layer's weight and computes a partial
+ *     result; the partials are combined at the layer boundary;
+ *   - section "Colwise and rowwise", style table: colwise shards the output
+ *     features (weight dim 0), each rank computing a slice of the output;
+ *     rowwise shards the input features (weight dim 1), each rank computing a
+ *     partial sum; the paragraph below it: a colwise projection followed by a
+ *     rowwise one needs a single AllReduce at the block boundary, and colwise
+ *     Q/K/V give each rank a subset of the heads;
+ *   - section "Fused projections": a Linear that packs several tensors along
+ *     the sharded dimension is sharded block by block (Q/K/V: blocks [1,1,1]);
+ *   - section "Constraints and validation": the degree must divide the head
+ *     count and every packed block, checked before any weight is split.
+ *
+ * Here all tp_degree shards live on ONE GPU: every shard's slice is
+ * materialised, each shard runs its own colwise GEMM, and the sum that the
+ * AllReduce would perform is accumulated inside the rowwise GEMM (one fp32
+ * accumulator walks every shard's K range), plus the rowwise bias once.
+ *
+ * Conventions for every entry point
+ *   - Tensors are row-major.  bf16 values travel as uint16_t bit patterns.
+ *   - Every pointer argument is a DEVICE pointer on the current CUDA device,
+ *     owned by the caller, and must be 16-byte aligned.  Workspaces must be
+ *     256-byte aligned.  Weights are nn.Linear-shaped: [out_features x in_features].
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work is enqueued on it and the call returns without waiting.
+ *   - Every argument check runs before anything is launched; a call that
+ *     returns an error has written nothing and launched nothing.  There is no
+ *     fallback path of any kind: an unsupported shape is an error.
+ *   - A returned TP_OK covers argument checks and launch errors.  A kernel's
+ *     own watchdog (every wait is bounded; a wait that runs out records an
+ *     error and the kernel exits) is reported by tp_check_device_error().
+ */
+#ifndef TP_B200_TP_H_
+#define TP_B200_TP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TP_ABI_VERSION 1
+#define TP_HEAD_DIM 128
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_NULL = 1,               /* a required pointer is NULL */
+  TP_ERR_BAD_DEGREE = 2,         /* tp_degree < 1 */
+  TP_ERR_BAD_RANK = 3,           /* rank outside [0, tp_degree) */
+  TP_ERR_INDIVISIBLE = 4,        /* a sharded dimension (or packed block) % tp_degree != 0 */
+  TP_ERR_HEADS_INDIVISIBLE = 5,  /* heads % tp_degree != 0 */
+  TP_ERR_BAD_SHAPE = 6,          /* negative/zero size, D != heads*128, size above the supported range */
+  TP_ERR_ALIGNMENT = 7,          /* pointer not 16-byte aligned, or a shard row not a multiple of 16 bytes */
+  TP_ERR_WORKSPACE = 8,          /* workspace NULL, too small or not 256-byte aligned */
+  TP_ERR_CUDA = 9,               /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
+  TP_ERR_DEVICE_TIMEOUT = 10,    /* a kernel's bounded wait ran out (see tp_check_device_error) */
+  TP_ERR_BAD_STYLE = 11,         /* unknown tp_style */
+  TP_ERR_BAD_HANDLE = 12         /* NULL or foreign handle */
+} tp_status;
+
+typedef enum {
+  TP_COLWISE = 0, /* slice output features: rows [r*N/T, (r+1)*N/T) of W[N x K] */
+  TP_ROWWISE = 1  /* slice input features: columns [r*K/T, (r+1)*K/T) of every row */
+} tp_style;
+
+/* Human-readable name of a status code (static storage). */
+const char* tp_status_string(int status);
+int tp_abi_version(void);
+
+/* Synchronises `stream`, then reports (and clears) the device error word that
+ * the kernels' bounded waits set: TP_OK, or TP_ERR_DEVICE_TIMEOUT.  Returns
+ * TP_ERR_CUDA if the synchronisation itself fails. */
+tp_status tp_check_device_error(void* stream);
+
+/* ---------------------------------------------------------------------------
+ * a1. Shard slicing (style table, "Colwise and rowwise"; "Fused projections").
+ * Bit-exact copies; a coalesced 128-bit vectorised HBM copy kernel.
+ * ------------------------------------------------------------------------- */
+
+/* out = slice `rank` of W[rows x cols] in `style`.
+ *   colwise: out is [rows/T x cols] = W[rank*rows/T : (rank+1)*rows/T, :]
+ *   rowwise: out is [rows x cols/T] = W[:, rank*cols/T : (rank+1)*cols/T]
+ * Errors: NULL, BAD_STYLE, BAD_DEGREE, BAD_RANK, BAD_SHAPE (rows or cols < 1),
+ * INDIVISIBLE (sharded dim % T), ALIGNMENT (pointers, or row lengths of W or
+ * out not multiples of 8 elements). */
+tp_status tp_shard_weight(const uint16_t* W, int64_t rows, int64_t cols, int style,
+                          int tp_degree, int rank, uint16_t* out, void* stream);
+
+/* out[n/T] = b[rank*n/T : (rank+1)*n/T] (a colwise layer's bias).  n/T must be
+ * a multiple of 8. */
+tp_status tp_shard_bias(const uint16_t* b, int64_t n, int tp_degree, int rank,
+                        uint16_t* out, void* stream);
+
+/* Head split of a fused QKV weight W_qkv[3D x D] = [Q; K; V] (D rows each,
+ * head h at rows h*128 .. h*128+127 inside each block): packed colwise with
+ * blocks [1,1,1].  out is [3D/T x D] = [Q_r; K_r; V_r], where X_r holds heads
+ * [rank*H/T, (rank+1)*H/T).  Requires D == heads*128 (BAD_SHAPE) and
+ * heads % T == 0 (HEADS_INDIVISIBLE). */
+tp_status tp_shard_qkv_heads(const uint16_t* W_qkv, int64_t D, int heads, int tp_degree,
+                             int rank, uint16_t* out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Step-level calls (each one kernel), on already-sharded operands.
+ * ------------------------------------------------------------------------- */
+
+/* a2/a3/a5. Colwise GEMM for every shard:
+ *   out[r] = epi( X[M x K] . W_shards[r]^T + b_shards[r] ),   r = 0..T-1
+ * W_shards: [T x N_s x K] (shard r's [N_s x K] weight, contiguous);
+ * b_shards: [T x N_s] or NULL; out: [T x M x N_s].  epi = GELU(tanh form)
+ * when gelu != 0, identity otherwise.  bf16 operands, fp32 accumulation in
+ * tensor memory (tcgen05), one bf16 rounding at the end.
+ * Requires K % 8 == 0 and N_s % 8 == 0 (ALIGNMENT).  M == 0 is a no-op. */
+tp_status tp_colwise_linear(const uint16_t* X, int64_t M, int64_t K,
+                            const uint16_t* W_shards, const uint16_t* b_shards, int64_t N_s,
+                            int tp_degree, int gelu, uint16_t* out, void* stream);
+
+/* a4/a7. Rowwise GEMM with the cross-shard sum fused:
+ *   Y[M x N] = bf16( sum_r A_shards[r] . W_shards[r]^T + bias )
+ * A_shards: [T x M x K_s]; W_shards: [T x N x K_s]; bias: [N] or NULL (added
+ * once, after the sum).  One fp32 accumulator walks r = 0..T-1 in order, so
+ * no partial is ever written out.  Requires K_s % 8 == 0, N % 8 == 0. */
+tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s,
+                                const uint16_t* W_shards, int64_t N, const uint16_t* bias,
+                                int tp_degree, uint16_t* Y, void* stream);
+
+/* a6. Per-shard scaled dot-product attention, non-causal, scale 1/sqrt(128):
+ * QKV: [T x M x 3*Hs*128] with Hs = heads/T; inside a row: Q heads, then K
+ * heads, then V heads, 128 columns per head (the colwise QKV output).
+ * O: [T x M x Hs*128], O[r][:, j*128:(j+1)*128] = softmax(Q K^T/sqrt(128)) V
+ * for head j of shard r.  Online softmax (running max and sum, fp32), P
+ * rounded to bf16 for the P.V product, fp32 accumulation. */
+tp_status tp_sdpa_shards(const uint16_t* QKV, int64_t M, int heads, int tp_degree,
+                         uint16_t* O, void* stream);
+
+/* a8. Standalone partial-sum reduction (the per-element meaning of the
+ * block-boundary AllReduce; the unfused alternative of a4):
+ *   Y[M x N] = bf16( sum_{r ascending} parts[r] + bias )
+ * parts: fp32 [T x M x N]; bias: [N] bf16 or NULL.  N % 8 == 0. */
+tp_status tp_reduce_partials(const float* parts, int64_t M, int64_t N, int tp_degree,
+                             const uint16_t* bias, uint16_t* Y, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Layer calls.  The one-shot calls slice the full weights into the caller's
+ * workspace (a1) and then run the layer; the prepare/run pair slices once
+ * into library-owned memory and runs many times, like sharding at load time
+ * and running a forward every step.
+ * ------------------------------------------------------------------------- */
+
+/* MLP pair: Y = bf16( sum_r GELU(X W_up,r^T + b_up,r) W_down,r^T + b_down ).
+ * X[M x D], W_up[F x D] (colwise), b_up[F], W_down[D x F] (rowwise), b_down[D],
+ * Y[M x D].  F % T == 0 (INDIVISIBLE); D and F/T multiples of 8 (ALIGNMENT).
+ * b_up / b_down may be NULL (no bias).  Workspace: tp_mlp_workspace_bytes(). */
+size_t tp_mlp_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree);
+tp_status tp_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F,
+                      const uint16_t* W_up, const uint16_t* b_up,
+                      const uint16_t* W_down, const uint16_t* b_down,
+                      int tp_degree, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* Attention block: Y = bf16( sum_r O_r W_o,r^T ), O_r = per-shard SDPA of the
+ * head-split QKV projection X W_qkv,r^T.  X[M x D], W_qkv[3D x D], W_o[D x D],
+ * Y[M x D]; D == heads*128; heads % T == 0.  No biases.
+ * Workspace: tp_attn_workspace_bytes(). */
+size_t tp_attn_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree);
+tp_status tp_attn_block(const uint16_t* X, int64_t M, int64_t D,
+                        const uint16_t* W_qkv, const uint16_t* W_o, int heads, int tp_degree,
+                        uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* Load-once / run-many.  *handle receives a library object that owns the
+ * sharded weights (device memory allocated here, freed by tp_destroy).  The
+ * slicing is enqueued on `stream`; later runs must be ordered after it.
+ * tp_*_run_workspace_bytes(M, ...) gives the activation workspace a run needs. */
+tp_status tp_mlp_prepare(const uint16_t* W_up, const uint16_t* b_up,
+                         const uint16_t* W_down, const uint16_t* b_down,
+                         int64_t D, int64_t F, int tp_degree, void* stream, void** handle);
+size_t tp_mlp_run_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree);
+tp_status tp_mlp_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y,
+                     void* ws, size_t ws_bytes, void* stream);
+
+tp_status tp_attn_prepare(const uint16_t* W_qkv, const uint16_t* W_o, int64_t D, int heads,
+                          int tp_degree, void* stream, void** handle);
+size_t tp_attn_run_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree);
+tp_status tp_attn_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Frees a handle from tp_*_prepare (synchronises the device first). NULL is a no-op. */
+void tp_destroy(void* handle);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_B200_TP_H_ */

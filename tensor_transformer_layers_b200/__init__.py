@@ -1,0 +1,312 @@
+"""Python binding of libtp (include/tp.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors (or raw device addresses as ints) and forwards plain pointers and
+sizes through ctypes.  Nothing here computes: every step of every layer runs
+in the CUDA kernels of ``libtp.so``.  If the library is missing this module
+raises on first use; there is no fallback.
+
+The convenience wrappers at the end (``mlp_pair``, ``attn_block``,
+``MlpPair``, ``AttnBlock``) only allocate outputs and workspaces with torch
+and call the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtp.so")
+
+TP_COLWISE = 0
+TP_ROWWISE = 1
+
+STATUS = {
+    0: "TP_OK", 1: "TP_ERR_NULL", 2: "TP_ERR_BAD_DEGREE", 3: "TP_ERR_BAD_RANK",
+    4: "TP_ERR_INDIVISIBLE", 5: "TP_ERR_HEADS_INDIVISIBLE", 6: "TP_ERR_BAD_SHAPE",
+    7: "TP_ERR_ALIGNMENT", 8: "TP_ERR_WORKSPACE", 9: "TP_ERR_CUDA",
+    10: "TP_ERR_DEVICE_TIMEOUT", 11: "TP_ERR_BAD_STYLE", 12: "TP_ERR_BAD_HANDLE",
+}
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/tp.h
+SIGNATURES = {
+    "tp_status_string": (ctypes.c_char_p, [_I]),
+    "tp_abi_version": (_I, []),
+    "tp_check_device_error": (_I, [_P]),
+    "tp_shard_weight": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P]),
+    "tp_shard_bias": (_I, [_P, _I64, _I, _I, _P, _P]),
+    "tp_shard_qkv_heads": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
+    "tp_colwise_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _P, _P]),
+    "tp_rowwise_linear_sum": (_I, [_P, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
+    "tp_sdpa_shards": (_I, [_P, _I64, _I, _I, _P, _P]),
+    "tp_reduce_partials": (_I, [_P, _I64, _I64, _I, _P, _P, _P]),
+    "tp_mlp_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
+    "tp_mlp_pair": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "tp_attn_workspace_bytes": (_SZ, [_I64, _I64, _I, _I]),
+    "tp_attn_block": (_I, [_P, _I64, _I64, _P, _P, _I, _I, _P, _P, _SZ, _P]),
+    "tp_mlp_prepare": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _P, ctypes.POINTER(_P)]),
+    "tp_mlp_run_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
+    "tp_mlp_run": (_I, [_P, _P, _I64, _P, _P, _SZ, _P]),
+    "tp_attn_prepare": (_I, [_P, _P, _I64, _I, _I, _P, ctypes.POINTER(_P)]),
+    "tp_attn_run_workspace_bytes": (_SZ, [_I64, _I64, _I, _I]),
+    "tp_attn_run": (_I, [_P, _P, _I64, _P, _P, _SZ, _P]),
+    "tp_destroy": (None, [_P]),
+}
+
+_lib = None
+
+
+class TPError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib().tp_status_string(status).decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libtp.so (loaded once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m tensor_transformer_layers_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return x.data_ptr()
+    return int(x)
+
+
+def _stream(s):
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, torch.cuda.Stream):
+        return s.cuda_stream
+    return int(s)
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise TPError(status, where)
+
+
+# --------------------------------------------------------------------------- raw entry points
+def tp_status_string(status: int) -> str:
+    return lib().tp_status_string(status).decode()
+
+
+def tp_abi_version() -> int:
+    return lib().tp_abi_version()
+
+
+def tp_check_device_error(stream=None) -> int:
+    return lib().tp_check_device_error(_stream(stream))
+
+
+def tp_shard_weight(W, rows, cols, style, tp_degree, rank, out, stream=None) -> int:
+    return lib().tp_shard_weight(_ptr(W), rows, cols, style, tp_degree, rank, _ptr(out), _stream(stream))
+
+
+def tp_shard_bias(b, n, tp_degree, rank, out, stream=None) -> int:
+    return lib().tp_shard_bias(_ptr(b), n, tp_degree, rank, _ptr(out), _stream(stream))
+
+
+def tp_shard_qkv_heads(W_qkv, D, heads, tp_degree, rank, out, stream=None) -> int:
+    return lib().tp_shard_qkv_heads(_ptr(W_qkv), D, heads, tp_degree, rank, _ptr(out), _stream(stream))
+
+
+def tp_colwise_linear(X, M, K, W_shards, b_shards, N_s, tp_degree, gelu, out, stream=None) -> int:
+    return lib().tp_colwise_linear(_ptr(X), M, K, _ptr(W_shards), _ptr(b_shards), N_s, tp_degree,
+                                   int(bool(gelu)), _ptr(out), _stream(stream))
+
+
+def tp_rowwise_linear_sum(A_shards, M, K_s, W_shards, N, bias, tp_degree, Y, stream=None) -> int:
+    return lib().tp_rowwise_linear_sum(_ptr(A_shards), M, K_s, _ptr(W_shards), N, _ptr(bias), tp_degree,
+                                       _ptr(Y), _stream(stream))
+
+
+def tp_sdpa_shards(QKV, M, heads, tp_degree, O, stream=None) -> int:
+    return lib().tp_sdpa_shards(_ptr(QKV), M, heads, tp_degree, _ptr(O), _stream(stream))
+
+
+def tp_reduce_partials(parts, M, N, tp_degree, bias, Y, stream=None) -> int:
+    return lib().tp_reduce_partials(_ptr(parts), M, N, tp_degree, _ptr(bias), _ptr(Y), _stream(stream))
+
+
+def tp_mlp_workspace_bytes(M, D, F, tp_degree) -> int:
+    return lib().tp_mlp_workspace_bytes(M, D, F, tp_degree)
+
+
+def tp_mlp_run_workspace_bytes(M, D, F, tp_degree) -> int:
+    return lib().tp_mlp_run_workspace_bytes(M, D, F, tp_degree)
+
+
+def tp_attn_workspace_bytes(M, D, heads, tp_degree) -> int:
+    return lib().tp_attn_workspace_bytes(M, D, heads, tp_degree)
+
+
+def tp_attn_run_workspace_bytes(M, D, heads, tp_degree) -> int:
+    return lib().tp_attn_run_workspace_bytes(M, D, heads, tp_degree)
+
+
+def tp_mlp_pair(X, M, D, F, W_up, b_up, W_down, b_down, tp_degree, Y, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_mlp_pair(_ptr(X), M, D, F, _ptr(W_up), _ptr(b_up), _ptr(W_down), _ptr(b_down), tp_degree,
+                             _ptr(Y), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def tp_attn_block(X, M, D, W_qkv, W_o, heads, tp_degree, Y, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_attn_block(_ptr(X), M, D, _ptr(W_qkv), _ptr(W_o), heads, tp_degree, _ptr(Y), _ptr(ws),
+                               ws_bytes, _stream(stream))
+
+
+def tp_mlp_prepare(W_up, b_up, W_down, b_down, D, F, tp_degree, stream=None):
+    h = _P()
+    st = lib().tp_mlp_prepare(_ptr(W_up), _ptr(b_up), _ptr(W_down), _ptr(b_down), D, F, tp_degree,
+                              _stream(stream), ctypes.byref(h))
+    return st, h.value
+
+
+def tp_mlp_run(handle, X, M, Y, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_mlp_run(handle, _ptr(X), M, _ptr(Y), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def tp_attn_prepare(W_qkv, W_o, D, heads, tp_degree, stream=None):
+    h = _P()
+    st = lib().tp_attn_prepare(_ptr(W_qkv), _ptr(W_o), D, heads, tp_degree, _stream(stream), ctypes.byref(h))
+    return st, h.value
+
+
+def tp_attn_run(handle, X, M, Y, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_attn_run(handle, _ptr(X), M, _ptr(Y), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def tp_destroy(handle) -> None:
+    lib().tp_destroy(handle)
+
+
+# --------------------------------------------------------------------------- convenience
+def _u16(t: torch.Tensor) -> torch.Tensor:
+    """bf16 bit patterns travel as 16-bit tensors; accept bfloat16 or int16/uint16 storage."""
+    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16, torch.float16):
+        raise TypeError(f"expected a 16-bit tensor of bf16 values, got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return t
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def mlp_pair(X, W_up, b_up, W_down, b_down, tp_degree: int, stream=None) -> torch.Tensor:
+    """One-shot MLP pair (slices the weights, then runs); returns Y [M, D] (bf16)."""
+    _u16(X), _u16(W_up), _u16(W_down)
+    M, D = X.shape
+    F = W_up.shape[0]
+    Y = torch.empty((M, D), dtype=torch.bfloat16, device=X.device)
+    nb = tp_mlp_workspace_bytes(M, D, F, tp_degree)
+    ws = _workspace(nb, X.device)
+    _check(tp_mlp_pair(X, M, D, F, W_up, b_up, W_down, b_down, tp_degree, Y, ws, nb, stream), "tp_mlp_pair")
+    return Y
+
+
+def attn_block(X, W_qkv, W_o, heads: int, tp_degree: int, stream=None) -> torch.Tensor:
+    """One-shot attention block; returns Y [M, D] (bf16)."""
+    _u16(X), _u16(W_qkv), _u16(W_o)
+    M, D = X.shape
+    Y = torch.empty((M, D), dtype=torch.bfloat16, device=X.device)
+    nb = tp_attn_workspace_bytes(M, D, heads, tp_degree)
+    ws = _workspace(nb, X.device)
+    _check(tp_attn_block(X, M, D, W_qkv, W_o, heads, tp_degree, Y, ws, nb, stream), "tp_attn_block")
+    return Y
+
+
+class MlpPair:
+    """Shards once (tp_mlp_prepare), runs many times (tp_mlp_run)."""
+
+    def __init__(self, W_up, b_up, W_down, b_down, tp_degree: int, stream=None):
+        self.D = W_up.shape[1]
+        self.F = W_up.shape[0]
+        self.T = tp_degree
+        st, self.handle = tp_mlp_prepare(W_up, b_up, W_down, b_down, self.D, self.F, tp_degree, stream)
+        _check(st, "tp_mlp_prepare")
+        self._ws = None
+
+    def workspace(self, M, device):
+        nb = tp_mlp_run_workspace_bytes(M, self.D, self.F, self.T)
+        if self._ws is None or self._ws.numel() < nb:
+            self._ws = _workspace(nb, device)
+        return self._ws, nb
+
+    def __call__(self, X, Y=None, stream=None) -> torch.Tensor:
+        M = X.shape[0]
+        if Y is None:
+            Y = torch.empty((M, self.D), dtype=torch.bfloat16, device=X.device)
+        ws, nb = self.workspace(M, X.device)
+        _check(tp_mlp_run(self.handle, X, M, Y, ws, nb, stream), "tp_mlp_run")
+        return Y
+
+    def close(self):
+        if self.handle:
+            tp_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 - interpreter shutdown
+            pass
+
+
+class AttnBlock:
+    """Shards once (tp_attn_prepare), runs many times (tp_attn_run)."""
+
+    def __init__(self, W_qkv, W_o, heads: int, tp_degree: int, stream=None):
+        self.D = W_qkv.shape[1]
+        self.heads = heads
+        self.T = tp_degree
+        st, self.handle = tp_attn_prepare(W_qkv, W_o, self.D, heads, tp_degree, stream)
+        _check(st, "tp_attn_prepare")
+        self._ws = None
+
+    def workspace(self, M, device):
+        nb = tp_attn_run_workspace_bytes(M, self.D, self.heads, self.T)
+        if self._ws is None or self._ws.numel() < nb:
+            self._ws = _workspace(nb, device)
+        return self._ws, nb
+
+    def __call__(self, X, Y=None, stream=None) -> torch.Tensor:
+        M = X.shape[0]
+        if Y is None:
+            Y = torch.empty((M, self.D), dtype=torch.bfloat16, device=X.device)
+        ws, nb = self.workspace(M, X.device)
+        _check(tp_attn_run(self.handle, X, M, Y, ws, nb, stream), "tp_attn_run")
+        return Y
+
+    def close(self):
+        if self.handle:
+            tp_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001
+            pass

@@ -1,0 +1,627 @@
+// api.cu - the C ABI declared in include/tp.h: argument checks, workspace
+// layout, TMA tensor maps, handles, and the launch sequence of each layer.
+//
+// Error policy (Diffusers "Tensor parallelism" page, sections "Limitations"
+// and "Constraints and validation"): every constraint is checked before any
+// weight is sliced or any kernel is launched, and a failed check returns an
+// error instead of doing something else silently.  Nothing here computes on
+// the host: every step of every layer runs in the kernels of slice.cu,
+// gemm.cu, attn.cu and reduce.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tp.h"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace tp {
+
+__device__ int g_device_error;  // OR of kErr* bits set by kernels' bounded waits
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kMlpMagic = 0x54504D4C50484E44ull;   // "TPMLPHND"
+constexpr uint64_t kAttnMagic = 0x5450415454484E44ull;  // "TPATTHND"
+constexpr int64_t kMaxDim = int64_t(1) << 31;           // TMA coordinates are 32-bit
+
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+  int* err = nullptr;  // device address of g_device_error
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+tp_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TP_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return TP_ERR_CUDA;
+    d.err = static_cast<int*>(p);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return TP_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return TP_OK;
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t up256(size_t n) { return (n + 255) & ~size_t(255); }
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                          uint32_t box1) {
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};  // bytes, dims 1 and 2
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Internal launch helpers (arguments already validated).
+// ---------------------------------------------------------------------------
+
+// colwise: out[g] = epi(X . W[g]^T + b[g]), g < T.
+tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, const uint16_t* b,
+                      int64_t Ns, int T, int gelu, uint16_t* out, cudaStream_t s) {
+  if (M == 0) return TP_OK;
+  CUtensorMap amap, bmap;
+  if (make_map_3d_bf16(&amap, X, uint64_t(K), uint64_t(M), 1, 64, 128) != CUDA_SUCCESS) return TP_ERR_CUDA;
+  if (make_map_3d_bf16(&bmap, W, uint64_t(K), uint64_t(Ns), uint64_t(T), 64, 256) != CUDA_SUCCESS) return TP_ERR_CUDA;
+  GemmArgs a;
+  a.M = int(M);
+  a.N = int(Ns);
+  a.k_blocks = int((K + 63) / 64);
+  a.kshards = 1;
+  a.groups = T;
+  a.a_follows_shard = 0;
+  a.out = out;
+  a.out_gstride = M * Ns;
+  a.ldo = Ns;
+  a.bias = b;
+  a.bias_gstride = Ns;
+  a.gelu = gelu;
+  a.err = di->err;
+  return launch_gemm(amap, bmap, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+// rowwise: Y = sum_r A[r] . W[r]^T + bias.
+tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, const uint16_t* W, int64_t N,
+                      const uint16_t* bias, int T, uint16_t* Y, cudaStream_t s) {
+  if (M == 0) return TP_OK;
+  CUtensorMap amap, bmap;
+  if (make_map_3d_bf16(&amap, A, uint64_t(Ks), uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS) return TP_ERR_CUDA;
+  if (make_map_3d_bf16(&bmap, W, uint64_t(Ks), uint64_t(N), uint64_t(T), 64, 256) != CUDA_SUCCESS) return TP_ERR_CUDA;
+  GemmArgs a;
+  a.M = int(M);
+  a.N = int(N);
+  a.k_blocks = int((Ks + 63) / 64);
+  a.kshards = T;
+  a.groups = 1;
+  a.a_follows_shard = 1;
+  a.out = Y;
+  a.out_gstride = 0;
+  a.ldo = N;
+  a.bias = bias;
+  a.bias_gstride = 0;
+  a.gelu = 0;
+  a.err = di->err;
+  return launch_gemm(amap, bmap, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status run_sdpa(DeviceInfo* di, const uint16_t* QKV, int64_t M, int heads, int T, uint16_t* O, cudaStream_t s) {
+  if (M == 0) return TP_OK;
+  const int Hs = heads / T;
+  CUtensorMap map;
+  if (make_map_3d_bf16(&map, QKV, uint64_t(3) * Hs * TP_HEAD_DIM, uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS)
+    return TP_ERR_CUDA;
+  AttnArgs a;
+  a.M = int(M);
+  a.Hs = Hs;
+  a.T = T;
+  a.out = O;
+  a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(TP_HEAD_DIM)));  // log2(e) / sqrt(d)
+  a.err = di->err;
+  return launch_attention(map, a, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+// Slices of whole weights (all T shards), used by the one-shot calls and prepare.
+tp_status slice_all_colwise(const uint16_t* W, int64_t rows, int64_t cols, uint16_t* out, cudaStream_t s) {
+  // Colwise shards stacked in rank order occupy W's own layout: one contiguous copy.
+  return launch_slice_copy(W, out, 1, rows, cols, cols, 0, 0, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status slice_all_rowwise(const uint16_t* W, int64_t rows, int64_t cols, int T, uint16_t* out, cudaStream_t s) {
+  const int64_t cs = cols / T;
+  // shard r: rows x cs block starting at column r*cs; blocks are the shards.
+  return launch_slice_copy(W, out, T, rows, cs, cols, cs, rows * cs, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status slice_all_qkv(const uint16_t* Wqkv, int64_t D, int T, uint16_t* out, cudaStream_t s) {
+  // shard r = [Q_r; K_r; V_r]; X_r = rows [r*D/T, (r+1)*D/T) of block X.
+  const int64_t rs = D / T;
+  for (int r = 0; r < T; ++r) {
+    if (launch_slice_copy(Wqkv + r * rs * D, out + int64_t(r) * 3 * rs * D, 3, rs, D, D, D * D, rs * D, s) !=
+        cudaSuccess)
+      return TP_ERR_CUDA;
+  }
+  return TP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Shape checks shared by the layer calls.
+// ---------------------------------------------------------------------------
+tp_status check_mlp_shape(int64_t M, int64_t D, int64_t F, int T) {
+  if (T < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || D < 1 || F < 1 || M >= kMaxDim || D >= kMaxDim || F >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (F % T != 0) return TP_ERR_INDIVISIBLE;
+  if (D % 8 != 0 || (F / T) % 8 != 0) return TP_ERR_ALIGNMENT;
+  return TP_OK;
+}
+
+tp_status check_attn_shape(int64_t M, int64_t D, int heads, int T) {
+  if (T < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || D < 1 || heads < 1 || M >= kMaxDim || D >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (heads % T != 0) return TP_ERR_HEADS_INDIVISIBLE;
+  if (D != int64_t(heads) * TP_HEAD_DIM) return TP_ERR_BAD_SHAPE;
+  return TP_OK;
+}
+
+struct MlpLayout {
+  size_t w_up, b_up, w_down, h, total;
+};
+MlpLayout mlp_layout(int64_t M, int64_t D, int64_t F, bool with_weights) {
+  MlpLayout L{};
+  size_t off = 0;
+  if (with_weights) {
+    L.w_up = off;
+    off += up256(size_t(F) * D * 2);
+    L.b_up = off;
+    off += up256(size_t(F) * 2);
+    L.w_down = off;
+    off += up256(size_t(D) * F * 2);
+  }
+  L.h = off;
+  off += up256(size_t(M) * F * 2);
+  L.total = off;
+  return L;
+}
+
+struct AttnLayout {
+  size_t w_qkv, w_o, qkv, o, total;
+};
+AttnLayout attn_layout(int64_t M, int64_t D, bool with_weights) {
+  AttnLayout L{};
+  size_t off = 0;
+  if (with_weights) {
+    L.w_qkv = off;
+    off += up256(size_t(3) * D * D * 2);
+    L.w_o = off;
+    off += up256(size_t(D) * D * 2);
+  }
+  L.qkv = off;
+  off += up256(size_t(M) * 3 * D * 2);
+  L.o = off;
+  off += up256(size_t(M) * D * 2);
+  L.total = off;
+  return L;
+}
+
+tp_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return TP_OK;
+  if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return TP_ERR_WORKSPACE;
+  return TP_OK;
+}
+
+// The MLP pair on sharded weights (a2..a4).
+tp_status mlp_forward(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t D, int64_t F, int T,
+                      const uint16_t* w_up_sh, const uint16_t* b_up_sh, const uint16_t* w_down_sh,
+                      const uint16_t* b_down, uint16_t* H, uint16_t* Y, cudaStream_t s) {
+  const int64_t Fs = F / T;
+  tp_status st = run_colwise(di, X, M, D, w_up_sh, b_up_sh, Fs, T, 1, H, s);
+  if (st != TP_OK) return st;
+  return run_rowwise(di, H, M, Fs, w_down_sh, D, b_down, T, Y, s);
+}
+
+// The attention block on sharded weights (a5..a7).
+tp_status attn_forward(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t D, int heads, int T,
+                       const uint16_t* w_qkv_sh, const uint16_t* w_o_sh, uint16_t* QKV, uint16_t* O, uint16_t* Y,
+                       cudaStream_t s) {
+  const int64_t Ds = D / T;
+  tp_status st = run_colwise(di, X, M, D, w_qkv_sh, nullptr, 3 * Ds, T, 0, QKV, s);
+  if (st != TP_OK) return st;
+  st = run_sdpa(di, QKV, M, heads, T, O, s);
+  if (st != TP_OK) return st;
+  return run_rowwise(di, O, M, Ds, w_o_sh, D, nullptr, T, Y, s);
+}
+
+struct MlpHandle {
+  uint64_t magic;
+  int device;
+  int64_t D, F;
+  int T;
+  uint16_t* w_up;    // [T][F/T][D]
+  uint16_t* b_up;    // [T][F/T] or null
+  uint16_t* w_down;  // [T][D][F/T]
+  uint16_t* b_down;  // [D] or null (replicated)
+};
+
+struct AttnHandle {
+  uint64_t magic;
+  int device;
+  int64_t D;
+  int heads, T;
+  uint16_t* w_qkv;  // [T][3D/T][D]
+  uint16_t* w_o;    // [T][D][D/T]
+};
+
+}  // namespace
+}  // namespace tp
+
+using namespace tp;
+
+extern "C" {
+
+const char* tp_status_string(int s) {
+  switch (s) {
+    case TP_OK: return "ok";
+    case TP_ERR_NULL: return "a required pointer is NULL";
+    case TP_ERR_BAD_DEGREE: return "tp_degree must be >= 1";
+    case TP_ERR_BAD_RANK: return "rank outside [0, tp_degree)";
+    case TP_ERR_INDIVISIBLE: return "a sharded dimension is not divisible by tp_degree";
+    case TP_ERR_HEADS_INDIVISIBLE: return "tp_degree does not divide the number of attention heads";
+    case TP_ERR_BAD_SHAPE: return "unsupported shape";
+    case TP_ERR_ALIGNMENT: return "pointer or shard row not 16-byte aligned";
+    case TP_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case TP_ERR_CUDA: return "CUDA call failed";
+    case TP_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait timed out";
+    case TP_ERR_BAD_STYLE: return "unknown sharding style";
+    case TP_ERR_BAD_HANDLE: return "invalid handle";
+    default: return "unknown status";
+  }
+}
+
+int tp_abi_version(void) { return TP_ABI_VERSION; }
+
+tp_status tp_check_device_error(void* stream) {
+  DeviceInfo* di = nullptr;
+  tp_status st = device_info(&di);
+  if (st != TP_OK) return st;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return TP_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, di->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TP_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TP_ERR_CUDA;
+    return TP_ERR_DEVICE_TIMEOUT;
+  }
+  return TP_OK;
+}
+
+// ----------------------------------------------------------------------- a1
+tp_status tp_shard_weight(const uint16_t* W, int64_t rows, int64_t cols, int style, int tp_degree, int rank,
+                          uint16_t* out, void* stream) {
+  if (!W || !out) return TP_ERR_NULL;
+  if (style != TP_COLWISE && style != TP_ROWWISE) return TP_ERR_BAD_STYLE;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (rank < 0 || rank >= tp_degree) return TP_ERR_BAD_RANK;
+  if (rows < 1 || cols < 1) return TP_ERR_BAD_SHAPE;
+  if (style == TP_COLWISE && rows % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  if (style == TP_ROWWISE && cols % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  if (!al16(W) || !al16(out) || cols % 8 != 0) return TP_ERR_ALIGNMENT;
+  if (style == TP_ROWWISE && (cols / tp_degree) % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaError_t e;
+  if (style == TP_COLWISE) {
+    const int64_t rs = rows / tp_degree;
+    e = launch_slice_copy(W + int64_t(rank) * rs * cols, out, 1, rs, cols, cols, 0, 0, as_stream(stream));
+  } else {
+    const int64_t cs = cols / tp_degree;
+    e = launch_slice_copy(W + int64_t(rank) * cs, out, 1, rows, cs, cols, 0, 0, as_stream(stream));
+  }
+  return e == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status tp_shard_bias(const uint16_t* b, int64_t n, int tp_degree, int rank, uint16_t* out, void* stream) {
+  if (!b || !out) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (rank < 0 || rank >= tp_degree) return TP_ERR_BAD_RANK;
+  if (n < 1) return TP_ERR_BAD_SHAPE;
+  if (n % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  const int64_t ns = n / tp_degree;
+  if (!al16(b) || !al16(out) || ns % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return launch_slice_copy(b + int64_t(rank) * ns, out, 1, 1, ns, ns, 0, 0, as_stream(stream)) == cudaSuccess
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_shard_qkv_heads(const uint16_t* W_qkv, int64_t D, int heads, int tp_degree, int rank, uint16_t* out,
+                             void* stream) {
+  if (!W_qkv || !out) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (rank < 0 || rank >= tp_degree) return TP_ERR_BAD_RANK;
+  if (D < 1 || heads < 1) return TP_ERR_BAD_SHAPE;
+  if (heads % tp_degree != 0) return TP_ERR_HEADS_INDIVISIBLE;
+  if (D != int64_t(heads) * TP_HEAD_DIM) return TP_ERR_BAD_SHAPE;
+  if (!al16(W_qkv) || !al16(out)) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  const int64_t rs = D / tp_degree;
+  return launch_slice_copy(W_qkv + int64_t(rank) * rs * D, out, 3, rs, D, D, D * D, rs * D, as_stream(stream)) ==
+                 cudaSuccess
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------- step-level calls
+tp_status tp_colwise_linear(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W_shards,
+                            const uint16_t* b_shards, int64_t N_s, int tp_degree, int gelu, uint16_t* out,
+                            void* stream) {
+  if (!X || !W_shards || !out) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || K < 1 || N_s < 1 || M >= kMaxDim || K >= kMaxDim || N_s * tp_degree >= kMaxDim)
+    return TP_ERR_BAD_SHAPE;
+  if (!al16(X) || !al16(W_shards) || !al16(out) || (b_shards && !al16(b_shards))) return TP_ERR_ALIGNMENT;
+  if (K % 8 != 0 || N_s % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_colwise(di, X, M, K, W_shards, b_shards, N_s, tp_degree, gelu ? 1 : 0, out, as_stream(stream));
+}
+
+tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s, const uint16_t* W_shards,
+                                int64_t N, const uint16_t* bias, int tp_degree, uint16_t* Y, void* stream) {
+  if (!A_shards || !W_shards || !Y) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || K_s < 1 || N < 1 || M >= kMaxDim || K_s >= kMaxDim || N >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (!al16(A_shards) || !al16(W_shards) || !al16(Y) || (bias && !al16(bias))) return TP_ERR_ALIGNMENT;
+  if (K_s % 8 != 0 || N % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_rowwise(di, A_shards, M, K_s, W_shards, N, bias, tp_degree, Y, as_stream(stream));
+}
+
+tp_status tp_sdpa_shards(const uint16_t* QKV, int64_t M, int heads, int tp_degree, uint16_t* O, void* stream) {
+  if (!QKV || !O) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || heads < 1 || M >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (heads % tp_degree != 0) return TP_ERR_HEADS_INDIVISIBLE;
+  if (!al16(QKV) || !al16(O)) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_sdpa(di, QKV, M, heads, tp_degree, O, as_stream(stream));
+}
+
+tp_status tp_reduce_partials(const float* parts, int64_t M, int64_t N, int tp_degree, const uint16_t* bias,
+                             uint16_t* Y, void* stream) {
+  if (!parts || !Y) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || N < 1) return TP_ERR_BAD_SHAPE;
+  if (!al16(parts) || !al16(Y) || (bias && !al16(bias)) || N % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return launch_reduce_partials(parts, M, N, tp_degree, bias, Y, as_stream(stream)) == cudaSuccess ? TP_OK
+                                                                                                   : TP_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------------- MLP pair
+size_t tp_mlp_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree) {
+  if (check_mlp_shape(M, D, F, tp_degree) != TP_OK) return 0;
+  return mlp_layout(M, D, F, true).total;
+}
+
+size_t tp_mlp_run_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree) {
+  if (check_mlp_shape(M, D, F, tp_degree) != TP_OK) return 0;
+  return mlp_layout(M, D, F, false).total;
+}
+
+tp_status tp_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F, const uint16_t* W_up,
+                      const uint16_t* b_up, const uint16_t* W_down, const uint16_t* b_down, int tp_degree,
+                      uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !W_up || !W_down || !Y) return TP_ERR_NULL;
+  tp_status st = check_mlp_shape(M, D, F, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(X) || !al16(W_up) || !al16(W_down) || !al16(Y) || (b_up && !al16(b_up)) || (b_down && !al16(b_down)))
+    return TP_ERR_ALIGNMENT;
+  if (M == 0) return TP_OK;  // empty input: nothing to compute or write
+  const MlpLayout L = mlp_layout(M, D, F, true);
+  st = check_ws(ws, ws_bytes, L.total);
+  if (st != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* w_up_sh = reinterpret_cast<uint16_t*>(w + L.w_up);
+  uint16_t* b_up_sh = b_up ? reinterpret_cast<uint16_t*>(w + L.b_up) : nullptr;
+  uint16_t* w_down_sh = reinterpret_cast<uint16_t*>(w + L.w_down);
+  uint16_t* H = reinterpret_cast<uint16_t*>(w + L.h);
+  // a1: materialise every shard (what each rank would hold after sharded loading).
+  if ((st = slice_all_colwise(W_up, F, D, w_up_sh, s)) != TP_OK) return st;
+  if (b_up && (st = slice_all_colwise(b_up, 1, F, b_up_sh, s)) != TP_OK) return st;
+  if ((st = slice_all_rowwise(W_down, D, F, tp_degree, w_down_sh, s)) != TP_OK) return st;
+  // a2..a4
+  return mlp_forward(di, X, M, D, F, tp_degree, w_up_sh, b_up_sh, w_down_sh, b_down, H, Y, s);
+}
+
+tp_status tp_mlp_prepare(const uint16_t* W_up, const uint16_t* b_up, const uint16_t* W_down, const uint16_t* b_down,
+                         int64_t D, int64_t F, int tp_degree, void* stream, void** handle) {
+  if (!W_up || !W_down || !handle) return TP_ERR_NULL;
+  tp_status st = check_mlp_shape(0, D, F, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(W_up) || !al16(W_down) || (b_up && !al16(b_up)) || (b_down && !al16(b_down))) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  MlpHandle* h = new MlpHandle{};
+  h->magic = kMlpMagic;
+  cudaGetDevice(&h->device);
+  h->D = D;
+  h->F = F;
+  h->T = tp_degree;
+  bool ok = cudaMalloc(&h->w_up, size_t(F) * D * 2) == cudaSuccess &&
+            cudaMalloc(&h->w_down, size_t(D) * F * 2) == cudaSuccess &&
+            (!b_up || cudaMalloc(&h->b_up, size_t(F) * 2) == cudaSuccess) &&
+            (!b_down || cudaMalloc(&h->b_down, size_t(D) * 2) == cudaSuccess);
+  ok = ok && slice_all_colwise(W_up, F, D, h->w_up, s) == TP_OK &&
+       slice_all_rowwise(W_down, D, F, tp_degree, h->w_down, s) == TP_OK &&
+       (!b_up || slice_all_colwise(b_up, 1, F, h->b_up, s) == TP_OK) &&
+       (!b_down || cudaMemcpyAsync(h->b_down, b_down, size_t(D) * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess);
+  if (!ok) {
+    tp_destroy(h);
+    return TP_ERR_CUDA;
+  }
+  *handle = h;
+  return TP_OK;
+}
+
+tp_status tp_mlp_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y, void* ws, size_t ws_bytes,
+                     void* stream) {
+  MlpHandle* h = static_cast<MlpHandle*>(handle);
+  if (!h) return TP_ERR_BAD_HANDLE;
+  if (h->magic != kMlpMagic) return TP_ERR_BAD_HANDLE;
+  if (!X || !Y) return TP_ERR_NULL;
+  tp_status st = check_mlp_shape(M, h->D, h->F, h->T);
+  if (st != TP_OK) return st;
+  if (!al16(X) || !al16(Y)) return TP_ERR_ALIGNMENT;
+  if (M == 0) return TP_OK;
+  const MlpLayout L = mlp_layout(M, h->D, h->F, false);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  uint16_t* H = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.h);
+  return mlp_forward(di, X, M, h->D, h->F, h->T, h->w_up, h->b_up, h->w_down, h->b_down, H, Y, as_stream(stream));
+}
+
+// ----------------------------------------------------------------------- attention block
+size_t tp_attn_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree) {
+  if (check_attn_shape(M, D, heads, tp_degree) != TP_OK) return 0;
+  return attn_layout(M, D, true).total;
+}
+
+size_t tp_attn_run_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree) {
+  if (check_attn_shape(M, D, heads, tp_degree) != TP_OK) return 0;
+  return attn_layout(M, D, false).total;
+}
+
+tp_status tp_attn_block(const uint16_t* X, int64_t M, int64_t D, const uint16_t* W_qkv, const uint16_t* W_o,
+                        int heads, int tp_degree, uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !W_qkv || !W_o || !Y) return TP_ERR_NULL;
+  tp_status st = check_attn_shape(M, D, heads, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(X) || !al16(W_qkv) || !al16(W_o) || !al16(Y)) return TP_ERR_ALIGNMENT;
+  if (M == 0) return TP_OK;
+  const AttnLayout L = attn_layout(M, D, true);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* wq = reinterpret_cast<uint16_t*>(w + L.w_qkv);
+  uint16_t* wo = reinterpret_cast<uint16_t*>(w + L.w_o);
+  if ((st = slice_all_qkv(W_qkv, D, tp_degree, wq, s)) != TP_OK) return st;
+  if ((st = slice_all_rowwise(W_o, D, D, tp_degree, wo, s)) != TP_OK) return st;
+  return attn_forward(di, X, M, D, heads, tp_degree, wq, wo, reinterpret_cast<uint16_t*>(w + L.qkv),
+                      reinterpret_cast<uint16_t*>(w + L.o), Y, s);
+}
+
+tp_status tp_attn_prepare(const uint16_t* W_qkv, const uint16_t* W_o, int64_t D, int heads, int tp_degree,
+                          void* stream, void** handle) {
+  if (!W_qkv || !W_o || !handle) return TP_ERR_NULL;
+  tp_status st = check_attn_shape(0, D, heads, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(W_qkv) || !al16(W_o)) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  AttnHandle* h = new AttnHandle{};
+  h->magic = kAttnMagic;
+  cudaGetDevice(&h->device);
+  h->D = D;
+  h->heads = heads;
+  h->T = tp_degree;
+  bool ok = cudaMalloc(&h->w_qkv, size_t(3) * D * D * 2) == cudaSuccess &&
+            cudaMalloc(&h->w_o, size_t(D) * D * 2) == cudaSuccess;
+  ok = ok && slice_all_qkv(W_qkv, D, tp_degree, h->w_qkv, s) == TP_OK &&
+       slice_all_rowwise(W_o, D, D, tp_degree, h->w_o, s) == TP_OK;
+  if (!ok) {
+    tp_destroy(h);
+    return TP_ERR_CUDA;
+  }
+  *handle = h;
+  return TP_OK;
+}
+
+tp_status tp_attn_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y, void* ws, size_t ws_bytes,
+                      void* stream) {
+  AttnHandle* h = static_cast<AttnHandle*>(handle);
+  if (!h) return TP_ERR_BAD_HANDLE;
+  if (h->magic != kAttnMagic) return TP_ERR_BAD_HANDLE;
+  if (!X || !Y) return TP_ERR_NULL;
+  tp_status st = check_attn_shape(M, h->D, h->heads, h->T);
+  if (st != TP_OK) return st;
+  if (!al16(X) || !al16(Y)) return TP_ERR_ALIGNMENT;
+  if (M == 0) return TP_OK;
+  const AttnLayout L = attn_layout(M, h->D, false);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  return attn_forward(di, X, M, h->D, h->heads, h->T, h->w_qkv, h->w_o, reinterpret_cast<uint16_t*>(w + L.qkv),
+                      reinterpret_cast<uint16_t*>(w + L.o), Y, as_stream(stream));
+}
+
+void tp_destroy(void* handle) {
+  if (!handle) return;
+  const uint64_t magic = *static_cast<uint64_t*>(handle);
+  if (magic == kMlpMagic) {
+    MlpHandle* h = static_cast<MlpHandle*>(handle);
+    cudaDeviceSynchronize();
+    cudaFree(h->w_up);
+    cudaFree(h->b_up);
+    cudaFree(h->w_down);
+    cudaFree(h->b_down);
+    h->magic = 0;
+    delete h;
+  } else if (magic == kAttnMagic) {
+    AttnHandle* h = static_cast<AttnHandle*>(handle);
+    cudaDeviceSynchronize();
+    cudaFree(h->w_qkv);
+    cudaFree(h->w_o);
+    h->magic = 0;
+    delete h;
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,325 @@
+// attn.cu - a6, per-shard scaled dot-product attention on tcgen05.
+//
+// Under tensor parallelism the colwise Q/K/V projections give each rank a
+// subset of the heads (Diffusers "Tensor parallelism" page, section "Colwise
+// and rowwise", paragraph on attention), so attention runs independently per
+// (shard, head).  For every head j of shard r and every 128-row query tile:
+//     O = softmax(Q K^T / sqrt(128)) V     (non-causal, no mask)
+// computed with an online softmax over 128-key tiles.
+//
+// Structure (one CTA per (shard, head, query tile), 192 threads):
+//   warps 0-3  softmax: thread i owns query row i (its TMEM lane), so the row
+//              max and row sum are per-thread reductions over the 128 columns
+//              it loads; p = 2^(s*log2(e)/sqrt(d) - m) with the hardware ex2;
+//              P is packed to bf16 pairs and written to TMEM; O is rescaled in
+//              TMEM only when the running max grows by more than 2^8 (the
+//              stale max is otherwise kept for both O and the row sum, which
+//              leaves the final O/l unchanged); final O/l -> bf16 -> global.
+//   warp 4     TMA producer: Q once, then K and V tiles into a 2-stage ring.
+//   warp 5     TMEM allocator + MMA issuer: S_j = Q K_j^T (both operands in
+//              shared memory, K-major) into one of two S buffers, so S_{j+1}
+//              is computed while row j's softmax runs; O += P_j V_j with P read
+//              from TMEM and V in shared memory as an MN-major operand.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P [384,448) (bf16 pairs).
+// Every mbarrier wait is bounded (ptx.cuh); a timeout drains and exits.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace tp {
+namespace {
+
+constexpr int kD = 128;       // head dim
+constexpr int kBQ = 128;      // query rows per CTA
+constexpr int kBKV = 128;     // keys per tile
+constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16 (16 KB)
+constexpr int kQBytes = 2 * kBox;   // Q tile: d in two 64-column boxes
+constexpr int kKVBytes = 4 * kBox;  // K tile (2 boxes) + V tile (2 boxes)
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr int kQOff = 0;
+constexpr int kKVOff = kQBytes;
+constexpr int kBarOff = kKVOff + kStages * kKVBytes;
+constexpr int kSmemBytes = kBarOff + 256 + 1024;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr uint32_t kIdescS = idesc_bf16_f32(kBQ, kBKV, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(kBQ, kD, true);  // B (= V) is MN-major
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qkv, const AttnArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_empty = bars + 7;   // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pv_done = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int qb = blockIdx.x;
+  const int shard = blockIdx.y / p.Hs;
+  const int head = blockIdx.y - shard * p.Hs;
+  const int n_kv = (p.M + kBKV - 1) / kBKV;
+  const int qcol = head * kD;
+  const int kcol = (p.Hs + head) * kD;
+  const int vcol = (2 * p.Hs + head) * kD;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&qkv);
+      uint8_t* sq = smem + kQOff;
+      mbar_arrive_expect_tx(q_full, kQBytes);
+      tma_load_3d(sq, &qkv, q_full, qcol, qb * kBQ, shard);
+      tma_load_3d(sq + kBox, &qkv, q_full, qcol + 64, qb * kBQ, shard);
+      bool ok = true;
+      int issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sk = smem + kKVOff + st * kKVBytes;
+        mbar_arrive_expect_tx(&kv_full[st], kKVBytes);
+        tma_load_3d(sk, &qkv, &kv_full[st], kcol, j * kBKV, shard);
+        tma_load_3d(sk + kBox, &qkv, &kv_full[st], kcol + 64, j * kBKV, shard);
+        tma_load_3d(sk + 2 * kBox, &qkv, &kv_full[st], vcol, j * kBKV, shard);
+        tma_load_3d(sk + 3 * kBox, &qkv, &kv_full[st], vcol + 64, j * kBKV, shard);
+        ++issued;
+      }
+      if (!ok) {
+        report_timeout(p.err, abort_flag);
+        const volatile int no_abort = 0;
+        mbar_wait(q_full, 0, &no_abort);
+        // the last (up to) two tiles issued may still be landing
+        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
+          mbar_wait(&kv_full[j & 1], (j >> 1) & 1, &no_abort);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      const uint32_t sq = smem_u32(smem + kQOff);
+      auto issue_s = [&](int j) -> bool {
+        const int st = j & 1;
+        if (!mbar_wait(&kv_full[st], (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&s_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t sk = smem_u32(smem + kKVOff + st * kKVBytes);
+        const uint32_t d_tmem = tmem_base + kColS + uint32_t(st * kBKV);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = uint32_t((kk >> 2) * kBox + (kk & 3) * 32);
+          umma_ss(d_tmem, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), kIdescS,
+                  kk != 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[st]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv) {
+          if (!issue_s(j + 1)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!mbar_wait(p_full, j & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int st = j & 1;
+        const uint32_t sv = smem_u32(smem + kKVOff + st * kKVBytes + 2 * kBox);
+#pragma unroll
+        for (int kk = 0; kk < kBKV / 16; ++kk) {
+          // 16 keys per step: rows kk*16.. of both V boxes (LBO = box stride, SBO = 8 rows).
+          umma_ts(tmem_base + kColO, tmem_base + kColP + uint32_t(kk * 8),
+                  sdesc_sw128(sv + uint32_t(kk * 16 * 128), kBox, 1024), kIdescPV, (j | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(pv_done);
+        umma_commit(&kv_empty[st]);
+      }
+      if (!ok) {
+        report_timeout(p.err, abort_flag);
+        const volatile int no_abort = 0;
+        umma_commit(drain);
+        mbar_wait(drain, 0, &no_abort);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-3)
+    const int row = qb * kBQ + warp * 32 + lane;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    float m_run = -INFINITY;  // running max (log2-scaled units) used for O and l
+    float l_run = 0.f;
+    bool ok = true;
+    const float sl2 = p.scale_log2;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&s_full[st], (j >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[kBKV];
+#pragma unroll
+      for (int c = 0; c < kBKV / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32_sync(tmem_base + lane_off + kColS + uint32_t(st * kBKV + c * 32), r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[st]);
+
+      const int kv0 = j * kBKV;
+      if (kv0 + kBKV > p.M) {  // ragged last key tile: keys >= M do not exist
+#pragma unroll
+        for (int i = 0; i < kBKV; ++i)
+          if (kv0 + i >= p.M) s[i] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < kBKV; ++i) mx = fmaxf(mx, s[i]);
+      mx *= sl2;
+      // P and O are free once the previous P.V finished.
+      if (j > 0) {
+        if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (j == 0) {
+        m_run = mx;
+      } else {
+        // Rescale only rows whose max grew by more than the threshold; the TMEM
+        // accesses are warp-collective, so the whole warp takes the branch if any
+        // lane needs it (other lanes scale by 1).
+        const bool need = mx > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m_run - mx) : 1.0f;
+          if (need) {
+            m_run = mx;
+            l_run *= alpha;
+          }
+#pragma unroll 1
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t r[32];
+            const uint32_t ta = tmem_base + lane_off + kColO + uint32_t(c * 32);
+            tmem_ld32_sync(ta, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(ta, r);
+          }
+        }
+      }
+      float lsum = 0.f;
+      uint32_t pk[kBKV / 2];
+#pragma unroll
+      for (int i = 0; i < kBKV / 2; ++i) {
+        const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -m_run));
+        const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -m_run));
+        lsum += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      l_run += lsum;
+#pragma unroll
+      for (int c = 0; c < kBKV / 64; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
+        tmem_st32(tmem_base + lane_off + kColP + uint32_t(c * 32), r);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok) ok = mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l_run;
+      uint16_t* orow = p.out + (int64_t(shard) * p.M + row) * int64_t(p.Hs * kD) + head * kD;
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32_sync(tmem_base + lane_off + kColO + uint32_t(c * 32), r);
+        uint4 o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          o[i].x = pack_bf16x2(__uint_as_float(r[8 * i + 0]) * inv_l, __uint_as_float(r[8 * i + 1]) * inv_l);
+          o[i].y = pack_bf16x2(__uint_as_float(r[8 * i + 2]) * inv_l, __uint_as_float(r[8 * i + 3]) * inv_l);
+          o[i].z = pack_bf16x2(__uint_as_float(r[8 * i + 4]) * inv_l, __uint_as_float(r[8 * i + 5]) * inv_l);
+          o[i].w = pack_bf16x2(__uint_as_float(r[8 * i + 6]) * inv_l, __uint_as_float(r[8 * i + 7]) * inv_l);
+        }
+        if (row < p.M) {
+          uint4* op = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) op[i] = o[i];
+        }
+      }
+    }
+    if (!ok && lane == 0) report_timeout(p.err, abort_flag);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s) {
+  if (a.M <= 0) return cudaSuccess;
+  const int q_tiles = (a.M + kBQ - 1) / kBQ;
+  dim3 grid(static_cast<unsigned>(q_tiles), static_cast<unsigned>(a.T * a.Hs));
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(qkv_map, a);
+  return cudaGetLastError();
+}
+
+}  // namespace tp

@@ -1,0 +1,70 @@
+// internal.h - launchers shared between the C-ABI layer (api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace tp {
+
+// ----------------------------------------------------------------------------
+// a1: blocked 2-D copy.  For b in [0, nblocks), r in [0, rows), c in [0, cols):
+//   dst[b*dst_bstride + r*cols + c] = src[b*src_bstride + r*src_ld + c]
+// (element units).  cols, src_ld, the strides and both pointers must be
+// multiples of 8 elements / 16 bytes (checked by the caller).
+// ----------------------------------------------------------------------------
+cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblocks, int64_t rows, int64_t cols,
+                              int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t s);
+
+// ----------------------------------------------------------------------------
+// a8: Y[M x N] = bf16(sum_r parts[r] + bias)
+// ----------------------------------------------------------------------------
+cudaError_t launch_reduce_partials(const float* parts, int64_t M, int64_t N, int T, const uint16_t* bias,
+                                   uint16_t* Y, cudaStream_t s);
+
+// ----------------------------------------------------------------------------
+// GEMM (tcgen05).  Computes, for each output group g and tile:
+//   out_g[M x N] = epi( sum_{s in K-shards of g} A_{za(s)} . B_{zb(g,s)}^T + bias_g )
+// A map: 3-D bf16 {K_s, M, ZA}; B map: 3-D bf16 {K_s, Nrows, ZB}.
+//   colwise: groups = T, kshards = 1, zb = g, za = 0.
+//   rowwise: groups = 1, kshards = T, zb = s, za = s.
+// ----------------------------------------------------------------------------
+struct GemmArgs {
+  int M;                 // output rows
+  int N;                 // output columns per group
+  int k_blocks;          // ceil(K_s / 64) per shard
+  int kshards;           // shards walked by one tile's K loop
+  int groups;            // output groups (colwise shards)
+  int a_follows_shard;   // 1: A's z coordinate = K-loop shard; 0: z = 0
+  uint16_t* out;         // bf16 output
+  int64_t out_gstride;   // elements between groups
+  int64_t ldo;           // output row stride (elements)
+  const uint16_t* bias;  // bf16 bias or nullptr
+  int64_t bias_gstride;  // elements between groups' biases
+  int gelu;              // 1: tanh-form GELU after bias
+  int* err;              // device error word
+};
+
+cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmArgs& a, int num_sms,
+                        cudaStream_t s);
+
+// ----------------------------------------------------------------------------
+// a6: per-shard SDPA.  qkv map: 3-D bf16 {3*Hs*128, M, T}, box {64, 128, 1}.
+// ----------------------------------------------------------------------------
+struct AttnArgs {
+  int M;            // tokens
+  int Hs;           // heads per shard
+  int T;            // shards
+  uint16_t* out;    // [T x M x Hs*128]
+  float scale_log2; // log2(e)/sqrt(128)
+  int* err;
+};
+
+cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s);
+
+// Host helpers (api.cu).
+CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                          uint32_t box0, uint32_t box1);
+
+}  // namespace tp

@@ -1,0 +1,79 @@
+// slice.cu - a1, shard slicing: a coalesced 128-bit vectorised blocked copy.
+//
+// A colwise shard (rows [r*N/T, (r+1)*N/T) of a row-major W[N x K]) is one
+// contiguous span; a rowwise shard (columns [r*K/T, (r+1)*K/T) of every row)
+// is N row segments of K/T elements at stride K; the packed head split of a
+// fused QKV weight is three contiguous spans.  All three are instances of a
+// blocked 2-D copy, done here with 16-byte loads/stores.  Each thread keeps
+// four 16-byte loads in flight before storing, and loads/stores use the
+// streaming cache policy: the data is touched exactly once.
+#include "internal.h"
+
+namespace tp {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+__global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                              uint32_t rows, uint32_t c8, int64_t src_ld8,
+                                                              int64_t src_b8, int64_t dst_b8) {
+  const uint32_t total = rows * c8;  // chunks in this block (host guarantees < 2^31)
+  const uint4* s = src + int64_t(blockIdx.y) * src_b8;
+  uint4* d = dst + int64_t(blockIdx.y) * dst_b8;
+  const uint32_t stride = gridDim.x * kThreads;
+  for (uint32_t base = blockIdx.x * kThreads + threadIdx.x; base < total; base += stride * kUnroll) {
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t j = base + u * stride;
+      if (j < total) {
+        const uint32_t r = j / c8;
+        const uint32_t c = j - r * c8;
+        v[u] = __ldcs(s + int64_t(r) * src_ld8 + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t j = base + u * stride;
+      if (j < total) __stcs(d + j, v[u]);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblocks, int64_t rows, int64_t cols,
+                              int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t st) {
+  if (nblocks <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
+  // A contiguous source (row segments back to back) is copied as one long span,
+  // split into virtual rows so the 32-bit chunk index never overflows.
+  if (src_ld == cols) {
+    int64_t n8 = rows * cols / 8;
+    int64_t vc8 = 1;
+    for (int64_t cand : {int64_t(4096), int64_t(1024), int64_t(256), int64_t(64), int64_t(8), int64_t(1)})
+      if (n8 % cand == 0) { vc8 = cand; break; }
+    rows = n8 / vc8;
+    cols = vc8 * 8;
+    src_ld = cols;
+  }
+  const int64_t c8 = cols / 8;
+  // Split very tall copies into pieces whose chunk count fits 31 bits.
+  const int64_t max_rows = (int64_t(1) << 30) / c8;
+  for (int64_t r0 = 0; r0 < rows; r0 += max_rows) {
+    const int64_t nr = rows - r0 < max_rows ? rows - r0 : max_rows;
+    const int64_t total = nr * c8;
+    int64_t blocks = (total + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks < 1) blocks = 1;
+    dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(nblocks));
+    slice_copy_kernel<<<grid, kThreads, 0, st>>>(reinterpret_cast<const uint4*>(src + r0 * src_ld),
+                                                 reinterpret_cast<uint4*>(dst + r0 * cols), uint32_t(nr),
+                                                 uint32_t(c8), src_ld / 8, src_bstride / 8, dst_bstride / 8);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace tp

@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/tp.h declares, and rejects bad arguments with the
+documented status before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tensor_transformer_layers_b200 as tp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tp.h")
+
+A = 1 << 20  # a fake, 256-byte aligned "device address" (never dereferenced: checks fail first)
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tp_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_builds_and_loads():
+    assert os.path.exists(tp.LIB_PATH), "libtp.so missing; run python -m tensor_transformer_layers_b200.build"
+    assert tp.tp_abi_version() == 1
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) >= 20
+    lib = ctypes.CDLL(tp.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert missing == []
+    assert set(names) == set(tp.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings():
+    for code in range(13):
+        assert tp.tp_status_string(code) not in ("", "unknown status")
+    assert tp.tp_status_string(99) == "unknown status"
+
+
+def test_workspace_sizes():
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    M, D, F, T = 4608, 3072, 12288, 4
+    assert tp.tp_mlp_workspace_bytes(M, D, F, T) == up(F * D * 2) + up(F * 2) + up(D * F * 2) + up(M * F * 2)
+    assert tp.tp_mlp_run_workspace_bytes(M, D, F, T) == up(M * F * 2)
+    assert tp.tp_attn_workspace_bytes(M, D, 24, T) == up(3 * D * D * 2) + up(D * D * 2) + up(M * 3 * D * 2) + up(M * D * 2)
+    assert tp.tp_attn_run_workspace_bytes(M, D, 24, T) == up(M * 3 * D * 2) + up(M * D * 2)
+    # invalid shapes report 0
+    assert tp.tp_mlp_workspace_bytes(M, D, F, 5) == 0
+    assert tp.tp_attn_workspace_bytes(M, D, 24, 5) == 0
+    assert tp.tp_attn_workspace_bytes(M, 3000, 24, 4) == 0
+
+
+S = {v: k for k, v in tp.STATUS.items()}
+
+
+@pytest.mark.parametrize("args,want", [
+    ((0, 8, 8, tp.TP_COLWISE, 2, 0, A), "TP_ERR_NULL"),
+    ((A, 8, 8, 7, 2, 0, A), "TP_ERR_BAD_STYLE"),
+    ((A, 8, 8, tp.TP_COLWISE, 0, 0, A), "TP_ERR_BAD_DEGREE"),
+    ((A, 8, 8, tp.TP_COLWISE, 2, 2, A), "TP_ERR_BAD_RANK"),
+    ((A, 8, 8, tp.TP_COLWISE, 2, -1, A), "TP_ERR_BAD_RANK"),
+    ((A, 0, 8, tp.TP_COLWISE, 1, 0, A), "TP_ERR_BAD_SHAPE"),
+    ((A, 9, 8, tp.TP_COLWISE, 2, 0, A), "TP_ERR_INDIVISIBLE"),
+    ((A, 8, 24, tp.TP_ROWWISE, 5, 0, A), "TP_ERR_INDIVISIBLE"),
+    ((A + 2, 8, 8, tp.TP_COLWISE, 2, 0, A), "TP_ERR_ALIGNMENT"),
+    ((A, 8, 12, tp.TP_COLWISE, 2, 0, A), "TP_ERR_ALIGNMENT"),
+    ((A, 8, 24, tp.TP_ROWWISE, 2, 0, A), "TP_ERR_ALIGNMENT"),  # 12-element shard rows
+])
+def test_shard_weight_checks(args, want):
+    assert tp.tp_shard_weight(*args, stream=0) == S[want]
+
+
+def test_qkv_and_bias_checks():
+    assert tp.tp_shard_qkv_heads(A, 384, 3, 2, 0, A, stream=0) == S["TP_ERR_HEADS_INDIVISIBLE"]
+    assert tp.tp_shard_qkv_heads(A, 300, 3, 1, 0, A, stream=0) == S["TP_ERR_BAD_SHAPE"]
+    assert tp.tp_shard_qkv_heads(A, 384, 3, 3, 3, A, stream=0) == S["TP_ERR_BAD_RANK"]
+    assert tp.tp_shard_bias(A, 100, 3, 0, A, stream=0) == S["TP_ERR_INDIVISIBLE"]
+    assert tp.tp_shard_bias(A, 24, 2, 0, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+
+
+def test_layer_checks():
+    ws = 1 << 30
+    # MLP pair
+    assert tp.tp_mlp_pair(A, 64, 128, 512, A, A, A, A, 3, A, A, ws, stream=0) == S["TP_ERR_INDIVISIBLE"]
+    assert tp.tp_mlp_pair(A, 64, 128, 512, A, A, A, A, 0, A, A, ws, stream=0) == S["TP_ERR_BAD_DEGREE"]
+    assert tp.tp_mlp_pair(A, 64, 128, 520, A, A, A, A, 4, A, A, ws, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_mlp_pair(A, -1, 128, 512, A, A, A, A, 2, A, A, ws, stream=0) == S["TP_ERR_BAD_SHAPE"]
+    assert tp.tp_mlp_pair(None, 64, 128, 512, A, A, A, A, 2, A, A, ws, stream=0) == S["TP_ERR_NULL"]
+    assert tp.tp_mlp_pair(A, 64, 128, 512, A, A, A, A, 2, A, A, 100, stream=0) == S["TP_ERR_WORKSPACE"]
+    assert tp.tp_mlp_pair(A, 64, 128, 512, A, A, A, A, 2, A, A + 16, ws, stream=0) == S["TP_ERR_WORKSPACE"]
+    assert tp.tp_mlp_pair(A, 64, 128, 512, A, A + 8, A, A, 2, A, A, ws, stream=0) == S["TP_ERR_ALIGNMENT"]
+    # an empty input is valid and does nothing (no device access)
+    assert tp.tp_mlp_pair(A, 0, 128, 512, A, A, A, A, 2, A, None, 0, stream=0) == 0
+    # attention block: the degree must divide the head count, D must be heads*128
+    assert tp.tp_attn_block(A, 64, 768, A, A, 6, 4, A, A, ws, stream=0) == S["TP_ERR_HEADS_INDIVISIBLE"]
+    assert tp.tp_attn_block(A, 64, 700, A, A, 6, 2, A, A, ws, stream=0) == S["TP_ERR_BAD_SHAPE"]
+    assert tp.tp_attn_block(A, 64, 768, A, A, 6, 2, A, A, 10, stream=0) == S["TP_ERR_WORKSPACE"]
+    assert tp.tp_attn_block(A, 0, 768, A, A, 6, 2, A, None, 0, stream=0) == 0
+    # step-level calls
+    assert tp.tp_colwise_linear(A, 64, 100, A, None, 64, 2, 1, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_rowwise_linear_sum(A, 64, 64, A, 100, None, 2, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_sdpa_shards(A, 64, 6, 4, A, stream=0) == S["TP_ERR_HEADS_INDIVISIBLE"]
+    assert tp.tp_reduce_partials(A, 64, 100, 2, None, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_reduce_partials(A, 64, 64, 0, None, A, stream=0) == S["TP_ERR_BAD_DEGREE"]
+    # handles
+    assert tp.tp_mlp_run(None, A, 64, A, A, ws, stream=0) == S["TP_ERR_BAD_HANDLE"]
+    assert tp.tp_attn_run(None, A, 64, A, A, ws, stream=0) == S["TP_ERR_BAD_HANDLE"]
+    st, h = tp.tp_mlp_prepare(A, A, A, A, 128, 512, 3, stream=0)
+    assert st == S["TP_ERR_INDIVISIBLE"] and not h
+    st, h = tp.tp_attn_prepare(A, A, 768, 6, 4, stream=0)
+    assert st == S["TP_ERR_HEADS_INDIVISIBLE"] and not h
+    tp.tp_destroy(None)

@@ -1,0 +1,64 @@
+"""Colwise (a2/a3/a5) and rowwise (a4/a7) tcgen05 GEMMs against the oracle,
+including ragged M, N and K tails and tiny sizes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as o
+import synthetic as syn
+import tensor_transformer_layers_b200 as tp
+from tests._util import assert_parity, f64, from_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("M,K,Ns,T,gelu,bias", [
+    (64, 128, 256, 2, True, True),     # tiny MLP's FFN-in
+    (1, 64, 8, 1, False, False),
+    (129, 72, 264, 3, True, True),     # ragged M, N and K tails
+    (300, 1024, 512, 4, False, True),
+    (256, 3072, 2304, 1, False, False),  # one QKV shard of the Flux attention block
+])
+def test_colwise(M, K, Ns, T, gelu, bias):
+    X = syn.normal_bf16((M, K), 1.0, seed=M, tid=300)
+    W = syn.normal_bf16((T, Ns, K), 1.0 / np.sqrt(K), seed=K, tid=301)
+    b = syn.normal_bf16((T, Ns), 0.02, seed=Ns, tid=302) if bias else None
+    out = torch.empty((T, M, Ns), dtype=torch.int16, device="cuda")
+    st = tp.tp_colwise_linear(to_dev(X), M, K, to_dev(W), to_dev(b) if bias else None, Ns, T, gelu, out)
+    assert st == 0
+    torch.cuda.synchronize()
+    g = from_dev(out)
+    act = o.gelu_tanh if gelu else (lambda x: x)
+    for r in range(T):
+        ref = act(o.linear(f64(X), f64(W[r]), f64(b[r]) if bias else None))
+        assert_parity(g[r], ref, f"colwise shard {r}")
+
+
+@pytest.mark.parametrize("M,Ks,N,T,bias", [
+    (64, 256, 128, 2, True),           # tiny MLP's FFN-out
+    (1, 8, 8, 1, True),
+    (129, 72, 264, 3, True),           # ragged
+    (300, 512, 520, 4, False),
+    (256, 768, 3072, 4, False),        # Flux attention out-projection shards
+])
+def test_rowwise_sum(M, Ks, N, T, bias):
+    A = syn.normal_bf16((T, M, Ks), 1.0, seed=M, tid=310)
+    W = syn.normal_bf16((T, N, Ks), 1.0 / np.sqrt(T * Ks), seed=Ks, tid=311)
+    b = syn.normal_bf16((N,), 0.02, seed=N, tid=312) if bias else None
+    Y = torch.empty((M, N), dtype=torch.int16, device="cuda")
+    st = tp.tp_rowwise_linear_sum(to_dev(A), M, Ks, to_dev(W), N, to_dev(b) if bias else None, T, Y)
+    assert st == 0
+    torch.cuda.synchronize()
+    ref = o.reduce_partials([o.linear(f64(A[r]), f64(W[r])) for r in range(T)], f64(b) if bias else None)
+    assert_parity(from_dev(Y), ref, "rowwise")
+
+
+def test_colwise_identity_weight_passes_input_through():
+    # W = I (bf16 exact) and no bias: every output equals its input exactly.
+    M, K = 200, 256
+    X = syn.normal_bf16((M, K), 1.0, seed=5, tid=320)
+    I = syn.f64_to_bf16_bits(np.eye(K))
+    out = torch.empty((1, M, K), dtype=torch.int16, device="cuda")
+    assert tp.tp_colwise_linear(to_dev(X), M, K, to_dev(I), None, K, 1, 0, out) == 0
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev(out)[0], X)
