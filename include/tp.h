@@ -71,9 +71,19 @@ typedef enum {
   TP_ROWWISE = 1  /* slice input features: columns [r*K/T, (r+1)*K/T) of every row */
 } tp_style;
 
+/* Storage type of a 16-bit activation output. */
+typedef enum {
+  TP_OUT_BF16 = 0,
+  TP_OUT_F16 = 1
+} tp_out_dtype;
+
 /* Human-readable name of a status code (static storage). */
 const char* tp_status_string(int status);
 int tp_abi_version(void);
+
+/* Number of kernels this library has launched in this process (all devices,
+ * all threads); a telemetry counter for benchmarks. */
+uint64_t tp_kernel_launches(void);
 
 /* Synchronises `stream`, then reports (and clears) the device error word that
  * the kernels' bounded waits set: TP_OK, or TP_ERR_DEVICE_TIMEOUT.  Returns
@@ -93,6 +103,14 @@ tp_status tp_check_device_error(void* stream);
  * out not multiples of 8 elements). */
 tp_status tp_shard_weight(const uint16_t* W, int64_t rows, int64_t cols, int style,
                           int tp_degree, int rank, uint16_t* out, void* stream);
+
+/* All T shards of W in one launch, stacked in rank order:
+ *   colwise: out is [T x rows/T x cols] (the same bytes as W: a colwise shard
+ *            of a row-major weight is a contiguous block of rows);
+ *   rowwise: out is [T x rows x cols/T].
+ * Same checks as tp_shard_weight (without `rank`). */
+tp_status tp_shard_weight_all(const uint16_t* W, int64_t rows, int64_t cols, int style,
+                              int tp_degree, uint16_t* out, void* stream);
 
 /* out[n/T] = b[rank*n/T : (rank+1)*n/T] (a colwise layer's bias).  n/T must be
  * a multiple of 8. */
@@ -116,11 +134,13 @@ tp_status tp_shard_qkv_heads(const uint16_t* W_qkv, int64_t D, int heads, int tp
  * W_shards: [T x N_s x K] (shard r's [N_s x K] weight, contiguous);
  * b_shards: [T x N_s] or NULL; out: [T x M x N_s].  epi = GELU(tanh form)
  * when gelu != 0, identity otherwise.  bf16 operands, fp32 accumulation in
- * tensor memory (tcgen05), one bf16 rounding at the end.
+ * tensor memory (tcgen05), one rounding at the end to out_dtype
+ * (TP_OUT_BF16, or TP_OUT_F16 as used for the Q/K/V that feed attention;
+ * anything else is TP_ERR_BAD_STYLE).
  * Requires K % 8 == 0 and N_s % 8 == 0 (ALIGNMENT).  M == 0 is a no-op. */
 tp_status tp_colwise_linear(const uint16_t* X, int64_t M, int64_t K,
                             const uint16_t* W_shards, const uint16_t* b_shards, int64_t N_s,
-                            int tp_degree, int gelu, uint16_t* out, void* stream);
+                            int tp_degree, int gelu, int out_dtype, uint16_t* out, void* stream);
 
 /* a4/a7. Rowwise GEMM with the cross-shard sum fused:
  *   Y[M x N] = bf16( sum_r A_shards[r] . W_shards[r]^T + bias )
@@ -132,11 +152,12 @@ tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s
                                 int tp_degree, uint16_t* Y, void* stream);
 
 /* a6. Per-shard scaled dot-product attention, non-causal, scale 1/sqrt(128):
- * QKV: [T x M x 3*Hs*128] with Hs = heads/T; inside a row: Q heads, then K
- * heads, then V heads, 128 columns per head (the colwise QKV output).
- * O: [T x M x Hs*128], O[r][:, j*128:(j+1)*128] = softmax(Q K^T/sqrt(128)) V
+ * QKV: fp16 [T x M x 3*Hs*128] with Hs = heads/T; inside a row: Q heads,
+ * then K heads, then V heads, 128 columns per head (the colwise QKV output,
+ * stored in fp16 by the attention block).
+ * O: bf16 [T x M x Hs*128], O[r][:, j*128:(j+1)*128] = softmax(Q K^T/sqrt(128)) V
  * for head j of shard r.  Online softmax (running max and sum, fp32), P
- * rounded to bf16 for the P.V product, fp32 accumulation. */
+ * rounded to fp16 for the P.V product, fp32 accumulation. */
 tp_status tp_sdpa_shards(const uint16_t* QKV, int64_t M, int heads, int tp_degree,
                          uint16_t* O, void* stream);
 

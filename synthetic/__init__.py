@@ -95,6 +95,18 @@ def normal_bf16(shape, std: float, seed: int, tid: int) -> np.ndarray:
     return out.reshape(shape)
 
 
+def normal_f16(shape, std: float, seed: int, tid: int) -> np.ndarray:
+    """The same seeded draws as ``normal_bf16`` (bf16-valued), encoded as fp16 bit
+    patterns (uint16).  bf16 values of moderate magnitude are exact in fp16."""
+    v = bf16_bits_to_f64(normal_bf16(shape, std, seed, tid))
+    return v.astype(np.float16).view(np.uint16)
+
+
+def f16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact decode of fp16 bit patterns (uint16) to float64."""
+    return np.ascontiguousarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
     """Exact decode of bf16 bit patterns (uint16) to float64."""
     b = np.ascontiguousarray(bits, dtype=np.uint16)

@@ -22,6 +22,8 @@ LIB_PATH = os.path.join(_HERE, "libtp.so")
 
 TP_COLWISE = 0
 TP_ROWWISE = 1
+TP_OUT_BF16 = 0
+TP_OUT_F16 = 1
 
 STATUS = {
     0: "TP_OK", 1: "TP_ERR_NULL", 2: "TP_ERR_BAD_DEGREE", 3: "TP_ERR_BAD_RANK",
@@ -41,9 +43,11 @@ SIGNATURES = {
     "tp_abi_version": (_I, []),
     "tp_check_device_error": (_I, [_P]),
     "tp_shard_weight": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P]),
+    "tp_shard_weight_all": (_I, [_P, _I64, _I64, _I, _I, _P, _P]),
+    "tp_kernel_launches": (ctypes.c_uint64, []),
     "tp_shard_bias": (_I, [_P, _I64, _I, _I, _P, _P]),
     "tp_shard_qkv_heads": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
-    "tp_colwise_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _P, _P]),
+    "tp_colwise_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _I, _P, _P]),
     "tp_rowwise_linear_sum": (_I, [_P, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
     "tp_sdpa_shards": (_I, [_P, _I64, _I, _I, _P, _P]),
     "tp_reduce_partials": (_I, [_P, _I64, _I64, _I, _P, _P, _P]),
@@ -124,6 +128,14 @@ def tp_shard_weight(W, rows, cols, style, tp_degree, rank, out, stream=None) -> 
     return lib().tp_shard_weight(_ptr(W), rows, cols, style, tp_degree, rank, _ptr(out), _stream(stream))
 
 
+def tp_shard_weight_all(W, rows, cols, style, tp_degree, out, stream=None) -> int:
+    return lib().tp_shard_weight_all(_ptr(W), rows, cols, style, tp_degree, _ptr(out), _stream(stream))
+
+
+def tp_kernel_launches() -> int:
+    return lib().tp_kernel_launches()
+
+
 def tp_shard_bias(b, n, tp_degree, rank, out, stream=None) -> int:
     return lib().tp_shard_bias(_ptr(b), n, tp_degree, rank, _ptr(out), _stream(stream))
 
@@ -132,9 +144,9 @@ def tp_shard_qkv_heads(W_qkv, D, heads, tp_degree, rank, out, stream=None) -> in
     return lib().tp_shard_qkv_heads(_ptr(W_qkv), D, heads, tp_degree, rank, _ptr(out), _stream(stream))
 
 
-def tp_colwise_linear(X, M, K, W_shards, b_shards, N_s, tp_degree, gelu, out, stream=None) -> int:
+def tp_colwise_linear(X, M, K, W_shards, b_shards, N_s, tp_degree, gelu, out_dtype, out, stream=None) -> int:
     return lib().tp_colwise_linear(_ptr(X), M, K, _ptr(W_shards), _ptr(b_shards), N_s, tp_degree,
-                                   int(bool(gelu)), _ptr(out), _stream(stream))
+                                   int(bool(gelu)), int(out_dtype), _ptr(out), _stream(stream))
 
 
 def tp_rowwise_linear_sum(A_shards, M, K_s, W_shards, N, bias, tp_degree, Y, stream=None) -> int:

@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -38,6 +39,7 @@ struct DeviceInfo {
 
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
+std::atomic<uint64_t> g_launches{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -74,15 +76,26 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 }  // namespace
 
-CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
-                          uint32_t box1) {
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static CUresult make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                            uint64_t d2, uint32_t box0, uint32_t box1) {
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};  // bytes, dims 1 and 2
   const cuuint32_t box[3] = {box0, box1, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
-  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estride,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                          uint32_t box1) {
+  return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d0, d1, d2, box0, box1);
+}
+
+CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                         uint32_t box1) {
+  return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, d0, d1, d2, box0, box1);
 }
 
 namespace {
@@ -93,7 +106,7 @@ namespace {
 
 // colwise: out[g] = epi(X . W[g]^T + b[g]), g < T.
 tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, const uint16_t* b,
-                      int64_t Ns, int T, int gelu, uint16_t* out, cudaStream_t s) {
+                      int64_t Ns, int T, int gelu, int out_f16, uint16_t* out, cudaStream_t s) {
   if (M == 0) return TP_OK;
   CUtensorMap amap, bmap;
   if (make_map_3d_bf16(&amap, X, uint64_t(K), uint64_t(M), 1, 64, 128) != CUDA_SUCCESS) return TP_ERR_CUDA;
@@ -111,6 +124,7 @@ tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, c
   a.bias = b;
   a.bias_gstride = Ns;
   a.gelu = gelu;
+  a.out_f16 = out_f16;
   a.err = di->err;
   return launch_gemm(amap, bmap, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
@@ -135,6 +149,7 @@ tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, 
   a.bias = bias;
   a.bias_gstride = 0;
   a.gelu = 0;
+  a.out_f16 = 0;
   a.err = di->err;
   return launch_gemm(amap, bmap, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
@@ -143,7 +158,7 @@ tp_status run_sdpa(DeviceInfo* di, const uint16_t* QKV, int64_t M, int heads, in
   if (M == 0) return TP_OK;
   const int Hs = heads / T;
   CUtensorMap map;
-  if (make_map_3d_bf16(&map, QKV, uint64_t(3) * Hs * TP_HEAD_DIM, uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS)
+  if (make_map_3d_f16(&map, QKV, uint64_t(3) * Hs * TP_HEAD_DIM, uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS)
     return TP_ERR_CUDA;
   AttnArgs a;
   a.M = int(M);
@@ -248,7 +263,7 @@ tp_status mlp_forward(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t D, i
                       const uint16_t* w_up_sh, const uint16_t* b_up_sh, const uint16_t* w_down_sh,
                       const uint16_t* b_down, uint16_t* H, uint16_t* Y, cudaStream_t s) {
   const int64_t Fs = F / T;
-  tp_status st = run_colwise(di, X, M, D, w_up_sh, b_up_sh, Fs, T, 1, H, s);
+  tp_status st = run_colwise(di, X, M, D, w_up_sh, b_up_sh, Fs, T, 1, 0, H, s);
   if (st != TP_OK) return st;
   return run_rowwise(di, H, M, Fs, w_down_sh, D, b_down, T, Y, s);
 }
@@ -258,7 +273,8 @@ tp_status attn_forward(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t D, 
                        const uint16_t* w_qkv_sh, const uint16_t* w_o_sh, uint16_t* QKV, uint16_t* O, uint16_t* Y,
                        cudaStream_t s) {
   const int64_t Ds = D / T;
-  tp_status st = run_colwise(di, X, M, D, w_qkv_sh, nullptr, 3 * Ds, T, 0, QKV, s);
+  // Q/K/V are stored in fp16 for the attention kernel (see attn.cu, "Precision").
+  tp_status st = run_colwise(di, X, M, D, w_qkv_sh, nullptr, 3 * Ds, T, 0, 1, QKV, s);
   if (st != TP_OK) return st;
   st = run_sdpa(di, QKV, M, heads, T, O, s);
   if (st != TP_OK) return st;
@@ -313,6 +329,8 @@ const char* tp_status_string(int s) {
 
 int tp_abi_version(void) { return TP_ABI_VERSION; }
 
+uint64_t tp_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
 tp_status tp_check_device_error(void* stream) {
   DeviceInfo* di = nullptr;
   tp_status st = device_info(&di);
@@ -353,6 +371,22 @@ tp_status tp_shard_weight(const uint16_t* W, int64_t rows, int64_t cols, int sty
   return e == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
+tp_status tp_shard_weight_all(const uint16_t* W, int64_t rows, int64_t cols, int style, int tp_degree, uint16_t* out,
+                              void* stream) {
+  if (!W || !out) return TP_ERR_NULL;
+  if (style != TP_COLWISE && style != TP_ROWWISE) return TP_ERR_BAD_STYLE;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (rows < 1 || cols < 1) return TP_ERR_BAD_SHAPE;
+  if (style == TP_COLWISE && rows % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  if (style == TP_ROWWISE && cols % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  if (!al16(W) || !al16(out) || cols % 8 != 0) return TP_ERR_ALIGNMENT;
+  if (style == TP_ROWWISE && (cols / tp_degree) % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return style == TP_COLWISE ? slice_all_colwise(W, rows, cols, out, as_stream(stream))
+                             : slice_all_rowwise(W, rows, cols, tp_degree, out, as_stream(stream));
+}
+
 tp_status tp_shard_bias(const uint16_t* b, int64_t n, int tp_degree, int rank, uint16_t* out, void* stream) {
   if (!b || !out) return TP_ERR_NULL;
   if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
@@ -388,17 +422,19 @@ tp_status tp_shard_qkv_heads(const uint16_t* W_qkv, int64_t D, int heads, int tp
 
 // ----------------------------------------------------------------------- step-level calls
 tp_status tp_colwise_linear(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W_shards,
-                            const uint16_t* b_shards, int64_t N_s, int tp_degree, int gelu, uint16_t* out,
-                            void* stream) {
+                            const uint16_t* b_shards, int64_t N_s, int tp_degree, int gelu, int out_dtype,
+                            uint16_t* out, void* stream) {
   if (!X || !W_shards || !out) return TP_ERR_NULL;
   if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
   if (M < 0 || K < 1 || N_s < 1 || M >= kMaxDim || K >= kMaxDim || N_s * tp_degree >= kMaxDim)
     return TP_ERR_BAD_SHAPE;
   if (!al16(X) || !al16(W_shards) || !al16(out) || (b_shards && !al16(b_shards))) return TP_ERR_ALIGNMENT;
   if (K % 8 != 0 || N_s % 8 != 0) return TP_ERR_ALIGNMENT;
+  if (out_dtype != TP_OUT_BF16 && out_dtype != TP_OUT_F16) return TP_ERR_BAD_STYLE;
   DeviceInfo* di = nullptr;
   if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
-  return run_colwise(di, X, M, K, W_shards, b_shards, N_s, tp_degree, gelu ? 1 : 0, out, as_stream(stream));
+  return run_colwise(di, X, M, K, W_shards, b_shards, N_s, tp_degree, gelu ? 1 : 0, out_dtype == TP_OUT_F16 ? 1 : 0,
+                     out, as_stream(stream));
 }
 
 tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s, const uint16_t* W_shards,

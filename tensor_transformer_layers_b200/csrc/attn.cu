@@ -11,7 +11,7 @@
 //   warps 0-3  softmax: thread i owns query row i (its TMEM lane), so the row
 //              max and row sum are per-thread reductions over the 128 columns
 //              it loads; p = 2^(s*log2(e)/sqrt(d) - m) with the hardware ex2;
-//              P is packed to bf16 pairs and written to TMEM; O is rescaled in
+//              P is packed to fp16 pairs and written to TMEM; O is rescaled in
 //              TMEM only when the running max grows by more than 2^8 (the
 //              stale max is otherwise kept for both O and the row sum, which
 //              leaves the final O/l unchanged); final O/l -> bf16 -> global.
@@ -20,7 +20,14 @@
 //              shared memory, K-major) into one of two S buffers, so S_{j+1}
 //              is computed while row j's softmax runs; O += P_j V_j with P read
 //              from TMEM and V in shared memory as an MN-major operand.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P [384,448) (bf16 pairs).
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P [384,448) (fp16 pairs).
+//
+// Precision: Q, K, V arrive in fp16 and P is rounded to fp16 (11-bit
+// significand; |Q|, |K|, |V| of a unit-variance projection stay far below the
+// fp16 limit, and P <= 2^8 by the rescale rule), because bf16's 8-bit
+// significand at these two points alone costs more than the stated max-error
+// budget of the block.  S, the row statistics and O accumulate in fp32; O is
+// written in bf16 for the out-projection.
 // Every mbarrier wait is bounded (ptx.cuh); a timeout drains and exits.
 #include <cuda_bf16.h>
 
@@ -43,8 +50,8 @@ constexpr int kKVOff = kQBytes;
 constexpr int kBarOff = kKVOff + kStages * kKVBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
-constexpr uint32_t kIdescS = idesc_bf16_f32(kBQ, kBKV, false);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(kBQ, kD, true);  // B (= V) is MN-major
+constexpr uint32_t kIdescS = idesc_f32acc(kBQ, kBKV, false, false);  // fp16 Q, K
+constexpr uint32_t kIdescPV = idesc_f32acc(kBQ, kD, false, true);    // fp16 P, V; B (= V) is MN-major
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -259,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -m_run));
         const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -m_run));
         lsum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
+        pk[i] = pack_f16x2(p0, p1);
       }
       l_run += lsum;
 #pragma unroll
@@ -319,6 +326,7 @@ cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cuda
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(qkv_map, a);
+  count_launch();
   return cudaGetLastError();
 }
 

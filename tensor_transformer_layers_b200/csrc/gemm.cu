@@ -20,8 +20,9 @@
 //            epilogue.  Two 256-column fp32 accumulators (all 512 TMEM
 //            columns) let tile i+1's MMAs run while tile i drains.
 //   warps 2-5 epilogue: tcgen05.ld 32 columns at a time (thread = output
-//            row), bias, optional tanh-form GELU, bf16 rounding, 16-byte
-//            global stores; then release the accumulator.
+//            row), bias, optional tanh-form GELU, rounding to bf16 (or fp16
+//            for the Q/K/V projection that feeds attention), 16-byte global
+//            stores; then release the accumulator.
 // Every mbarrier wait is bounded (see ptx.cuh): a wait that runs out sets the
 // device error word, the CTA's roles stop, in-flight copies and MMAs are
 // drained with bounded waits, TMEM is freed and the kernel returns.
@@ -248,12 +249,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
         }
         uint4 o[4];
+        if (p.out_f16) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          o[j].x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-          o[j].y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-          o[j].z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-          o[j].w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+          for (int j = 0; j < 4; ++j) {
+            o[j].x = pack_f16x2(v[8 * j + 0], v[8 * j + 1]);
+            o[j].y = pack_f16x2(v[8 * j + 2], v[8 * j + 3]);
+            o[j].z = pack_f16x2(v[8 * j + 4], v[8 * j + 5]);
+            o[j].w = pack_f16x2(v[8 * j + 6], v[8 * j + 7]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            o[j].x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+            o[j].y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+            o[j].z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+            o[j].w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+          }
         }
         if (row < p.M) {
           uint4* op = reinterpret_cast<uint4*>(orow + col0);
@@ -290,6 +301,7 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(amap, bmap, a);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -43,6 +43,7 @@ struct GemmArgs {
   const uint16_t* bias;  // bf16 bias or nullptr
   int64_t bias_gstride;  // elements between groups' biases
   int gelu;              // 1: tanh-form GELU after bias
+  int out_f16;           // 1: store fp16 instead of bf16
   int* err;              // device error word
 };
 
@@ -50,7 +51,7 @@ cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const 
                         cudaStream_t s);
 
 // ----------------------------------------------------------------------------
-// a6: per-shard SDPA.  qkv map: 3-D bf16 {3*Hs*128, M, T}, box {64, 128, 1}.
+// a6: per-shard SDPA.  qkv map: 3-D fp16 {3*Hs*128, M, T}, box {64, 128, 1}.
 // ----------------------------------------------------------------------------
 struct AttnArgs {
   int M;            // tokens
@@ -63,8 +64,13 @@ struct AttnArgs {
 
 cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s);
 
+// Counts kernel launches (api.cu); every launcher calls it once per launch.
+void count_launch();
+
 // Host helpers (api.cu).
 CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                           uint32_t box0, uint32_t box1);
+CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                         uint32_t box1);
 
 }  // namespace tp

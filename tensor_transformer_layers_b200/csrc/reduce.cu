@@ -74,6 +74,7 @@ cudaError_t launch_reduce_partials(const float* parts, int64_t M, int64_t N, int
   reduce_partials_kernel<<<unsigned(blocks), kThreads, 0, s>>>(reinterpret_cast<const float4*>(parts), bias,
                                                                reinterpret_cast<uint4*>(Y), n8_total,
                                                                uint32_t(N / 8), M * N / 4, T);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -70,6 +70,7 @@ cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblock
     slice_copy_kernel<<<grid, kThreads, 0, st>>>(reinterpret_cast<const uint4*>(src + r0 * src_ld),
                                                  reinterpret_cast<uint4*>(dst + r0 * cols), uint32_t(nr),
                                                  uint32_t(c8), src_ld / 8, src_bstride / 8, dst_bstride / 8);
+    count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

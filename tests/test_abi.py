@@ -101,7 +101,8 @@ def test_layer_checks():
     assert tp.tp_attn_block(A, 64, 768, A, A, 6, 2, A, A, 10, stream=0) == S["TP_ERR_WORKSPACE"]
     assert tp.tp_attn_block(A, 0, 768, A, A, 6, 2, A, None, 0, stream=0) == 0
     # step-level calls
-    assert tp.tp_colwise_linear(A, 64, 100, A, None, 64, 2, 1, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_colwise_linear(A, 64, 100, A, None, 64, 2, 1, 0, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_colwise_linear(A, 64, 128, A, None, 64, 2, 1, 7, A, stream=0) == S["TP_ERR_BAD_STYLE"]
     assert tp.tp_rowwise_linear_sum(A, 64, 64, A, 100, None, 2, A, stream=0) == S["TP_ERR_ALIGNMENT"]
     assert tp.tp_sdpa_shards(A, 64, 6, 4, A, stream=0) == S["TP_ERR_HEADS_INDIVISIBLE"]
     assert tp.tp_reduce_partials(A, 64, 100, 2, None, A, stream=0) == S["TP_ERR_ALIGNMENT"]

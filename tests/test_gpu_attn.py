@@ -7,7 +7,7 @@ import torch
 import oracle as o
 import synthetic as syn
 import tensor_transformer_layers_b200 as tp
-from tests._util import assert_parity, f64, from_dev, to_dev
+from tests._util import assert_parity, assert_rounded_once, f64, from_dev, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -15,35 +15,34 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("M,Hs,T", [(1, 1, 1), (128, 1, 1), (200, 2, 2), (256, 1, 3), (1000, 2, 1), (4608, 1, 1)])
 def test_sdpa_step(M, Hs, T):
     W = 3 * Hs * 128
-    # Q, K, V of unit variance, like the projections of a unit-variance input
-    QKV = syn.normal_bf16((T, M, W), 1.0, seed=M + Hs, tid=400)
+    # Q, K, V of unit variance, like the projections of a unit-variance input (fp16 storage)
+    QKV = syn.normal_f16((T, M, W), 1.0, seed=M + Hs, tid=400)
     O = torch.empty((T, M, Hs * 128), dtype=torch.int16, device="cuda")
     assert tp.tp_sdpa_shards(to_dev(QKV), M, Hs * T, T, O) == 0
     torch.cuda.synchronize()
     g = from_dev(O)
-    q = f64(QKV)
+    q = syn.f16_bits_to_f64(QKV)
     for r in range(T):
         for j in range(Hs):
             Q = q[r][:, j * 128:(j + 1) * 128]
             K = q[r][:, (Hs + j) * 128:(Hs + j + 1) * 128]
             V = q[r][:, (2 * Hs + j) * 128:(2 * Hs + j + 1) * 128]
-            assert_parity(g[r][:, j * 128:(j + 1) * 128], o.sdpa(Q, K, V), f"sdpa r={r} j={j}")
+            assert_rounded_once(g[r][:, j * 128:(j + 1) * 128], o.sdpa(Q, K, V), f"sdpa r={r} j={j}")
 
 
 def test_sdpa_large_scores_rescale_path():
     # Scores spread over a wide range force the running-max rescale of O.
     M, Hs, T = 512, 1, 1
-    QKV = syn.normal_bf16((T, M, 3 * 128), 1.0, seed=7, tid=401)
-    q = f64(QKV)
-    # scale Q up so that maxima grow along the key sequence
-    Qs = syn.f64_to_bf16_bits(q[0][:, :128] * 6.0)
-    QKV[0][:, :128] = Qs
-    q = f64(QKV)
+    QKV = syn.normal_f16((T, M, 3 * 128), 1.0, seed=7, tid=401)
+    q = syn.f16_bits_to_f64(QKV)
+    # scale Q up (exact in fp16: a power of two) so that maxima grow along the key sequence
+    QKV[0][:, :128] = (q[0][:, :128] * 8.0).astype(np.float16).view(np.uint16)
+    q = syn.f16_bits_to_f64(QKV)
     O = torch.empty((T, M, 128), dtype=torch.int16, device="cuda")
     assert tp.tp_sdpa_shards(to_dev(QKV), M, 1, 1, O) == 0
     torch.cuda.synchronize()
     ref = o.sdpa(q[0][:, :128], q[0][:, 128:256], q[0][:, 256:])
-    assert_parity(from_dev(O)[0], ref, "sdpa wide scores")
+    assert_rounded_once(from_dev(O)[0], ref, "sdpa wide scores")
 
 
 @pytest.mark.parametrize("M,heads,T", [(200, 4, 2), (64, 2, 1), (333, 4, 4)])

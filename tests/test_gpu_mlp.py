@@ -108,3 +108,31 @@ def test_empty_input_writes_nothing(tiny):
     torch.cuda.synchronize()
     assert np.all(from_dev(Y) == 0x3C3C)
     assert tp.tp_check_device_error() == 0
+
+
+def test_bench_step_sequence_matches_one_shot(flux):
+    # bench.py times the five calls that tp_mlp_pair makes, one by one; they must
+    # produce exactly the one-shot result.
+    c, d, _ = flux
+    M, D, F, T = c["M"], c["D"], c["F"], c["T"]
+    Fs = F // T
+    dd = _dev(d)
+    w_up = torch.empty((T, Fs, D), dtype=torch.int16, device="cuda")
+    b_up = torch.empty((T, Fs), dtype=torch.int16, device="cuda")
+    w_down = torch.empty((T, D, Fs), dtype=torch.int16, device="cuda")
+    H = torch.empty((T, M, Fs), dtype=torch.int16, device="cuda")
+    Y = torch.empty((M, D), dtype=torch.int16, device="cuda")
+    n0 = tp.tp_kernel_launches()
+    assert tp.tp_shard_weight_all(dd["W_up"], F, D, tp.TP_COLWISE, T, w_up) == 0
+    assert tp.tp_shard_weight_all(dd["b_up"], T, Fs, tp.TP_COLWISE, T, b_up) == 0
+    assert tp.tp_shard_weight_all(dd["W_down"], D, F, tp.TP_ROWWISE, T, w_down) == 0
+    assert tp.tp_colwise_linear(dd["X"], M, D, w_up, b_up, Fs, T, 1, tp.TP_OUT_BF16, H) == 0
+    assert tp.tp_rowwise_linear_sum(H, M, Fs, w_down, D, dd["b_down"], T, Y) == 0
+    assert tp.tp_kernel_launches() - n0 == 5
+    torch.cuda.synchronize()
+    one = _run_pair(dd, M, D, F, T)
+    assert np.array_equal(from_dev(Y), one)
+    # the stacked shards are the oracle's slices
+    for r in (0, T - 1):
+        assert np.array_equal(from_dev(w_up[r]), o.slice_colwise(d["W_up"], T, r))
+        assert np.array_equal(from_dev(w_down[r]), o.slice_rowwise(d["W_down"], T, r))
