@@ -275,9 +275,11 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
 
 
 def block_rows(X, W_qkv, W_o, heads, W_up, b_up, W_down, b_down, rows, tp_degree=1, round_between=True):
-    """Composed block at selected token rows.  The attention output A is a bf16 tensor
-    handed to the MLP, so it is rounded to bf16 in between (``round_between``)."""
+    """Composed block at selected token rows; returns (A, Y).
+
+    A is the attention layer's output (exact, to compare with that layer's
+    result).  The tensor handed from the attention layer to the MLP pair is a
+    bf16 tensor, so the MLP's input is A rounded to bf16 (``round_between``)."""
     A = attn_rows(X, W_qkv, W_o, heads, rows, tp_degree)
-    if round_between:
-        A = round_bf16(A)
-    return A, mlp_sharded_summed(A, W_up, b_up, W_down, b_down, tp_degree)
+    A_in = round_bf16(A) if round_between else A
+    return A, mlp_sharded_summed(A_in, W_up, b_up, W_down, b_down, tp_degree)

@@ -434,3 +434,16 @@ def test_bf16_encoding():
     bits = syn._f32_to_bf16_bits(v)
     assert list(bits) == [0x3F80, 0xC000, 0x0000, 0x3F80, 0x3F82]
     assert np.array_equal(syn.bf16_bits_to_f64(bits), np.array([1.0, -2.0, 0.0, 1.0, 1.0 + 2 ** -6]))
+
+
+def test_block_rows_returns_exact_attention_and_mlp_of_rounded_input():
+    heads, M, D, F = 2, 12, 256, 512
+    d = syn.block_inputs(M, D, F, seed=21)
+    f = {k: syn.bf16_bits_to_f64(v) for k, v in d.items()}
+    rows = [0, 5, 11]
+    A, Y = o.block_rows(f["X"], f["W_qkv"], f["W_o"], heads, f["W_up"], f["b_up"], f["W_down"], f["b_down"],
+                        rows, tp_degree=2)
+    A_full = o.attn_unsharded(f["X"], f["W_qkv"], f["W_o"], heads)
+    assert np.allclose(A, A_full[rows], atol=1e-12)
+    Y_want = o.mlp_unsharded(o.round_bf16(A_full[rows]), f["W_up"], f["b_up"], f["W_down"], f["b_down"])
+    assert np.allclose(Y, Y_want, atol=1e-12)
