@@ -37,7 +37,7 @@ if ROOT not in sys.path:
 METRIC = "TP layer-pair bf16 TFLOP/s and % of dense-BF16 tensor peak on 1 B200"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FLUSH_BYTES = 256 << 20  # > 126 MB L2
+L2_BYTES = 126 << 20
 
 
 # --------------------------------------------------------------------------- distributed helpers
@@ -258,7 +258,8 @@ def config_dict(cfg, world):
                          f"cross-shard sum fused), all tp_degree shards on one GPU; M={cfg['M']} tokens "
                          f"(4096 image + 512 text), D={cfg['D']}, F={cfg['F']}"),
             "M": cfg["M"], "D": cfg["D"], "F": cfg["F"], "tp_degree": cfg["T"], "global_batch_tokens": cfg["M"] * world,
-            "l2": "flushed before every step (256 MiB write, outside the step's events)",
+            "l2": ("not flushed: inputs larger than L2 (each step reads 179 MB of inputs, > 126 MB L2, "
+                   "and moves about 0.6 GB in total)"),
             "parallelism": "single GPU" if world == 1 else f"{world} independent replicas (one per GPU)"}
 
 
@@ -281,7 +282,8 @@ def run_ours(args, cfg, rank, local_rank, world):
     w_down = torch.empty((T, D, Fs), dtype=torch.int16, device=dev)
     H = torch.empty((T, M, Fs), dtype=torch.int16, device=dev)
     Y = torch.empty((M, D), dtype=torch.int16, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    input_bytes = sum(v.numel() * v.element_size() for v in g.values())
+    assert input_bytes > L2_BYTES, "the step's inputs must exceed L2 (no flush between steps)"
     check = tp._check
 
     names = ["slice_w_up", "slice_b_up", "slice_w_down", "colwise_gemm", "rowwise_gemm"]
@@ -303,7 +305,6 @@ def run_ours(args, cfg, rank, local_rank, world):
         return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
 
     for _ in range(args.warmup):
-        flush.zero_()
         step(new_events())
     torch.cuda.synchronize()
 
@@ -315,7 +316,6 @@ def run_ours(args, cfg, rank, local_rank, world):
     sampler.start()
     t_wall0 = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()
         step(evs[i])
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall0
