@@ -63,7 +63,8 @@ typedef enum {
   TP_ERR_CUDA = 9,               /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
   TP_ERR_DEVICE_TIMEOUT = 10,    /* a kernel's bounded wait ran out (see tp_check_device_error) */
   TP_ERR_BAD_STYLE = 11,         /* unknown tp_style */
-  TP_ERR_BAD_HANDLE = 12         /* NULL or foreign handle */
+  TP_ERR_BAD_HANDLE = 12,        /* NULL or foreign handle */
+  TP_ERR_SCRATCH_LIMIT = 13      /* problem too large for the no-allocation entry point's fixed scratch */
 } tp_status;
 
 typedef enum {
@@ -213,6 +214,39 @@ tp_status tp_attn_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y,
 
 /* Frees a handle from tp_*_prepare (synchronises the device first). NULL is a no-op. */
 void tp_destroy(void* handle);
+
+/* ---------------------------------------------------------------------------
+ * Allocation-free MLP pair.  The paper has no counterpart: this entry point
+ * exists for callers that must not allocate device memory themselves or
+ * through the library, e.g. code whose device memory is owned by another
+ * allocator (a raw cudaMalloc would bypass its accounting and can fail when
+ * that allocator holds most of the device), or code that cannot accept the
+ * device-wide synchronisation cudaMalloc/cudaFree may cause.
+ *
+ * Same result as tp_mlp_pair on already-sharded weights (what each rank holds
+ * after sharded loading; tp_shard_weight_all produces them into caller
+ * memory without allocating):
+ *   W_up_shards [T x F/T x D], b_up_shards [T x F/T] or NULL,
+ *   W_down_shards [T x D x F/T], b_down [D] or NULL, X [M x D], Y [M x D].
+ * The hidden activations live in a file-scope device array of
+ * TP_NOALLOC_SCRATCH_BYTES (64 MiB) that every GPU loading the library holds
+ * until the process exits.  Tokens are processed in chunks of
+ * floor(64 MiB / (2*F)) rows rounded down to a multiple of 128; if even 128
+ * rows do not fit (F > 262144) the call returns TP_ERR_SCRATCH_LIMIT before
+ * launching anything.  Other checks as tp_mlp_pair.
+ * The first call on a device looks up the array's device address (once per
+ * device); make that first call before any stream capture.  Every call shares
+ * the one array: calls that overlap on the GPU (different streams, or
+ * different host threads on one device) race and corrupt each other's
+ * results.  Nothing in the array has to start at zero: a chunk's activations
+ * are written in full before they are read, and reads past a chunk's rows
+ * come from the TMA unit's out-of-bounds zero fill, never from the array.
+ * Calls no cudaMalloc, cudaFree or other allocating routine. */
+#define TP_NOALLOC_SCRATCH_BYTES (64ull << 20)
+tp_status tp_mlp_pair_sharded_noalloc(const uint16_t* X, int64_t M, int64_t D, int64_t F,
+                                      const uint16_t* W_up_shards, const uint16_t* b_up_shards,
+                                      const uint16_t* W_down_shards, const uint16_t* b_down,
+                                      int tp_degree, uint16_t* Y, void* stream);
 
 #ifdef __cplusplus
 }

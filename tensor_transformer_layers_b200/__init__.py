@@ -30,6 +30,7 @@ STATUS = {
     4: "TP_ERR_INDIVISIBLE", 5: "TP_ERR_HEADS_INDIVISIBLE", 6: "TP_ERR_BAD_SHAPE",
     7: "TP_ERR_ALIGNMENT", 8: "TP_ERR_WORKSPACE", 9: "TP_ERR_CUDA",
     10: "TP_ERR_DEVICE_TIMEOUT", 11: "TP_ERR_BAD_STYLE", 12: "TP_ERR_BAD_HANDLE",
+    13: "TP_ERR_SCRATCH_LIMIT",
 }
 
 _P = ctypes.c_void_p
@@ -62,6 +63,7 @@ SIGNATURES = {
     "tp_attn_run_workspace_bytes": (_SZ, [_I64, _I64, _I, _I]),
     "tp_attn_run": (_I, [_P, _P, _I64, _P, _P, _SZ, _P]),
     "tp_destroy": (None, [_P]),
+    "tp_mlp_pair_sharded_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _P]),
 }
 
 _lib = None
@@ -211,6 +213,15 @@ def tp_attn_run(handle, X, M, Y, ws, ws_bytes, stream=None) -> int:
 
 def tp_destroy(handle) -> None:
     lib().tp_destroy(handle)
+
+
+def tp_mlp_pair_sharded_noalloc(X, M, D, F, W_up_shards, b_up_shards, W_down_shards, b_down, tp_degree, Y,
+                                stream=None) -> int:
+    """The MLP pair on pre-sharded weights with no device allocation (fixed
+    64 MiB library scratch); see include/tp.h."""
+    return lib().tp_mlp_pair_sharded_noalloc(_ptr(X), M, D, F, _ptr(W_up_shards), _ptr(b_up_shards),
+                                             _ptr(W_down_shards), _ptr(b_down), tp_degree, _ptr(Y),
+                                             _stream(stream))
 
 
 # --------------------------------------------------------------------------- convenience

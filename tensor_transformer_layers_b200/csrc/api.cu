@@ -78,6 +78,15 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int current_device_context(int* num_sms, int** err) {
+  DeviceInfo* di = nullptr;
+  const tp_status st = device_info(&di);
+  if (st != TP_OK) return st;
+  *num_sms = di->num_sms;
+  *err = di->err;
+  return TP_OK;
+}
+
 static CUresult make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
                             uint64_t d2, uint32_t box0, uint32_t box1) {
   const cuuint64_t dims[3] = {d0, d1, d2};
@@ -323,6 +332,8 @@ const char* tp_status_string(int s) {
     case TP_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait timed out";
     case TP_ERR_BAD_STYLE: return "unknown sharding style";
     case TP_ERR_BAD_HANDLE: return "invalid handle";
+    case TP_ERR_SCRATCH_LIMIT:
+      return "size exceeds the 64 MiB static scratch of tp_mlp_pair_sharded_noalloc (F * 256 bytes must fit)";
     default: return "unknown status";
   }
 }

@@ -67,6 +67,11 @@ cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cuda
 // Counts kernel launches (api.cu); every launcher calls it once per launch.
 void count_launch();
 
+// SM count and device error word of the current device, initialising the
+// library's per-device state (tensor-map encoder included) on first use.
+// Returns a tp_status value.
+int current_device_context(int* num_sms, int** err);
+
 // Host helpers (api.cu).
 CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                           uint32_t box0, uint32_t box1);
