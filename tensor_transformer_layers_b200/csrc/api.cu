@@ -117,9 +117,8 @@ namespace {
 tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, const uint16_t* b,
                       int64_t Ns, int T, int gelu, int out_f16, uint16_t* out, cudaStream_t s) {
   if (M == 0) return TP_OK;
-  CUtensorMap amap, bmap;
-  if (make_map_3d_bf16(&amap, X, uint64_t(K), uint64_t(M), 1, 64, 128) != CUDA_SUCCESS) return TP_ERR_CUDA;
-  if (make_map_3d_bf16(&bmap, W, uint64_t(K), uint64_t(Ns), uint64_t(T), 64, 256) != CUDA_SUCCESS) return TP_ERR_CUDA;
+  const GemmOperand A{X, uint64_t(K), uint64_t(M), 1};
+  const GemmOperand B{W, uint64_t(K), uint64_t(Ns), uint64_t(T)};
   GemmArgs a;
   a.M = int(M);
   a.N = int(Ns);
@@ -135,16 +134,15 @@ tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, c
   a.gelu = gelu;
   a.out_f16 = out_f16;
   a.err = di->err;
-  return launch_gemm(amap, bmap, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return launch_gemm(A, B, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 // rowwise: Y = sum_r A[r] . W[r]^T + bias.
 tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, const uint16_t* W, int64_t N,
                       const uint16_t* bias, int T, uint16_t* Y, cudaStream_t s) {
   if (M == 0) return TP_OK;
-  CUtensorMap amap, bmap;
-  if (make_map_3d_bf16(&amap, A, uint64_t(Ks), uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS) return TP_ERR_CUDA;
-  if (make_map_3d_bf16(&bmap, W, uint64_t(Ks), uint64_t(N), uint64_t(T), 64, 256) != CUDA_SUCCESS) return TP_ERR_CUDA;
+  const GemmOperand Aop{A, uint64_t(Ks), uint64_t(M), uint64_t(T)};
+  const GemmOperand Bop{W, uint64_t(Ks), uint64_t(N), uint64_t(T)};
   GemmArgs a;
   a.M = int(M);
   a.N = int(N);
@@ -160,7 +158,7 @@ tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, 
   a.gelu = 0;
   a.out_f16 = 0;
   a.err = di->err;
-  return launch_gemm(amap, bmap, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return launch_gemm(Aop, Bop, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 tp_status run_sdpa(DeviceInfo* di, const uint16_t* QKV, int64_t M, int heads, int T, uint16_t* O, cudaStream_t s) {

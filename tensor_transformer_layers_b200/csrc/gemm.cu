@@ -2,8 +2,8 @@
 // 5th-generation tensor cores (tcgen05), fed by TMA, accumulating in tensor
 // memory (TMEM).
 //
-// One kernel serves both styles of the Diffusers "Tensor parallelism" page
-// (section "Colwise and rowwise", style table):
+// One kernel family serves both styles of the Diffusers "Tensor parallelism"
+// page (section "Colwise and rowwise", style table):
 //   colwise  out_r = epi(X . W_r^T + b_r) for every shard r: the tile's K loop
 //            covers the shared input X against shard r's weight rows;
 //   rowwise  Y = sum_r A_r . W_r^T + b: the tile's K loop walks every shard's
@@ -11,22 +11,29 @@
 //            block-boundary AllReduce performs happens inside the accumulator
 //            and the bias is added once in the epilogue.
 //
-// Structure (one CTA per SM, persistent over output tiles, 192 threads):
-//   warp 0   TMA producer: 128x64 A tile + 256x64 B tile per stage, 128-byte
-//            swizzle, 4-stage ring of full/empty mbarriers.
-//   warp 1   TMEM allocator + MMA issuer: one thread issues 4 x
-//            tcgen05.mma (M=128, N=256, K=16) per stage, commits the stage
-//            back to the producer, and commits a finished accumulator to the
-//            epilogue.  Two 256-column fp32 accumulators (all 512 TMEM
-//            columns) let tile i+1's MMAs run while tile i drains.
-//   warps 2-5 epilogue: tcgen05.ld 32 columns at a time (thread = output
-//            row), bias, optional tanh-form GELU, rounding to bf16 (or fp16
-//            for the Q/K/V projection that feeds attention), 16-byte global
-//            stores; then release the accumulator.
+// Two kernels, same roles (192 threads, persistent over output tiles):
+//   warp 0    TMA producer (128-byte swizzle, ring of full/empty mbarriers);
+//   warp 1    TMEM allocator + single-thread MMA issuer; two 256-column fp32
+//             accumulators (all 512 TMEM columns) so tile i's epilogue runs
+//             while tile i+1's MMAs do;
+//   warps 2-5 epilogue: tcgen05.ld 32 columns at a time (thread = output row),
+//             bias, optional tanh-form GELU, rounding to bf16 (or fp16 for the
+//             Q/K/V that feed attention), 16-byte global stores.
+// * gemm_tc_kernel: one CTA per SM, 128x256 tile, M=128 N=256 K=16 MMAs,
+//   4 stages of 48 KB (A 128x64 + B 256x64).  Used for M < 256.
+// * gemm_pair_kernel: CTA pairs (cluster of 2, tcgen05 cta_group::2), 256x256
+//   tile per pair.  Each CTA loads its 128 rows of A and its 128 rows of B
+//   (32 KB per k-block instead of 48 KB: the B tile is split between the two
+//   SMs), so the shared-memory fill per MMA cycle drops by a third and 6
+//   stages fit.  The even CTA issues M=256 N=256 K=16 MMAs over both CTAs'
+//   shared memory; each CTA's TMEM holds its 128 accumulator rows.  No TMA
+//   multicast: each CTA fetches its own tiles.
 // Every mbarrier wait is bounded (see ptx.cuh): a wait that runs out sets the
 // device error word, the CTA's roles stop, in-flight copies and MMAs are
 // drained with bounded waits, TMEM is freed and the kernel returns.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -34,22 +41,31 @@
 namespace tp {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 64;  // 64 bf16 = one 128-byte swizzle row
-constexpr int kStages = 4;
-constexpr int kABytes = BM * BK * 2;
-constexpr int kBBytes = BN * BK * 2;
-constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kAccCols = BN;      // fp32 TMEM columns per accumulator
-constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kThreads = 192;
-constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + 1 KB alignment slack
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN, false);
+constexpr int kAccCols = 256;  // fp32 TMEM columns per accumulator (N = 256)
+constexpr int kTmemCols = 2 * kAccCols;
+
+// single-CTA kernel
+constexpr int BM1 = 128, BN1 = 256;
+constexpr int kStages1 = 4;
+constexpr int kABytes1 = BM1 * BK * 2;
+constexpr int kStageBytes1 = kABytes1 + BN1 * BK * 2;
+constexpr int kBarOff1 = kStages1 * kStageBytes1;
+constexpr int kSmemBytes1 = kBarOff1 + 256 + 1024;  // + barriers + 1 KB alignment slack
+constexpr uint32_t kIdesc1 = idesc_bf16_f32(BM1, BN1, false);
+
+// CTA-pair kernel (per CTA: 128 rows of A and 128 rows of B per stage)
+constexpr int BM2 = 256, BN2 = 256;
+constexpr int kStages2 = 6;
+constexpr int kHalfBytes = 128 * BK * 2;
+constexpr int kStageBytes2 = 2 * kHalfBytes;
+constexpr int kBarOff2 = kStages2 * kStageBytes2;
+constexpr int kSmemBytes2 = kBarOff2 + 512 + 1024;
+constexpr uint32_t kIdesc2 = idesc_bf16_f32(BM2, BN2, false);
 
 static_assert(kTmemCols == 512, "two 256-column accumulators fill TMEM");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert(kSmemBytes1 <= 227 * 1024 && kSmemBytes2 <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ float gelu_tanh(float x) {
   // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))  (Hendrycks & Gimpel, 2016)
@@ -71,14 +87,80 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int m_tiles, int n_tiles
   return c;
 }
 
+// Drains one 128-row x 256-column fp32 accumulator (this warp's 32 lanes) to
+// global memory: bias, GELU, rounding, masked 16-byte stores.
+__device__ __forceinline__ void epilogue_rows(const GemmArgs& p, uint32_t taddr, int row, int g, int col_base) {
+  uint16_t* orow = p.out + int64_t(g) * p.out_gstride + int64_t(row) * p.ldo;
+  const uint16_t* bias = p.bias ? p.bias + int64_t(g) * p.bias_gstride : nullptr;
+  const int n_left = p.N - col_base;
+  const int chunks = n_left >= kAccCols ? kAccCols / 32 : (n_left + 31) / 32;  // warp-uniform
+  for (int c = 0; c < chunks; ++c) {
+    uint32_t r[32];
+    __syncwarp();
+    tmem_ld32_sync(taddr + uint32_t(c * 32), r);
+    const int col0 = col_base + c * 32;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    if (bias != nullptr) {
+      const uint4* bp = reinterpret_cast<const uint4*>(bias + col0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (col0 + 8 * j < p.N) {
+          const uint4 b = __ldg(bp + j);
+          v[8 * j + 0] += bf16_lo(b.x);
+          v[8 * j + 1] += bf16_hi(b.x);
+          v[8 * j + 2] += bf16_lo(b.y);
+          v[8 * j + 3] += bf16_hi(b.y);
+          v[8 * j + 4] += bf16_lo(b.z);
+          v[8 * j + 5] += bf16_hi(b.z);
+          v[8 * j + 6] += bf16_lo(b.w);
+          v[8 * j + 7] += bf16_hi(b.w);
+        }
+      }
+    }
+    if (p.gelu) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+    }
+    uint4 o[4];
+    if (p.out_f16) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        o[j].x = pack_f16x2(v[8 * j + 0], v[8 * j + 1]);
+        o[j].y = pack_f16x2(v[8 * j + 2], v[8 * j + 3]);
+        o[j].z = pack_f16x2(v[8 * j + 4], v[8 * j + 5]);
+        o[j].w = pack_f16x2(v[8 * j + 6], v[8 * j + 7]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        o[j].x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+        o[j].y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+        o[j].z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+        o[j].w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+      }
+    }
+    if (row < p.M) {
+      uint4* op = reinterpret_cast<uint4*>(orow + col0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (col0 + 8 * j < p.N) op[j] = o[j];
+    }
+  }
+}
+
+// ============================================================================
+// Single-CTA kernel
+// ============================================================================
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                    const GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff1);
+  uint64_t* empty = full + kStages1;
+  uint64_t* tfull = empty + kStages1;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
@@ -86,13 +168,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_tiles = (p.M + BM - 1) / BM;
-  const int n_tiles = (p.N + BN - 1) / BN;
+  const int m_tiles = (p.M + BM1 - 1) / BM1;
+  const int n_tiles = (p.N + BN1 - 1) / BN1;
   const int tiles = m_tiles * n_tiles * p.groups;
   const int k_iters = p.k_blocks * p.kshards;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStages1; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -133,12 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int s = it / p.k_blocks;
           const int kb = it - s * p.k_blocks;
-          uint8_t* sa = smem + stage * kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          tma_load_3d(sa, &amap, &full[stage], kb * BK, tc.mb * BM, p.a_follows_shard ? s : 0);
-          tma_load_3d(sa + kABytes, &bmap, &full[stage], kb * BK, tc.nb * BN, tc.g + s);
+          uint8_t* sa = smem + stage * kStageBytes1;
+          mbar_arrive_expect_tx(&full[stage], kStageBytes1);
+          tma_load_3d(sa, &amap, &full[stage], kb * BK, tc.mb * BM1, p.a_follows_shard ? s : 0);
+          tma_load_3d(sa + kABytes1, &bmap, &full[stage], kb * BK, tc.nb * BN1, tc.g + s);
           ++issued;
-          if (++stage == kStages) {
+          if (++stage == kStages1) {
             stage = 0;
             phase ^= 1u;
           }
@@ -149,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Let every issued copy land before the CTA's shared memory goes away.
         // Stage s was last armed in the current phase if s < stage, else in the previous one.
         const volatile int no_abort = 0;
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStages1; ++s) {
           if (issued <= s) break;
           mbar_wait(&full[s], s < stage ? phase : (phase ^ 1u), &no_abort);
         }
@@ -176,14 +258,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+          const uint32_t sa = smem_u32(smem + stage * kStageBytes1);
           const uint64_t da = sdesc_sw128(sa, 16, 1024);
-          const uint64_t db = sdesc_sw128(sa + kABytes, 16, 1024);
+          const uint64_t db = sdesc_sw128(sa + kABytes1, 16, 1024);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)  // advance 16 bf16 = 32 bytes inside the swizzle row
-            umma_ss(d_tmem, da + uint64_t(2 * k), db + uint64_t(2 * k), kIdesc, (it | k) != 0 ? 1u : 0u);
+            umma_ss(d_tmem, da + uint64_t(2 * k), db + uint64_t(2 * k), kIdesc1, (it | k) != 0 ? 1u : 0u);
           umma_commit(&empty[stage]);
-          if (++stage == kStages) {
+          if (++stage == kStages1) {
             stage = 0;
             phase ^= 1u;
           }
@@ -212,67 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int row = tc.mb * BM + q * 32 + lane;
-      const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
-      uint16_t* orow = p.out + int64_t(tc.g) * p.out_gstride + int64_t(row) * p.ldo;
-      const uint16_t* bias = p.bias ? p.bias + int64_t(tc.g) * p.bias_gstride : nullptr;
-      const int col_base = tc.nb * BN;
-      const int n_left = p.N - col_base;
-      const int chunks = n_left >= BN ? BN / 32 : (n_left + 31) / 32;  // warp-uniform
-      for (int c = 0; c < chunks; ++c) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32_sync(taddr + uint32_t(c * 32), r);
-        const int col0 = col_base + c * 32;
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (bias != nullptr) {
-          const uint4* bp = reinterpret_cast<const uint4*>(bias + col0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (col0 + 8 * j < p.N) {
-              const uint4 b = __ldg(bp + j);
-              v[8 * j + 0] += bf16_lo(b.x);
-              v[8 * j + 1] += bf16_hi(b.x);
-              v[8 * j + 2] += bf16_lo(b.y);
-              v[8 * j + 3] += bf16_hi(b.y);
-              v[8 * j + 4] += bf16_lo(b.z);
-              v[8 * j + 5] += bf16_hi(b.z);
-              v[8 * j + 6] += bf16_lo(b.w);
-              v[8 * j + 7] += bf16_hi(b.w);
-            }
-          }
-        }
-        if (p.gelu) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
-        }
-        uint4 o[4];
-        if (p.out_f16) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            o[j].x = pack_f16x2(v[8 * j + 0], v[8 * j + 1]);
-            o[j].y = pack_f16x2(v[8 * j + 2], v[8 * j + 3]);
-            o[j].z = pack_f16x2(v[8 * j + 4], v[8 * j + 5]);
-            o[j].w = pack_f16x2(v[8 * j + 6], v[8 * j + 7]);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            o[j].x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-            o[j].y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-            o[j].z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-            o[j].w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-          }
-        }
-        if (row < p.M) {
-          uint4* op = reinterpret_cast<uint4*>(orow + col0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (col0 + 8 * j < p.N) op[j] = o[j];
-        }
-      }
+      epilogue_rows(p, tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols), tc.mb * BM1 + q * 32 + lane,
+                    tc.g, tc.nb * BN1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -289,18 +312,254 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ============================================================================
+// CTA-pair kernel (cluster of 2, tcgen05 cta_group::2)
+// ============================================================================
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                     const GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff2);  // the leader's copy is the one used
+  uint64_t* empty = full + kStages2;                               // both CTAs' copies used
+  uint64_t* tfull = empty + kStages2;                              // both
+  uint64_t* tempty = tfull + 2;                                    // the leader's copy used
+  uint64_t* drain = tempty + 2;
+  uint64_t* exit_bar = drain + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(exit_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader, 1 = peer
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int m_tiles = (p.M + BM2 - 1) / BM2;
+  const int n_tiles = (p.N + BN2 - 1) / BN2;
+  const int tiles = m_tiles * n_tiles * p.groups;
+  const int k_iters = p.k_blocks * p.kshards;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&full[s], 1);   // the leader's producer arrives (+ both CTAs' TMA bytes)
+      mbar_init(&empty[s], 1);  // one multicast commit per use
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);   // one multicast commit per use
+      mbar_init(&tempty[a], 8);  // four epilogue warps in each CTA
+    }
+    mbar_init(drain, 1);
+    mbar_init(exit_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&bmap);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised before any cross-CTA use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int64_t issued = 0;
+      for (int t = pair; t < tiles && ok; t += n_pairs) {
+        const TileCoord tc = decode_tile(t, m_tiles, n_tiles);
+        for (int it = 0; it < k_iters; ++it) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int s = it / p.k_blocks;
+          const int kb = it - s * p.k_blocks;
+          uint8_t* sa = smem + stage * kStageBytes2;
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes2);  // both CTAs' bytes
+          tma_load_3d_pair(sa, &amap, fb, kb * BK, tc.mb * BM2 + int(rank) * 128, p.a_follows_shard ? s : 0);
+          tma_load_3d_pair(sa + kHalfBytes, &bmap, fb, kb * BK, tc.nb * BN2 + int(rank) * 128, tc.g + s);
+          ++issued;
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) report_timeout(p.err, abort_flag);
+      // Tail: every stage this CTA filled must be released (the MMAs reading it
+      // done and the commit arrived here) before the CTA may exit.  Bounded.
+      const volatile int no_abort = 0;
+      for (int s = 0; s < kStages2; ++s) {
+        if (issued <= s) break;
+        // stage s was last filled in the current round if s < stage, else in the previous one
+        mbar_wait(&empty[s], s < stage ? phase : (phase ^ 1u), ok ? abort_flag : &no_abort);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = pair; t < tiles && ok; t += n_pairs, ++local) {
+        const int acc = local & 1;
+        if (!mbar_wait(&tempty[acc], ((local >> 1) & 1) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(acc * kAccCols);
+        for (int it = 0; it < k_iters; ++it) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * kStageBytes2);
+          const uint64_t da = sdesc_sw128(sa, 16, 1024);
+          const uint64_t db = sdesc_sw128(sa + kHalfBytes, 16, 1024);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_ss_pair(d_tmem, da + uint64_t(2 * k), db + uint64_t(2 * k), kIdesc2, (it | k) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(&tfull[acc], 0x3);
+      }
+      const volatile int no_abort = 0;
+      if (!ok) {
+        report_timeout(p.err, abort_flag);
+        umma_commit_pair_mc(drain, 0x1);
+        mbar_wait(drain, 0, &no_abort);
+      } else {
+        // Tail: both CTAs' epilogues have released the last accumulators (their
+        // arrivals, some remote, have landed here) before the leader may exit.
+        for (int i = local - 2 < 0 ? 0 : local - 2; i < local; ++i)
+          mbar_wait(&tempty[i & 1], (i >> 1) & 1, abort_flag);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    int local = 0;
+    bool ok = true;
+    for (int t = pair; t < tiles; t += n_pairs, ++local) {
+      const TileCoord tc = decode_tile(t, m_tiles, n_tiles);
+      const int acc = local & 1;
+      if (!mbar_wait(&tfull[acc], (local >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      epilogue_rows(p, tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols),
+                    tc.mb * BM2 + int(rank) * 128 + q * 32 + lane, tc.g, tc.nb * BN2);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader + uint32_t(acc * sizeof(uint64_t)));
+    }
+    if (!ok && lane == 0) report_timeout(p.err, abort_flag);
+  }
+
+  // Exit handshake: neither CTA leaves while the other may still signal its
+  // barriers.  Bounded like every other wait.
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_cluster(mapa_shared(smem_u32(exit_bar), rank ^ 1u));
+    const volatile int no_abort = 0;
+    if (!mbar_wait(exit_bar, 0, &no_abort)) report_timeout(p.err, abort_flag);
+  }
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+int g_max_pairs[64] = {};
+std::mutex g_pairs_mu;
+
+int max_active_pairs(int num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
+  std::lock_guard<std::mutex> lock(g_pairs_mu);
+  if (g_max_pairs[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(num_sms & ~1));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes2;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel, &cfg) != cudaSuccess || n <= 0) n = num_sms / 2;
+    g_max_pairs[dev] = n;
+  }
+  return g_max_pairs[dev];
+}
+
 }  // namespace
 
-cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmArgs& a, int num_sms,
+cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms,
                         cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.groups <= 0) return cudaSuccess;
-  const int m_tiles = (a.M + BM - 1) / BM;
-  const int n_tiles = (a.N + BN - 1) / BN;
+  CUtensorMap amap, bmap;
+  if (a.M >= BM2) {
+    // CTA-pair kernel: each CTA loads 128-row halves of both operands.
+    if (make_map_3d_bf16(&amap, A.base, A.k, A.rows, A.z, BK, 128) != CUDA_SUCCESS ||
+        make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, 128) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = int64_t((a.M + BM2 - 1) / BM2) * ((a.N + BN2 - 1) / BN2) * a.groups;
+    int pairs = max_active_pairs(num_sms);
+    if (tiles < pairs) pairs = int(tiles);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(2 * pairs));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes2;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, amap, bmap, a);
+    count_launch();
+    return e != cudaSuccess ? e : cudaGetLastError();
+  }
+  if (make_map_3d_bf16(&amap, A.base, A.k, A.rows, A.z, BK, BM1) != CUDA_SUCCESS ||
+      make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, BN1) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int m_tiles = (a.M + BM1 - 1) / BM1;
+  const int n_tiles = (a.N + BN1 - 1) / BN1;
   const int64_t tiles = int64_t(m_tiles) * n_tiles * a.groups;
   const int grid = int(tiles < num_sms ? tiles : num_sms);
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes1);
   if (e != cudaSuccess) return e;
-  gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(amap, bmap, a);
+  gemm_tc_kernel<<<grid, kThreads, kSmemBytes1, s>>>(amap, bmap, a);
   count_launch();
   return cudaGetLastError();
 }

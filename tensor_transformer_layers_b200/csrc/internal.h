@@ -47,8 +47,14 @@ struct GemmArgs {
   int* err;              // device error word
 };
 
-cudaError_t launch_gemm(const CUtensorMap& amap, const CUtensorMap& bmap, const GemmArgs& a, int num_sms,
-                        cudaStream_t s);
+// A bf16 operand seen as a 3-D tensor {k (contiguous), rows, z}: the GEMM
+// builds its TMA maps from this (box sizes depend on the kernel it picks).
+struct GemmOperand {
+  const void* base;
+  uint64_t k, rows, z;
+};
+
+cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------------------------
 // a6: per-shard SDPA.  qkv map: 3-D fp16 {3*Hs*128, M, T}, box {64, 128, 1}.

@@ -82,20 +82,14 @@ extern "C" tp_status tp_mlp_pair_sharded_noalloc(const uint16_t* X, int64_t M, i
   uint16_t* H = static_cast<uint16_t*>(scratch);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  CUtensorMap wup_map, wdown_map;
-  if (make_map_3d_bf16(&wup_map, W_up_shards, uint64_t(D), uint64_t(Fs), uint64_t(tp_degree), 64, 256) !=
-          CUDA_SUCCESS ||
-      make_map_3d_bf16(&wdown_map, W_down_shards, uint64_t(Fs), uint64_t(D), uint64_t(tp_degree), 64, 256) !=
-          CUDA_SUCCESS)
-    return TP_ERR_CUDA;
+  const GemmOperand wup{W_up_shards, uint64_t(D), uint64_t(Fs), uint64_t(tp_degree)};
+  const GemmOperand wdown{W_down_shards, uint64_t(Fs), uint64_t(D), uint64_t(tp_degree)};
 
   for (int64_t m0 = 0; m0 < M; m0 += chunk) {
     const int64_t mc = (M - m0) < chunk ? (M - m0) : chunk;
     // colwise: H[r][0:mc] = GELU(X[m0:m0+mc] . W_up,r^T + b_up,r) for every shard r
-    CUtensorMap x_map, h_map;
-    if (make_map_3d_bf16(&x_map, X + m0 * D, uint64_t(D), uint64_t(mc), 1, 64, 128) != CUDA_SUCCESS ||
-        make_map_3d_bf16(&h_map, H, uint64_t(Fs), uint64_t(mc), uint64_t(tp_degree), 64, 128) != CUDA_SUCCESS)
-      return TP_ERR_CUDA;
+    const GemmOperand xop{X + m0 * D, uint64_t(D), uint64_t(mc), 1};
+    const GemmOperand hop{H, uint64_t(Fs), uint64_t(mc), uint64_t(tp_degree)};
     GemmArgs c{};
     c.M = int(mc);
     c.N = int(Fs);
@@ -111,7 +105,7 @@ extern "C" tp_status tp_mlp_pair_sharded_noalloc(const uint16_t* X, int64_t M, i
     c.gelu = 1;
     c.out_f16 = 0;
     c.err = err;
-    if (launch_gemm(x_map, wup_map, c, num_sms, s) != cudaSuccess) return TP_ERR_CUDA;
+    if (launch_gemm(xop, wup, c, num_sms, s) != cudaSuccess) return TP_ERR_CUDA;
     // rowwise: Y[m0:m0+mc] = sum_r H[r][0:mc] . W_down,r^T + b_down
     GemmArgs r{};
     r.M = int(mc);
@@ -128,7 +122,7 @@ extern "C" tp_status tp_mlp_pair_sharded_noalloc(const uint16_t* X, int64_t M, i
     r.gelu = 0;
     r.out_f16 = 0;
     r.err = err;
-    if (launch_gemm(h_map, wdown_map, r, num_sms, s) != cudaSuccess) return TP_ERR_CUDA;
+    if (launch_gemm(hop, wdown, r, num_sms, s) != cudaSuccess) return TP_ERR_CUDA;
   }
   return TP_OK;
 }

@@ -19,6 +19,8 @@ pytestmark = pytest.mark.gpu
     (300, 1024, 512, 4, False, True, False),
     (256, 3072, 2304, 1, False, False, True),  # one QKV shard of the Flux attention block (fp16 out)
     (129, 72, 264, 3, True, True, True),
+    (257, 72, 264, 3, True, True, False),     # CTA-pair kernel: one row into a second 256-row tile
+    (512, 192, 520, 2, False, True, False),   # CTA-pair kernel, ragged N
 ])
 def test_colwise(M, K, Ns, T, gelu, bias, f16):
     X = syn.normal_bf16((M, K), 1.0, seed=M, tid=300)
@@ -51,6 +53,8 @@ def test_colwise(M, K, Ns, T, gelu, bias, f16):
     (129, 72, 264, 3, True),           # ragged
     (300, 512, 520, 4, False),
     (256, 768, 3072, 4, False),        # Flux attention out-projection shards
+    (257, 72, 264, 3, True),           # CTA-pair kernel, ragged everywhere
+    (1024, 1536, 520, 8, True),        # CTA-pair kernel, 8 shards in one K loop
 ])
 def test_rowwise_sum(M, Ks, N, T, bias):
     A = syn.normal_bf16((T, M, Ks), 1.0, seed=M, tid=310)
