@@ -11,6 +11,11 @@ duration is measured with CUDA events inside the timed region (a GPU test
 checks that the sequence is bit-identical to ``tp_mlp_pair``).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload flux_mlp|flux_attn|wide_block|flux_reduce]
+The default workload (flux_mlp) is the headline line.  The others time the
+remaining rows the same way: flux_attn (QKV head split, QKV GEMM, SDPA,
+out-projection), wide_block (attention then MLP pair at tp_degree 8, every
+row) and flux_reduce (the standalone partial-sum reduction, GB/s).
 Under torchrun (N > 1) every rank runs the same workload on its own tokens
 (independent replicas: the layer pair has no exchange step when all shards of
 a layer live on one GPU), so per-GPU work is fixed ("weak" scaling) and the
@@ -171,37 +176,7 @@ def recorded_traffic(kernel: str, workload: str):
     return e.get("dram_bytes_per_launch")
 
 
-# --------------------------------------------------------------------------- workload
-def workload_cfg():
-    import synthetic as syn
-    return syn.CONFIGS["flux_mlp"]
-
-
-def make_inputs(cfg, rank: int):
-    import synthetic as syn
-    M, D, F = cfg["M"], cfg["D"], cfg["F"]
-    d = syn.mlp_inputs(M, D, F, cfg["seed"])
-    if rank:
-        # every replica gets its own tokens; the weights are the layer's
-        d["X"] = syn.normal_bf16((M, D), 1.0, seed=cfg["seed"] + 1000 * rank, tid=syn.TID["X"])
-    return d
-
-
-def flops_mlp(M, D, F):
-    return 4.0 * M * D * F
-
-
-# --------------------------------------------------------------------------- CPU oracle legs
-def oracle_rows_run(d, rows: int, T: int):
-    import oracle as o
-    import synthetic as syn
-    f = {k: syn.bf16_bits_to_f64(v) for k, v in d.items() if k != "X"}
-    X = syn.bf16_bits_to_f64(d["X"][:rows])
-    t0 = time.perf_counter()
-    o.mlp_sharded_summed(X, f["W_up"], f["b_up"], f["W_down"], f["b_down"], T)
-    return time.perf_counter() - t0
-
-
+# --------------------------------------------------------------------------- workloads
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -213,58 +188,384 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(d, cfg, budget_s: float = 12.0):
+def _f64(d, keys):
+    import synthetic as syn
+    return {k: syn.bf16_bits_to_f64(d[k]) for k in keys}
+
+
+class Kernel:
+    """One timed entry in a step: a name, its unit (TFLOP/s or GB/s), its
+    algorithmic work per step, and the C-ABI calls that make it."""
+
+    def __init__(self, name, unit, work, fn):
+        self.name, self.unit, self.work, self.fn = name, unit, float(work), fn
+
+
+class MlpWorkload:
+    """flux_mlp (the default line): the MLP pair, a1..a4."""
+    key = "flux_mlp"
+    metric = METRIC
+    unit = UNIT
+
+    def __init__(self, cfg=None):
+        import synthetic as syn
+        self.cfg = cfg or syn.CONFIGS["flux_mlp"]
+
+    def host_inputs(self, rank):
+        import synthetic as syn
+        c = self.cfg
+        d = syn.mlp_inputs(c["M"], c["D"], c["F"], c["seed"])
+        if rank:  # every replica gets its own tokens; the weights are the layer's
+            d["X"] = syn.normal_bf16((c["M"], c["D"]), 1.0, seed=c["seed"] + 1000 * rank, tid=syn.TID["X"])
+        return d
+
+    def work(self):
+        c = self.cfg
+        return 4.0 * c["M"] * c["D"] * c["F"]
+
+    def kernels(self, tp, g, dev):
+        import torch
+        M, D, F, T = self.cfg["M"], self.cfg["D"], self.cfg["F"], self.cfg["T"]
+        Fs = F // T
+        b = {"w_up": torch.empty((T, Fs, D), dtype=torch.int16, device=dev),
+             "b_up": torch.empty((T, Fs), dtype=torch.int16, device=dev),
+             "w_down": torch.empty((T, D, Fs), dtype=torch.int16, device=dev),
+             "H": torch.empty((T, M, Fs), dtype=torch.int16, device=dev),
+             "Y": torch.empty((M, D), dtype=torch.int16, device=dev)}
+        ck = tp._check
+        self.bufs = b
+        return [
+            Kernel("slice_w_up", "GB/s", 2.0 * F * D * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["W_up"], F, D, tp.TP_COLWISE, T, b["w_up"]), "slice W_up")),
+            Kernel("slice_b_up", "GB/s", 2.0 * F * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["b_up"], T, Fs, tp.TP_COLWISE, T, b["b_up"]), "slice b_up")),
+            Kernel("slice_w_down", "GB/s", 2.0 * D * F * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["W_down"], D, F, tp.TP_ROWWISE, T, b["w_down"]),
+                              "slice W_down")),
+            Kernel("colwise_gemm", "TFLOP/s", 2.0 * M * D * F,
+                   lambda: ck(tp.tp_colwise_linear(g["X"], M, D, b["w_up"], b["b_up"], Fs, T, 1, tp.TP_OUT_BF16,
+                                                   b["H"]), "colwise")),
+            Kernel("rowwise_gemm", "TFLOP/s", 2.0 * M * F * D,
+                   lambda: ck(tp.tp_rowwise_linear_sum(b["H"], M, Fs, b["w_down"], D, g["b_down"], T, b["Y"]),
+                              "rowwise")),
+        ]
+
+    def one_shot(self, tp, gi, dev):
+        """The public one-shot call on device inputs `gi`; returns the output tensor."""
+        import torch
+        M, D, F, T = self.cfg["M"], self.cfg["D"], self.cfg["F"], self.cfg["T"]
+        if not hasattr(self, "_ws"):
+            self._ws = torch.empty(tp.tp_mlp_workspace_bytes(M, D, F, T), dtype=torch.uint8, device=dev)
+            self._y = torch.empty((M, D), dtype=torch.int16, device=dev)
+        tp._check(tp.tp_mlp_pair(gi["X"], M, D, F, gi["W_up"], gi["b_up"], gi["W_down"], gi["b_down"], T, self._y,
+                                 self._ws, self._ws.numel()), "tp_mlp_pair")
+        return self._y
+
+    e2e_call = "tp_mlp_pair with X, W_up, b_up, W_down, b_down copied from pinned host memory and Y copied back"
+
+    def oracle_run(self, d, rows):
+        """Runs the oracle on the first `rows` tokens; returns (seconds, algorithmic work done)."""
+        import oracle as o
+        import synthetic as syn
+        c = self.cfg
+        f = _f64(d, ["W_up", "b_up", "W_down", "b_down"])
+        X = syn.bf16_bits_to_f64(d["X"][:rows])
+        t0 = time.perf_counter()
+        o.mlp_sharded_summed(X, f["W_up"], f["b_up"], f["W_down"], f["b_down"], c["T"])
+        return time.perf_counter() - t0, 4.0 * rows * c["D"] * c["F"]
+
+    oracle_fn = "mlp_sharded_summed"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": (f"flux_mlp: TP MLP pair (colwise FFN-in + GELU(tanh), rowwise FFN-out with the "
+                             f"cross-shard sum fused), all tp_degree shards on one GPU; M={c['M']} tokens "
+                             f"(4096 image + 512 text), D={c['D']}, F={c['F']}"),
+                "M": c["M"], "D": c["D"], "F": c["F"], "tp_degree": c["T"],
+                "global_batch_tokens": c["M"] * world}
+
+
+class AttnWorkload(MlpWorkload):
+    """flux_attn: the attention block, a1 (QKV head split, W_o rowwise) and a5..a7."""
+    key = "flux_attn"
+    metric = "TP attention-block TFLOP/s (QKV fp16, bf16 weights) on 1 B200"
+
+    def __init__(self, cfg=None):
+        import synthetic as syn
+        self.cfg = cfg or syn.CONFIGS["flux_attn"]
+
+    def host_inputs(self, rank):
+        import synthetic as syn
+        c = self.cfg
+        d = syn.attn_inputs(c["M"], c["D"], c["seed"])
+        if rank:
+            d["X"] = syn.normal_bf16((c["M"], c["D"]), 1.0, seed=c["seed"] + 1000 * rank, tid=syn.TID["X"])
+        return d
+
+    def work(self):
+        M, D = self.cfg["M"], self.cfg["D"]
+        return 2.0 * M * D * 3 * D + 4.0 * M * M * D + 2.0 * M * D * D
+
+    def attn_kernels(self, tp, g, dev, X, M, D, H, T, prefix=""):
+        import torch
+        Ds = D // T
+        b = {"w_qkv": torch.empty((T, 3 * Ds, D), dtype=torch.int16, device=dev),
+             "w_o": torch.empty((T, D, Ds), dtype=torch.int16, device=dev),
+             "QKV": torch.empty((T, M, 3 * Ds), dtype=torch.int16, device=dev),
+             "O": torch.empty((T, M, Ds), dtype=torch.int16, device=dev),
+             "A": torch.empty((M, D), dtype=torch.int16, device=dev)}
+        ck = tp._check
+
+        def slice_qkv():
+            for r in range(T):
+                ck(tp.tp_shard_qkv_heads(g["W_qkv"], D, H, T, r, b["w_qkv"][r]), "slice W_qkv")
+        ks = [
+            Kernel(prefix + "slice_w_qkv", "GB/s", 2.0 * 3 * D * D * 2, slice_qkv),
+            Kernel(prefix + "slice_w_o", "GB/s", 2.0 * D * D * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["W_o"], D, D, tp.TP_ROWWISE, T, b["w_o"]), "slice W_o")),
+            Kernel(prefix + "qkv_gemm", "TFLOP/s", 2.0 * M * D * 3 * D,
+                   lambda: ck(tp.tp_colwise_linear(X, M, D, b["w_qkv"], None, 3 * Ds, T, 0, tp.TP_OUT_F16,
+                                                   b["QKV"]), "qkv")),
+            Kernel(prefix + "sdpa", "TFLOP/s", 4.0 * M * M * D,
+                   lambda: ck(tp.tp_sdpa_shards(b["QKV"], M, H, T, b["O"]), "sdpa")),
+            Kernel(prefix + "out_gemm", "TFLOP/s", 2.0 * M * D * D,
+                   lambda: ck(tp.tp_rowwise_linear_sum(b["O"], M, Ds, b["w_o"], D, None, T, b["A"]), "out")),
+        ]
+        return ks, b
+
+    def kernels(self, tp, g, dev):
+        c = self.cfg
+        ks, self.bufs = self.attn_kernels(tp, g, dev, g["X"], c["M"], c["D"], c["H"], c["T"])
+        return ks
+
+    def one_shot(self, tp, gi, dev):
+        import torch
+        c = self.cfg
+        M, D, H, T = c["M"], c["D"], c["H"], c["T"]
+        if not hasattr(self, "_ws"):
+            self._ws = torch.empty(tp.tp_attn_workspace_bytes(M, D, H, T), dtype=torch.uint8, device=dev)
+            self._y = torch.empty((M, D), dtype=torch.int16, device=dev)
+        tp._check(tp.tp_attn_block(gi["X"], M, D, gi["W_qkv"], gi["W_o"], H, T, self._y, self._ws,
+                                   self._ws.numel()), "tp_attn_block")
+        return self._y
+
+    e2e_call = "tp_attn_block with X, W_qkv, W_o copied from pinned host memory and Y copied back"
+
+    def oracle_run(self, d, rows):
+        import oracle as o
+        c = self.cfg
+        M, D, H, T = c["M"], c["D"], c["H"], c["T"]
+        f = _f64(d, ["X", "W_qkv", "W_o"])
+        t0 = time.perf_counter()
+        o.attn_rows(f["X"], f["W_qkv"], f["W_o"], H, list(range(rows)), tp_degree=T)
+        # work actually done: K and V for every token, Q / attention / out-projection for `rows` tokens
+        done = 2.0 * M * D * 2 * D + 2.0 * rows * D * D + 4.0 * rows * M * D + 2.0 * rows * D * D
+        return time.perf_counter() - t0, done
+
+    oracle_fn = "attn_rows"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": (f"flux_attn: TP attention block (head-split QKV colwise, per-shard SDPA, rowwise "
+                             f"out-projection with the cross-shard sum fused); M={c['M']}, D={c['D']}, "
+                             f"{c['H']} heads x 128"),
+                "M": c["M"], "D": c["D"], "heads": c["H"], "tp_degree": c["T"],
+                "global_batch_tokens": c["M"] * world}
+
+
+class BlockWorkload(AttnWorkload):
+    """wide_block: attention then MLP pair at tp_degree 8 (every row a1..a7)."""
+    key = "wide_block"
+    metric = "TP DiT-block (attention + MLP pair) TFLOP/s on 1 B200"
+
+    def __init__(self, cfg=None):
+        import synthetic as syn
+        self.cfg = cfg or syn.CONFIGS["wide_block"]
+
+    def host_inputs(self, rank):
+        import synthetic as syn
+        c = self.cfg
+        d = syn.block_inputs(c["M"], c["D"], c["F"], c["seed"])
+        if rank:
+            d["X"] = syn.normal_bf16((c["M"], c["D"]), 1.0, seed=c["seed"] + 1000 * rank, tid=syn.TID["X"])
+        return d
+
+    def work(self):
+        c = self.cfg
+        return AttnWorkload.work(self) + 4.0 * c["M"] * c["D"] * c["F"]
+
+    def kernels(self, tp, g, dev):
+        c = self.cfg
+        M, D, H, F, T = c["M"], c["D"], c["H"], c["F"], c["T"]
+        ks, b = self.attn_kernels(tp, g, dev, g["X"], M, D, H, T, prefix="attn_")
+        mlp = MlpWorkload(dict(M=M, D=D, F=F, T=T, seed=c["seed"]))
+        g2 = dict(g)
+        g2["X"] = b["A"]
+        ks += [Kernel("mlp_" + k.name, k.unit, k.work, k.fn) for k in mlp.kernels(tp, g2, dev)]
+        self.bufs = {**b, **mlp.bufs}
+        return ks
+
+    def one_shot(self, tp, gi, dev):
+        import torch
+        c = self.cfg
+        M, D, H, F, T = c["M"], c["D"], c["H"], c["F"], c["T"]
+        if not hasattr(self, "_ws"):
+            self._ws = torch.empty(max(tp.tp_attn_workspace_bytes(M, D, H, T), tp.tp_mlp_workspace_bytes(M, D, F, T)),
+                                   dtype=torch.uint8, device=dev)
+            self._a = torch.empty((M, D), dtype=torch.int16, device=dev)
+            self._y = torch.empty((M, D), dtype=torch.int16, device=dev)
+        tp._check(tp.tp_attn_block(gi["X"], M, D, gi["W_qkv"], gi["W_o"], H, T, self._a, self._ws,
+                                   self._ws.numel()), "tp_attn_block")
+        tp._check(tp.tp_mlp_pair(self._a, M, D, F, gi["W_up"], gi["b_up"], gi["W_down"], gi["b_down"], T, self._y,
+                                 self._ws, self._ws.numel()), "tp_mlp_pair")
+        return self._y
+
+    e2e_call = ("tp_attn_block then tp_mlp_pair with X and all weights copied from pinned host memory and Y "
+                "copied back")
+
+    def oracle_run(self, d, rows):
+        import oracle as o
+        c = self.cfg
+        M, D, H, F, T = c["M"], c["D"], c["H"], c["F"], c["T"]
+        f = _f64(d, ["X", "W_qkv", "W_o", "W_up", "b_up", "W_down", "b_down"])
+        t0 = time.perf_counter()
+        o.block_rows(f["X"], f["W_qkv"], f["W_o"], H, f["W_up"], f["b_up"], f["W_down"], f["b_down"],
+                     list(range(rows)), tp_degree=T)
+        done = (2.0 * M * D * 2 * D + 2.0 * rows * D * D + 4.0 * rows * M * D + 2.0 * rows * D * D
+                + 4.0 * rows * D * F)
+        return time.perf_counter() - t0, done
+
+    oracle_fn = "block_rows"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": (f"wide_block: attention block then MLP pair, tp_degree {c['T']}; M={c['M']}, "
+                             f"D={c['D']}, {c['H']} heads x 128, F={c['F']}"),
+                "M": c["M"], "D": c["D"], "heads": c["H"], "F": c["F"], "tp_degree": c["T"],
+                "global_batch_tokens": c["M"] * world}
+
+
+class ReduceWorkload(MlpWorkload):
+    """flux_reduce: the standalone partial-sum reduction (a8) on flux_mlp-sized partials."""
+    key = "flux_reduce"
+    metric = "TP partial-sum reduction GB/s on 1 B200"
+    unit = "GB/s"
+
+    def __init__(self, cfg=None):
+        import synthetic as syn
+        c = syn.CONFIGS["flux_mlp"]
+        self.cfg = cfg or dict(M=c["M"], N=c["D"], T=c["T"], seed=c["seed"])
+
+    def host_inputs(self, rank):
+        import numpy as np
+        import synthetic as syn
+        c = self.cfg
+        parts = syn.bf16_bits_to_f32(syn.normal_bf16((c["T"], c["M"], c["N"]), 1.0, seed=c["seed"] + rank,
+                                                     tid=200))
+        return {"parts": np.ascontiguousarray(parts), "bias": syn.normal_bf16((c["N"],), 0.02, c["seed"], 202)}
+
+    def work(self):
+        c = self.cfg
+        return 4.0 * c["T"] * c["M"] * c["N"] + 2.0 * c["M"] * c["N"] + 2.0 * c["N"]
+
+    def kernels(self, tp, g, dev):
+        import torch
+        c = self.cfg
+        self.bufs = {"Y": torch.empty((c["M"], c["N"]), dtype=torch.int16, device=dev)}
+        return [Kernel("reduce", "GB/s", self.work(),
+                       lambda: tp._check(tp.tp_reduce_partials(g["parts"], c["M"], c["N"], c["T"], g["bias"],
+                                                               self.bufs["Y"]), "reduce"))]
+
+    def one_shot(self, tp, gi, dev):
+        c = self.cfg
+        tp._check(tp.tp_reduce_partials(gi["parts"], c["M"], c["N"], c["T"], gi["bias"], self.bufs["Y"]), "reduce")
+        return self.bufs["Y"]
+
+    e2e_call = "tp_reduce_partials with the fp32 partials copied from pinned host memory and Y copied back"
+
+    def oracle_run(self, d, rows):
+        import numpy as np
+        import oracle as o
+        import synthetic as syn
+        c = self.cfg
+        parts = [d["parts"][r][:rows].astype(np.float64) for r in range(c["T"])]
+        t0 = time.perf_counter()
+        o.reduce_partials(parts, syn.bf16_bits_to_f64(d["bias"]))
+        return time.perf_counter() - t0, rows * (4.0 * c["T"] * c["N"] + 2.0 * c["N"])
+
+    oracle_fn = "reduce_partials"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": f"flux_reduce: Y = bf16(sum of {c['T']} fp32 partials + bias), {c['M']} x {c['N']}",
+                "M": c["M"], "N": c["N"], "tp_degree": c["T"], "global_batch_tokens": c["M"] * world}
+
+
+WORKLOADS = {w.key: w for w in (MlpWorkload, AttnWorkload, BlockWorkload, ReduceWorkload)}
+
+
+def workload_cfg():
+    """The default workload's configuration."""
+    return MlpWorkload().cfg
+
+
+def _scale(unit):
+    return 1e12 if unit == "TFLOP/s" else 1e9
+
+
+# --------------------------------------------------------------------------- CPU oracle legs
+def cpu_baseline(wl, d, budget_s: float = 12.0):
     """The oracle as it stands, on a bounded sample of the workload's token rows."""
-    M, D, F, T = cfg["M"], cfg["D"], cfg["F"], cfg["T"]
-    probe = 64
-    oracle_rows_run(d, probe, T)  # warm
-    t = oracle_rows_run(d, probe, T)
+    M = wl.cfg["M"]
+    probe = 16
+    wl.oracle_run(d, probe)  # warm
+    t, _ = wl.oracle_run(d, probe)
     rows = int(min(M, max(probe, probe * budget_s / max(t, 1e-6))))
-    t = oracle_rows_run(d, rows, T)
-    return {"value": flops_mlp(rows, D, F) / t / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{rows} of {M} token rows of the workload through the fp64 oracle "
-                      f"(mlp_sharded_summed, tp_degree {T}), {t:.1f} s"}
+    if wl.key in ("flux_attn", "wide_block"):
+        rows = min(rows, 256)  # the K/V projection of every token dominates; more rows add little
+    t, done = wl.oracle_run(d, rows)
+    return {"value": done / t / _scale(wl.unit), "unit": wl.unit, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} of {M} token rows of the workload through the fp64 oracle ({wl.oracle_fn}, "
+                      f"tp_degree {wl.cfg['T']}), {t:.1f} s; value = work the oracle performed / time"}
 
 
-def run_reference(args, cfg, rank, world):
+def run_reference(args, wl, rank, world):
     if rank != 0:
         return None  # rank 0 alone runs the CPU reference
-    d = make_inputs(cfg, 0)
-    M, D, F, T = cfg["M"], cfg["D"], cfg["F"], cfg["T"]
-    probe = 32
-    oracle_rows_run(d, probe, T)
-    t = oracle_rows_run(d, probe, T)
+    d = wl.host_inputs(0)
+    M = wl.cfg["M"]
+    probe = 16
+    wl.oracle_run(d, probe)
+    t, _ = wl.oracle_run(d, probe)
     per_step = max(0.2, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
     rows = int(min(M, max(8, probe * per_step / max(t, 1e-6))))
     for _ in range(args.warmup):
-        oracle_rows_run(d, rows, T)
-    times = [oracle_rows_run(d, rows, T) for _ in range(args.steps)]
-    total = sum(times)
-    value = flops_mlp(rows, D, F) * args.steps / total / 1e12
-    sample = (f"{rows} of {M} token rows per step through the fp64 oracle (mlp_sharded_summed, "
-              f"tp_degree {T}) on host cores")
+        wl.oracle_run(d, rows)
+    res = [wl.oracle_run(d, rows) for _ in range(args.steps)]
+    total = sum(r[0] for r in res)
+    value = sum(r[1] for r in res) / total / _scale(wl.unit)
+    sample = (f"{rows} of {M} token rows per step through the fp64 oracle ({wl.oracle_fn}, "
+              f"tp_degree {wl.cfg['T']}) on host cores")
     return {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "impl": "reference", "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": config_dict(cfg, world),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "data": "synthetic", "config": config_dict(wl, world),
+        "cpu_baseline": {"value": value, "unit": wl.unit, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-def config_dict(cfg, world):
-    return {"workload": (f"flux_mlp: TP MLP pair (colwise FFN-in + GELU(tanh), rowwise FFN-out with the "
-                         f"cross-shard sum fused), all tp_degree shards on one GPU; M={cfg['M']} tokens "
-                         f"(4096 image + 512 text), D={cfg['D']}, F={cfg['F']}"),
-            "M": cfg["M"], "D": cfg["D"], "F": cfg["F"], "tp_degree": cfg["T"], "global_batch_tokens": cfg["M"] * world,
-            "l2": ("not flushed: inputs larger than L2 (each step reads 179 MB of inputs, > 126 MB L2, "
-                   "and moves about 0.6 GB in total)"),
-            "parallelism": "single GPU" if world == 1 else f"{world} independent replicas (one per GPU)"}
+def config_dict(wl, world):
+    d = wl.config(world)
+    d["l2"] = ("not flushed: inputs larger than L2 (the step reads more than 126 MB of inputs and moves "
+               "several times that)")
+    d["parallelism"] = "single GPU" if world == 1 else f"{world} independent replicas (one per GPU)"
+    return d
 
 
 # --------------------------------------------------------------------------- GPU leg
-def run_ours(args, cfg, rank, local_rank, world):
+def run_ours(args, wl, rank, local_rank, world):
     import numpy as np
     import torch
 
@@ -272,39 +573,34 @@ def run_ours(args, cfg, rank, local_rank, world):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    M, D, F, T = cfg["M"], cfg["D"], cfg["F"], cfg["T"]
-    Fs = F // T
-    d = make_inputs(cfg, rank)
-    host = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).pin_memory() for k, v in d.items()}
-    g = {k: v.to(dev) for k, v in host.items()}
-    w_up = torch.empty((T, Fs, D), dtype=torch.int16, device=dev)
-    b_up = torch.empty((T, Fs), dtype=torch.int16, device=dev)
-    w_down = torch.empty((T, D, Fs), dtype=torch.int16, device=dev)
-    H = torch.empty((T, M, Fs), dtype=torch.int16, device=dev)
-    Y = torch.empty((M, D), dtype=torch.int16, device=dev)
-    input_bytes = sum(v.numel() * v.element_size() for v in g.values())
-    assert input_bytes > L2_BYTES, "the step's inputs must exceed L2 (no flush between steps)"
-    check = tp._check
+    d = wl.host_inputs(rank)
 
-    names = ["slice_w_up", "slice_b_up", "slice_w_down", "colwise_gemm", "rowwise_gemm"]
+    def pin(v):
+        a = np.ascontiguousarray(v)
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.pin_memory()
+
+    host = {k: pin(v) for k, v in d.items()}
+    g = {k: v.to(dev) for k, v in host.items()}
+    input_bytes = sum(v.numel() * v.element_size() for v in g.values())
+    # Inputs larger than L2 need no flush between steps; smaller ones get one.
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if input_bytes <= L2_BYTES else None
+    kernels = wl.kernels(tp, g, dev)
+    names = [k.name for k in kernels]
+    nk = len(kernels)
 
     def step(ev):
         ev[0].record()
-        check(tp.tp_shard_weight_all(g["W_up"], F, D, tp.TP_COLWISE, T, w_up), "slice W_up")
-        ev[1].record()
-        check(tp.tp_shard_weight_all(g["b_up"], T, Fs, tp.TP_COLWISE, T, b_up), "slice b_up")
-        ev[2].record()
-        check(tp.tp_shard_weight_all(g["W_down"], D, F, tp.TP_ROWWISE, T, w_down), "slice W_down")
-        ev[3].record()
-        check(tp.tp_colwise_linear(g["X"], M, D, w_up, b_up, Fs, T, 1, tp.TP_OUT_BF16, H), "colwise")
-        ev[4].record()
-        check(tp.tp_rowwise_linear_sum(H, M, Fs, w_down, D, g["b_down"], T, Y), "rowwise")
-        ev[5].record()
+        for j, k in enumerate(kernels):
+            k.fn()
+            ev[j + 1].record()
 
     def new_events():
-        return [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        return [torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)]
 
     for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
         step(new_events())
     torch.cuda.synchronize()
 
@@ -316,6 +612,8 @@ def run_ours(args, cfg, rank, local_rank, world):
     sampler.start()
     t_wall0 = time.perf_counter()
     for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()  # outside the step's events
         step(evs[i])
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall0
@@ -329,51 +627,42 @@ def run_ours(args, cfg, rank, local_rank, world):
     for ev in evs:
         for j, n in enumerate(names):
             per_kernel[n].append(ev[j].elapsed_time(ev[j + 1]))
-        step_ms.append(ev[0].elapsed_time(ev[5]))
+        step_ms.append(ev[0].elapsed_time(ev[nk]))
     local_s = sum(step_ms) / 1e3
     max_s = max_over_ranks(local_s)
-    flops = flops_mlp(M, D, F)
-    value = job_value(flops, world, args.steps, max_s)
+    scale = _scale(wl.unit)
+    value = wl.work() * world * args.steps / max_s / scale
 
     peaks, peak_src = load_peaks()
     tc_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    kinfo = {}
-    algo = {
-        "slice_w_up": ("GB/s", 2.0 * F * D * 2),
-        "slice_b_up": ("GB/s", 2.0 * F * 2),
-        "slice_w_down": ("GB/s", 2.0 * D * F * 2),
-        "colwise_gemm": ("TFLOP/s", 2.0 * M * D * F),
-        "rowwise_gemm": ("TFLOP/s", 2.0 * M * F * D),
-    }
     tot = sum(statistics.mean(v) for v in per_kernel.values())
-    for n in names:
-        ms = statistics.mean(per_kernel[n])
-        unit, work = algo[n]
-        ach = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
-        pk = tc_peak if unit == "TFLOP/s" else hbm_peak
-        kinfo[n] = {"ms": round(ms, 5), "share": round(ms / tot, 4), "achieved": round(ach, 1), "unit": unit,
-                    "frac": round(ach / pk, 4)}
-    dom = max(("colwise_gemm", "rowwise_gemm"), key=lambda n: kinfo[n]["ms"])
-    roofline = {"kernel": dom, "bound": "tensor", "achieved": kinfo[dom]["achieved"], "peak": tc_peak,
-                "unit": "TFLOP/s", "frac": kinfo[dom]["frac"],
-                "traffic": recorded_traffic(dom, "flux_mlp"),
-                "peak_source": f"{peak_src} (bf16 burst; {'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})",
-                "algorithmic_flops_per_launch": algo[dom][1]}
+    kinfo = {}
+    for k in kernels:
+        ms = statistics.mean(per_kernel[k.name])
+        ach = k.work / (ms / 1e3) / _scale(k.unit)
+        pk = tc_peak if k.unit == "TFLOP/s" else hbm_peak
+        kinfo[k.name] = {"ms": round(ms, 5), "share": round(ms / tot, 4), "achieved": round(ach, 1),
+                         "unit": k.unit, "frac": round(ach / pk, 4)}
+    dom = max(kernels, key=lambda k: kinfo[k.name]["ms"])
+    src = "MEASURED_PEAKS.json" if peak_src == "measured" else "the recipe's fallback"
+    roofline = {"kernel": dom.name, "bound": "tensor" if dom.unit == "TFLOP/s" else "hbm",
+                "achieved": kinfo[dom.name]["achieved"], "peak": tc_peak if dom.unit == "TFLOP/s" else hbm_peak,
+                "unit": dom.unit, "frac": kinfo[dom.name]["frac"], "traffic": recorded_traffic(dom.name, wl.key),
+                "peak_source": f"{peak_src}: {'bf16 burst' if dom.unit == 'TFLOP/s' else 'HBM copy'} from {src}",
+                "algorithmic_work_per_launch": dom.work}
 
-    # ---- end to end: the one-shot public call with host buffers copied in and the result copied out.
-    ws = torch.empty(tp.tp_mlp_workspace_bytes(M, D, F, T), dtype=torch.uint8, device=dev)
-    y_host = torch.empty((M, D), dtype=torch.int16).pin_memory()
+    # ---- end to end: the public one-shot call with host buffers copied in and the result copied out.
+    y0 = wl.one_shot(tp, g, dev)
+    y_host = torch.empty(y0.shape, dtype=y0.dtype).pin_memory()
     gi = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = y_host.numel() * 2
+    d2h = y_host.numel() * y_host.element_size()
 
     def e2e_step():
         for k in host:
             gi[k].copy_(host[k], non_blocking=True)
-        check(tp.tp_mlp_pair(gi["X"], M, D, F, gi["W_up"], gi["b_up"], gi["W_down"], gi["b_down"], T, Y, ws,
-                             ws.numel()), "tp_mlp_pair")
-        y_host.copy_(Y, non_blocking=True)
+        y_host.copy_(wl.one_shot(tp, gi, dev), non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         e2e_step()
@@ -388,23 +677,25 @@ def run_ours(args, cfg, rank, local_rank, world):
     torch.cuda.synchronize()
     e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     barrier()
-    e2e = {"value": job_value(flops, world, n_e2e, e2e_s), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h,
-           "call": "tp_mlp_pair with X, W_up, b_up, W_down, b_down copied from pinned host memory and Y copied back"}
+    e2e = {"value": wl.work() * world * n_e2e / e2e_s / scale, "unit": wl.unit, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "call": wl.e2e_call}
 
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
-        "config": config_dict(cfg, world),
-        "frac_of_nominal_dense_bf16": round(value / world / 2250.0, 4),
-        "frac_of_measured_bf16": round(value / world / tc_peak, 4),
-        "roofline": roofline, "kernels": kinfo, "clocks": clocks, "e2e": e2e,
-        "gpu_launches": int(launches), "wall_s_timed_region": round(t_wall, 4),
-        "cpu_baseline": None,
+        "config": config_dict(wl, world),
     }
+    if flush is not None:
+        out["config"]["l2"] = (f"flushed before every step ({2 * L2_BYTES >> 20} MiB write, outside the step's "
+                               f"events): the inputs ({input_bytes >> 20} MiB) fit in L2")
+    if wl.unit == "TFLOP/s":
+        out["frac_of_nominal_dense_bf16"] = round(value / world / 2250.0, 4)
+        out["frac_of_measured_bf16"] = round(value / world / tc_peak, 4)
+    out.update({"roofline": roofline, "kernels": kinfo, "clocks": clocks, "e2e": e2e,
+                "gpu_launches": int(launches), "wall_s_timed_region": round(t_wall, 4), "cpu_baseline": None})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(d, cfg)
+        out["cpu_baseline"] = cpu_baseline(wl, d)
     return out
 
 
@@ -414,11 +705,13 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="flux_mlp",
+                    help="flux_mlp (default: the headline line); the others time the remaining rows")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle leg (cpu_baseline is then null)")
     args = ap.parse_args(argv)
     rank, local_rank, world = dist_env()
-    cfg = workload_cfg()
+    wl = WORKLOADS[args.workload]()
 
     if world > 1 and args.impl == "ours":
         import datetime
@@ -431,9 +724,9 @@ def main(argv=None):
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     try:
         if args.impl == "reference":
-            out = run_reference(args, cfg, rank, world)
+            out = run_reference(args, wl, rank, world)
         else:
-            out = run_ours(args, cfg, rank, local_rank, world)
+            out = run_ours(args, wl, rank, local_rank, world)
         if rank == 0 and out is not None:
             print(json.dumps(out), flush=True)
     finally:

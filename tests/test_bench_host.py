@@ -61,7 +61,7 @@ def test_job_value():
 def test_reference_arm_other_ranks_do_no_work():
     class A:
         steps, warmup = 1, 0
-    assert bench.run_reference(A(), bench.workload_cfg(), rank=1, world=2) is None
+    assert bench.run_reference(A(), bench.MlpWorkload(), rank=1, world=2) is None
 
 
 def test_reference_arm_json_line():
