@@ -317,8 +317,7 @@ class AttnWorkload(MlpWorkload):
         ck = tp._check
 
         def slice_qkv():
-            for r in range(T):
-                ck(tp.tp_shard_qkv_heads(g["W_qkv"], D, H, T, r, b["w_qkv"][r]), "slice W_qkv")
+            ck(tp.tp_shard_qkv_heads_all(g["W_qkv"], D, H, T, b["w_qkv"]), "slice W_qkv")
         ks = [
             Kernel(prefix + "slice_w_qkv", "GB/s", 2.0 * 3 * D * D * 2, slice_qkv),
             Kernel(prefix + "slice_w_o", "GB/s", 2.0 * D * D * 2,

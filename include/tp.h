@@ -126,6 +126,11 @@ tp_status tp_shard_bias(const uint16_t* b, int64_t n, int tp_degree, int rank,
 tp_status tp_shard_qkv_heads(const uint16_t* W_qkv, int64_t D, int heads, int tp_degree,
                              int rank, uint16_t* out, void* stream);
 
+/* All T head-split shards in one launch: out is [T x 3D/T x D], shard r at
+ * out + r*3D/T*D.  Same checks as tp_shard_qkv_heads (without `rank`). */
+tp_status tp_shard_qkv_heads_all(const uint16_t* W_qkv, int64_t D, int heads, int tp_degree,
+                                 uint16_t* out, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Step-level calls (each one kernel), on already-sharded operands.
  * ------------------------------------------------------------------------- */

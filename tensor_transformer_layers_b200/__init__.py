@@ -46,6 +46,7 @@ SIGNATURES = {
     "tp_shard_weight": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P]),
     "tp_shard_weight_all": (_I, [_P, _I64, _I64, _I, _I, _P, _P]),
     "tp_kernel_launches": (ctypes.c_uint64, []),
+    "tp_shard_qkv_heads_all": (_I, [_P, _I64, _I, _I, _P, _P]),
     "tp_shard_bias": (_I, [_P, _I64, _I, _I, _P, _P]),
     "tp_shard_qkv_heads": (_I, [_P, _I64, _I, _I, _I, _P, _P]),
     "tp_colwise_linear": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _I, _P, _P]),
@@ -132,6 +133,10 @@ def tp_shard_weight(W, rows, cols, style, tp_degree, rank, out, stream=None) -> 
 
 def tp_shard_weight_all(W, rows, cols, style, tp_degree, out, stream=None) -> int:
     return lib().tp_shard_weight_all(_ptr(W), rows, cols, style, tp_degree, _ptr(out), _stream(stream))
+
+
+def tp_shard_qkv_heads_all(W_qkv, D, heads, tp_degree, out, stream=None) -> int:
+    return lib().tp_shard_qkv_heads_all(_ptr(W_qkv), D, heads, tp_degree, _ptr(out), _stream(stream))
 
 
 def tp_kernel_launches() -> int:

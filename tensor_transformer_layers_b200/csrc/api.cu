@@ -190,14 +190,12 @@ tp_status slice_all_rowwise(const uint16_t* W, int64_t rows, int64_t cols, int T
 }
 
 tp_status slice_all_qkv(const uint16_t* Wqkv, int64_t D, int T, uint16_t* out, cudaStream_t s) {
-  // shard r = [Q_r; K_r; V_r]; X_r = rows [r*D/T, (r+1)*D/T) of block X.
+  // shard r = [Q_r; K_r; V_r]; X_r = rows [r*D/T, (r+1)*D/T) of block X.  One
+  // launch: block (r, x) copies X_r from Wqkv[x*D + r*D/T] to out[(3r + x)*D/T].
   const int64_t rs = D / T;
-  for (int r = 0; r < T; ++r) {
-    if (launch_slice_copy(Wqkv + r * rs * D, out + int64_t(r) * 3 * rs * D, 3, rs, D, D, D * D, rs * D, s) !=
-        cudaSuccess)
-      return TP_ERR_CUDA;
-  }
-  return TP_OK;
+  return launch_slice_copy(Wqkv, out, T, rs, D, D, rs * D, 3 * rs * D, s, 3, D * D, rs * D) == cudaSuccess
+             ? TP_OK
+             : TP_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -427,6 +425,19 @@ tp_status tp_shard_qkv_heads(const uint16_t* W_qkv, int64_t D, int heads, int tp
                  cudaSuccess
              ? TP_OK
              : TP_ERR_CUDA;
+}
+
+tp_status tp_shard_qkv_heads_all(const uint16_t* W_qkv, int64_t D, int heads, int tp_degree, uint16_t* out,
+                                 void* stream) {
+  if (!W_qkv || !out) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (D < 1 || heads < 1) return TP_ERR_BAD_SHAPE;
+  if (heads % tp_degree != 0) return TP_ERR_HEADS_INDIVISIBLE;
+  if (D != int64_t(heads) * TP_HEAD_DIM) return TP_ERR_BAD_SHAPE;
+  if (!al16(W_qkv) || !al16(out)) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return slice_all_qkv(W_qkv, D, tp_degree, out, as_stream(stream));
 }
 
 // ----------------------------------------------------------------------- step-level calls

@@ -3,24 +3,31 @@
 // Under tensor parallelism the colwise Q/K/V projections give each rank a
 // subset of the heads (Diffusers "Tensor parallelism" page, section "Colwise
 // and rowwise", paragraph on attention), so attention runs independently per
-// (shard, head).  For every head j of shard r and every 128-row query tile:
+// (shard, head).  For every head j of shard r:
 //     O = softmax(Q K^T / sqrt(128)) V     (non-causal, no mask)
 // computed with an online softmax over 128-key tiles.
 //
-// Structure (one CTA per (shard, head, query tile), 192 threads):
-//   warps 0-3  softmax: thread i owns query row i (its TMEM lane), so the row
-//              max and row sum are per-thread reductions over the 128 columns
-//              it loads; p = 2^(s*log2(e)/sqrt(d) - m) with the hardware ex2;
-//              P is packed to fp16 pairs and written to TMEM; O is rescaled in
-//              TMEM only when the running max grows by more than 2^8 (the
-//              stale max is otherwise kept for both O and the row sum, which
-//              leaves the final O/l unchanged); final O/l -> bf16 -> global.
-//   warp 4     TMA producer: Q once, then K and V tiles into a 2-stage ring.
-//   warp 5     TMEM allocator + MMA issuer: S_j = Q K_j^T (both operands in
-//              shared memory, K-major) into one of two S buffers, so S_{j+1}
-//              is computed while row j's softmax runs; O += P_j V_j with P read
-//              from TMEM and V in shared memory as an MN-major operand.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P [384,448) (fp16 pairs).
+// Structure: one CTA per (shard, head, 256 query rows) = two 128-row query
+// tiles t = 0, 1, 320 threads:
+//   warps 0-3  softmax of tile 0, warps 4-7 softmax of tile 1: thread i of a
+//              warpgroup owns query row i (its TMEM lane), so the row max and
+//              row sum are per-thread reductions over the 128 scores it loads;
+//              p = 2^(s*log2(e)/sqrt(d) - m) with the hardware ex2; P is packed
+//              to fp16 pairs and written back over the first 64 columns of its
+//              own S buffer; O is rescaled in TMEM only when the running max
+//              grows by more than 8 (log2 units) - otherwise the stale max is
+//              kept for both O and the row sum, which leaves O/l unchanged.
+//   warp 8     TMA producer: Q0, Q1 once, then K and V tiles into a 2-stage ring.
+//   warp 9     TMEM allocator + MMA issuer, in the order
+//                S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
+//              so that while one warpgroup computes its softmax the tensor core
+//              works on the other tile.  S = Q K^T reads both operands from
+//              shared memory (K-major); O += P V reads P from TMEM and V from
+//              shared memory as an MN-major operand.  tcgen05 MMAs of one
+//              thread execute in issue order, so S_t(j+1) cannot overwrite P_t(j)
+//              before PV_t(j) has read it, and when S_t(j) is signalled complete
+//              PV_t(j-1) has finished updating O_t (safe to rescale).
+// TMEM columns: S0/P0 [0,128), S1/P1 [128,256), O0 [256,384), O1 [384,512).
 //
 // Precision: Q, K, V arrive in fp16 and P is rounded to fp16 (11-bit
 // significand; |Q|, |K|, |V| of a unit-variance projection stay far below the
@@ -37,26 +44,29 @@
 namespace tp {
 namespace {
 
-constexpr int kD = 128;       // head dim
-constexpr int kBQ = 128;      // query rows per CTA
-constexpr int kBKV = 128;     // keys per tile
-constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 bf16 (16 KB)
-constexpr int kQBytes = 2 * kBox;   // Q tile: d in two 64-column boxes
+constexpr int kD = 128;             // head dim
+constexpr int kBQ = 128;            // query rows per tile
+constexpr int kTiles = 2;           // query tiles per CTA
+constexpr int kBKV = 128;           // keys per KV tile
+constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 fp16 (16 KB)
+constexpr int kQBytes = 2 * kBox;   // one Q tile: d in two 64-column boxes
 constexpr int kKVBytes = 4 * kBox;  // K tile (2 boxes) + V tile (2 boxes)
 constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kQOff = 0;
-constexpr int kKVOff = kQBytes;
+constexpr int kKVOff = kTiles * kQBytes;
 constexpr int kBarOff = kKVOff + kStages * kKVBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr uint32_t kColS0 = 0, kColO0 = 256;  // tile t: S at kColS0 + 128 t, O at kColO0 + 128 t
 constexpr uint32_t kIdescS = idesc_f32acc(kBQ, kBKV, false, false);  // fp16 Q, K
 constexpr uint32_t kIdescPV = idesc_f32acc(kBQ, kD, false, true);    // fp16 P, V; B (= V) is MN-major
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kRescaleThreshold = 8.0f;                           // log2 units
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(200)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qkv, const AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -64,10 +74,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars + 0;
   uint64_t* kv_full = bars + 1;   // [2]
   uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_empty = bars + 7;   // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* pv_done = bars + 10;
+  uint64_t* s_full = bars + 5;    // [2] per query tile
+  uint64_t* p_full = bars + 7;    // [2] per query tile
+  uint64_t* o_done = bars + 9;    // [2] per query tile (after the last P.V)
   uint64_t* drain = bars + 11;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -88,15 +97,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_empty[s], 4);
+      mbar_init(&p_full[s], 4);  // the four warps of that tile's softmax warpgroup
+      mbar_init(&o_done[s], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
@@ -105,14 +113,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&qkv);
-      uint8_t* sq = smem + kQOff;
-      mbar_arrive_expect_tx(q_full, kQBytes);
-      tma_load_3d(sq, &qkv, q_full, qcol, qb * kBQ, shard);
-      tma_load_3d(sq + kBox, &qkv, q_full, qcol + 64, qb * kBQ, shard);
+      mbar_arrive_expect_tx(q_full, kTiles * kQBytes);
+      for (int t = 0; t < kTiles; ++t) {
+        uint8_t* sq = smem + kQOff + t * kQBytes;
+        const int row = qb * (kTiles * kBQ) + t * kBQ;
+        tma_load_3d(sq, &qkv, q_full, qcol, row, shard);
+        tma_load_3d(sq + kBox, &qkv, q_full, qcol + 64, row, shard);
+      }
       bool ok = true;
       int issued = 0;
       for (int j = 0; j < n_kv; ++j) {
@@ -138,50 +149,67 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&kv_full[j & 1], (j >> 1) & 1, &no_abort);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      const uint32_t sq = smem_u32(smem + kQOff);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&kv_full[st], (j >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&s_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + kKVOff + st * kKVBytes);
-        const uint32_t d_tmem = tmem_base + kColS + uint32_t(st * kBKV);
+      const uint32_t sq0 = smem_u32(smem + kQOff);
+      auto issue_s = [&](int t, int j) {
+        const uint32_t sq = sq0 + uint32_t(t * kQBytes);
+        const uint32_t sk = smem_u32(smem + kKVOff + (j & 1) * kKVBytes);
+        const uint32_t d = tmem_base + kColS0 + uint32_t(t * 128);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = uint32_t((kk >> 2) * kBox + (kk & 3) * 32);
-          umma_ss(d_tmem, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), kIdescS,
-                  kk != 0 ? 1u : 0u);
+          umma_ss(d, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), kIdescS, kk != 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[st]);
-        return true;
+        umma_commit(&s_full[t]);
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv) {
-          if (!issue_s(j + 1)) {
-            ok = false;
-            break;
-          }
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t sv = smem_u32(smem + kKVOff + (j & 1) * kKVBytes + 2 * kBox);
+        const uint32_t d = tmem_base + kColO0 + uint32_t(t * 128);
+        const uint32_t a = tmem_base + kColS0 + uint32_t(t * 128);
+#pragma unroll
+        for (int kk = 0; kk < kBKV / 16; ++kk) {
+          // 16 keys per step: P columns kk*8.. (fp16 pairs); rows kk*16.. of both V boxes
+          umma_ts(d, a + uint32_t(kk * 8), sdesc_sw128(sv + uint32_t(kk * 16 * 128), kBox, 1024), kIdescPV,
+                  (j | kk) != 0 ? 1u : 0u);
         }
-        if (!mbar_wait(p_full, j & 1, abort_flag)) {
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int st = j & 1;
+        const bool more = j + 1 < n_kv;
+        // tile 0
+        if (!mbar_wait(&p_full[0], j & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int st = j & 1;
-        const uint32_t sv = smem_u32(smem + kKVOff + st * kKVBytes + 2 * kBox);
-#pragma unroll
-        for (int kk = 0; kk < kBKV / 16; ++kk) {
-          // 16 keys per step: rows kk*16.. of both V boxes (LBO = box stride, SBO = 8 rows).
-          umma_ts(tmem_base + kColO, tmem_base + kColP + uint32_t(kk * 8),
-                  sdesc_sw128(sv + uint32_t(kk * 16 * 128), kBox, 1024), kIdescPV, (j | kk) != 0 ? 1u : 0u);
+        issue_pv(0, j);
+        if (!more) umma_commit(&o_done[0]);
+        if (more) {
+          if (!mbar_wait(&kv_full[st ^ 1], ((j + 1) >> 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_s(0, j + 1);
         }
-        umma_commit(pv_done);
-        umma_commit(&kv_empty[st]);
+        // tile 1
+        if (!mbar_wait(&p_full[1], j & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(1, j);
+        if (!more) umma_commit(&o_done[1]);
+        umma_commit(&kv_empty[st]);  // K_j and V_j no longer read once these complete
+        if (more) issue_s(1, j + 1);
       }
       if (!ok) {
         report_timeout(p.err, abort_flag);
@@ -191,16 +219,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-3)
-    const int row = qb * kBQ + warp * 32 + lane;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    // ------------------------------------------------------------ softmax (warps 0-7)
+    const int t = warp >> 2;                                     // query tile of this warpgroup
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;  // TMEM lane quarter
+    const uint32_t colS = kColS0 + uint32_t(t * 128);
+    const uint32_t colO = kColO0 + uint32_t(t * 128);
+    const int row = qb * (kTiles * kBQ) + t * kBQ + (warp & 3) * 32 + lane;
     float m_run = -INFINITY;  // running max (log2-scaled units) used for O and l
     float l_run = 0.f;
     bool ok = true;
     const float sl2 = p.scale_log2;
     for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&s_full[st], (j >> 1) & 1, abort_flag)) {
+      if (!mbar_wait(&s_full[t], j & 1, abort_flag)) {
         ok = false;
         break;
       }
@@ -209,14 +239,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < kBKV / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32_sync(tmem_base + lane_off + kColS + uint32_t(st * kBKV + c * 32), r);
+        tmem_ld32_sync(tmem_base + lane_off + colS + uint32_t(c * 32), r);
 #pragma unroll
         for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[st]);
-
       const int kv0 = j * kBKV;
       if (kv0 + kBKV > p.M) {  // ragged last key tile: keys >= M do not exist
 #pragma unroll
@@ -227,20 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < kBKV; ++i) mx = fmaxf(mx, s[i]);
       mx *= sl2;
-      // P and O are free once the previous P.V finished.
-      if (j > 0) {
-        if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-      }
       if (j == 0) {
         m_run = mx;
       } else {
         // Rescale only rows whose max grew by more than the threshold; the TMEM
         // accesses are warp-collective, so the whole warp takes the branch if any
-        // lane needs it (other lanes scale by 1).
+        // lane needs it (other lanes scale by 1).  O_t already holds P_t(j-1) V.
         const bool need = mx > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = need ? ex2_approx(m_run - mx) : 1.0f;
@@ -251,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < kD / 32; ++c) {
             uint32_t r[32];
-            const uint32_t ta = tmem_base + lane_off + kColO + uint32_t(c * 32);
+            const uint32_t ta = tmem_base + lane_off + colO + uint32_t(c * 32);
             tmem_ld32_sync(ta, r);
 #pragma unroll
             for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
@@ -260,28 +278,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       float lsum = 0.f;
-      uint32_t pk[kBKV / 2];
-#pragma unroll
-      for (int i = 0; i < kBKV / 2; ++i) {
-        const float p0 = ex2_approx(fmaf(s[2 * i], sl2, -m_run));
-        const float p1 = ex2_approx(fmaf(s[2 * i + 1], sl2, -m_run));
-        lsum += p0 + p1;
-        pk[i] = pack_f16x2(p0, p1);
-      }
-      l_run += lsum;
 #pragma unroll
       for (int c = 0; c < kBKV / 64; ++c) {
-        uint32_t r[32];
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = pk[c * 32 + i];
-        tmem_st32(tmem_base + lane_off + kColP + uint32_t(c * 32), r);
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_run));
+          const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_run));
+          lsum += p0 + p1;
+          pk[i] = pack_f16x2(p0, p1);
+        }
+        tmem_st32(tmem_base + lane_off + colS + uint32_t(c * 32), pk);  // P over S's first 64 columns
       }
+      l_run += lsum;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok) ok = mbar_wait(pv_done, (n_kv - 1) & 1, abort_flag);
+    if (ok) ok = mbar_wait(&o_done[t], 0, abort_flag);
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
@@ -289,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32_sync(tmem_base + lane_off + kColO + uint32_t(c * 32), r);
+        tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(c * 32), r);
         uint4 o[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -310,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
@@ -321,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
-  const int q_tiles = (a.M + kBQ - 1) / kBQ;
-  dim3 grid(static_cast<unsigned>(q_tiles), static_cast<unsigned>(a.T * a.Hs));
+  const int q_blocks = (a.M + kTiles * kBQ - 1) / (kTiles * kBQ);
+  dim3 grid(static_cast<unsigned>(q_blocks), static_cast<unsigned>(a.T * a.Hs));
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(qkv_map, a);

@@ -9,13 +9,16 @@
 namespace tp {
 
 // ----------------------------------------------------------------------------
-// a1: blocked 2-D copy.  For b in [0, nblocks), r in [0, rows), c in [0, cols):
-//   dst[b*dst_bstride + r*cols + c] = src[b*src_bstride + r*src_ld + c]
+// a1: blocked 2-D copy.  For b in [0, nblocks), b2 in [0, nblocks2),
+// r in [0, rows), c in [0, cols):
+//   dst[b*dst_bstride + b2*dst_bstride2 + r*cols + c]
+//     = src[b*src_bstride + b2*src_bstride2 + r*src_ld + c]
 // (element units).  cols, src_ld, the strides and both pointers must be
 // multiples of 8 elements / 16 bytes (checked by the caller).
 // ----------------------------------------------------------------------------
 cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblocks, int64_t rows, int64_t cols,
-                              int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t s);
+                              int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t s,
+                              int64_t nblocks2 = 1, int64_t src_bstride2 = 0, int64_t dst_bstride2 = 0);
 
 // ----------------------------------------------------------------------------
 // a8: Y[M x N] = bf16(sum_r parts[r] + bias)

@@ -17,10 +17,11 @@ constexpr int kUnroll = 4;
 
 __global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                               uint32_t rows, uint32_t c8, int64_t src_ld8,
-                                                              int64_t src_b8, int64_t dst_b8) {
+                                                              int64_t src_b8, int64_t dst_b8, int64_t src_b8_2,
+                                                              int64_t dst_b8_2) {
   const uint32_t total = rows * c8;  // chunks in this block (host guarantees < 2^31)
-  const uint4* s = src + int64_t(blockIdx.y) * src_b8;
-  uint4* d = dst + int64_t(blockIdx.y) * dst_b8;
+  const uint4* s = src + int64_t(blockIdx.y) * src_b8 + int64_t(blockIdx.z) * src_b8_2;
+  uint4* d = dst + int64_t(blockIdx.y) * dst_b8 + int64_t(blockIdx.z) * dst_b8_2;
   const uint32_t stride = gridDim.x * kThreads;
   for (uint32_t base = blockIdx.x * kThreads + threadIdx.x; base < total; base += stride * kUnroll) {
     uint4 v[kUnroll];
@@ -44,8 +45,9 @@ __global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __res
 }  // namespace
 
 cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblocks, int64_t rows, int64_t cols,
-                              int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t st) {
-  if (nblocks <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
+                              int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t st,
+                              int64_t nblocks2, int64_t src_bstride2, int64_t dst_bstride2) {
+  if (nblocks <= 0 || nblocks2 <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
   // A contiguous source (row segments back to back) is copied as one long span,
   // split into virtual rows so the 32-bit chunk index never overflows.
   if (src_ld == cols) {
@@ -66,10 +68,11 @@ cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblock
     int64_t blocks = (total + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
     if (blocks > 148 * 16) blocks = 148 * 16;
     if (blocks < 1) blocks = 1;
-    dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(nblocks));
+    dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(nblocks), static_cast<unsigned>(nblocks2));
     slice_copy_kernel<<<grid, kThreads, 0, st>>>(reinterpret_cast<const uint4*>(src + r0 * src_ld),
                                                  reinterpret_cast<uint4*>(dst + r0 * cols), uint32_t(nr),
-                                                 uint32_t(c8), src_ld / 8, src_bstride / 8, dst_bstride / 8);
+                                                 uint32_t(c8), src_ld / 8, src_bstride / 8, dst_bstride / 8,
+                                                 src_bstride2 / 8, dst_bstride2 / 8);
     count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -61,6 +61,18 @@ def test_qkv_heads_bit_exact(heads, T):
         assert np.array_equal(from_dev(out), o.slice_qkv_heads(W, heads, T, r))
 
 
+@pytest.mark.parametrize("heads,T", [(2, 2), (4, 1), (24, 4), (48, 8)])
+def test_qkv_heads_all_bit_exact(heads, T):
+    D = heads * 128
+    W = _bits((3 * D, D), heads * 3 + T)
+    out = torch.full((T, 3 * D // T, D), 0x5A5A, dtype=torch.int16, device="cuda")
+    assert tp.tp_shard_qkv_heads_all(to_dev(W), D, heads, T, out) == 0
+    torch.cuda.synchronize()
+    h = from_dev(out)
+    for r in range(T):
+        assert np.array_equal(h[r], o.slice_qkv_heads(W, heads, T, r))
+
+
 @pytest.mark.parametrize("n,T", [(16, 2), (12288, 4), (24576, 8)])
 def test_bias_bit_exact(n, T):
     b = _bits((n,), n)
