@@ -82,6 +82,11 @@ typedef enum {
 const char* tp_status_string(int status);
 int tp_abi_version(void);
 
+/* Text describing the last CUDA failure seen by this thread inside the library
+ * (the failing call and the CUDA error name), or "" if none.  Thread-local,
+ * overwritten by the next failure; useful after a TP_ERR_CUDA. */
+const char* tp_last_error_message(void);
+
 /* Number of kernels this library has launched in this process (all devices,
  * all threads); a telemetry counter for benchmarks. */
 uint64_t tp_kernel_launches(void);

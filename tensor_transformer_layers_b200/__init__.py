@@ -42,6 +42,7 @@ _SZ = ctypes.c_size_t
 SIGNATURES = {
     "tp_status_string": (ctypes.c_char_p, [_I]),
     "tp_abi_version": (_I, []),
+    "tp_last_error_message": (ctypes.c_char_p, []),
     "tp_check_device_error": (_I, [_P]),
     "tp_shard_weight": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P]),
     "tp_shard_weight_all": (_I, [_P, _I64, _I64, _I, _I, _P, _P]),
@@ -74,7 +75,8 @@ class TPError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         msg = lib().tp_status_string(status).decode()
-        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+        extra = lib().tp_last_error_message().decode() if status == 9 else ""
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg}){' - ' + extra if extra else ''}")
 
 
 def lib() -> ctypes.CDLL:
@@ -121,6 +123,10 @@ def tp_status_string(status: int) -> str:
 
 def tp_abi_version() -> int:
     return lib().tp_abi_version()
+
+
+def tp_last_error_message() -> str:
+    return lib().tp_last_error_message().decode()
 
 
 def tp_check_device_error(stream=None) -> int:

@@ -13,6 +13,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -77,6 +78,15 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 }  // namespace
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+thread_local char g_last_error[512] = "";
+
+cudaError_t note_cuda_error(const char* where, cudaError_t e, const char* detail) {
+  if (e != cudaSuccess)
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)%s%s", where, cudaGetErrorName(e), cudaGetErrorString(e),
+             detail ? "; " : "", detail ? detail : "");
+  return e;
+}
 
 int current_device_context(int* num_sms, int** err) {
   DeviceInfo* di = nullptr;
@@ -165,8 +175,10 @@ tp_status run_sdpa(DeviceInfo* di, const uint16_t* QKV, int64_t M, int heads, in
   if (M == 0) return TP_OK;
   const int Hs = heads / T;
   CUtensorMap map;
-  if (make_map_3d_f16(&map, QKV, uint64_t(3) * Hs * TP_HEAD_DIM, uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS)
+  if (make_map_3d_f16(&map, QKV, uint64_t(3) * Hs * TP_HEAD_DIM, uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS) {
+    note_cuda_error("attention: tensor map encode", cudaErrorInvalidValue);
     return TP_ERR_CUDA;
+  }
   AttnArgs a;
   a.M = int(M);
   a.Hs = Hs;
@@ -335,6 +347,8 @@ const char* tp_status_string(int s) {
 }
 
 int tp_abi_version(void) { return TP_ABI_VERSION; }
+
+const char* tp_last_error_message(void) { return g_last_error; }
 
 uint64_t tp_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 

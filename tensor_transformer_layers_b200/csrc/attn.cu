@@ -38,6 +38,8 @@
 // Every mbarrier wait is bounded (ptx.cuh); a timeout drains and exits.
 #include <cuda_bf16.h>
 
+#include <cstdio>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -339,10 +341,21 @@ cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cuda
   const int q_blocks = (a.M + kTiles * kBQ - 1) / (kTiles * kBQ);
   dim3 grid(static_cast<unsigned>(q_blocks), static_cast<unsigned>(a.T * a.Hs));
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) return note_cuda_error("attention: set shared memory size", e);
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(qkv_map, a);
   count_launch();
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    cudaFuncAttributes fa{};
+    char detail[160];
+    if (cudaFuncGetAttributes(&fa, attn_tc_kernel) == cudaSuccess)
+      snprintf(detail, sizeof(detail), "kernel: %d registers/thread, max %d threads/block, %zu B static smem",
+               fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes);
+    else
+      snprintf(detail, sizeof(detail), "kernel attributes unavailable");
+    return note_cuda_error("attention: launch", e, detail);
+  }
+  return cudaSuccess;
 }
 
 }  // namespace tp

@@ -530,7 +530,7 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
         make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, 128) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) return note_cuda_error("gemm (CTA pairs): set shared memory size", e);
     const int64_t tiles = int64_t((a.M + BM2 - 1) / BM2) * ((a.N + BN2 - 1) / BN2) * a.groups;
     int pairs = max_active_pairs(num_sms);
     if (tiles < pairs) pairs = int(tiles);
@@ -548,20 +548,21 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, amap, bmap, a);
     count_launch();
-    return e != cudaSuccess ? e : cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return note_cuda_error("gemm (CTA pairs): launch", e);
   }
   if (make_map_3d_bf16(&amap, A.base, A.k, A.rows, A.z, BK, BM1) != CUDA_SUCCESS ||
       make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, BN1) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+    return note_cuda_error("gemm: tensor map encode", cudaErrorInvalidValue);
   const int m_tiles = (a.M + BM1 - 1) / BM1;
   const int n_tiles = (a.N + BN1 - 1) / BN1;
   const int64_t tiles = int64_t(m_tiles) * n_tiles * a.groups;
   const int grid = int(tiles < num_sms ? tiles : num_sms);
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes1);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) return note_cuda_error("gemm: set shared memory size", e);
   gemm_tc_kernel<<<grid, kThreads, kSmemBytes1, s>>>(amap, bmap, a);
   count_launch();
-  return cudaGetLastError();
+  return note_cuda_error("gemm: launch", cudaGetLastError());
 }
 
 }  // namespace tp

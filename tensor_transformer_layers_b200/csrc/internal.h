@@ -76,6 +76,10 @@ cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cuda
 // Counts kernel launches (api.cu); every launcher calls it once per launch.
 void count_launch();
 
+// Records why a CUDA call failed (thread-local; read by tp_last_error_message)
+// and returns `e` so launchers can `return note_cuda_error(...)`.
+cudaError_t note_cuda_error(const char* where, cudaError_t e, const char* detail = nullptr);
+
 // SM count and device error word of the current device, initialising the
 // library's per-device state (tensor-map encoder included) on first use.
 // Returns a tp_status value.

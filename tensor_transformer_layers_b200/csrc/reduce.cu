@@ -75,7 +75,7 @@ cudaError_t launch_reduce_partials(const float* parts, int64_t M, int64_t N, int
                                                                reinterpret_cast<uint4*>(Y), n8_total,
                                                                uint32_t(N / 8), M * N / 4, T);
   count_launch();
-  return cudaGetLastError();
+  return note_cuda_error("reduce: launch", cudaGetLastError());
 }
 
 }  // namespace tp

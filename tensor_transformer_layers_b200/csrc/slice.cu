@@ -75,7 +75,7 @@ cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblock
                                                  src_bstride2 / 8, dst_bstride2 / 8);
     count_launch();
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) return note_cuda_error("slice: launch", e);
   }
   return cudaSuccess;
 }
