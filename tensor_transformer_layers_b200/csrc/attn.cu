@@ -68,7 +68,9 @@ constexpr float kRescaleThreshold = 8.0f;                           // log2 unit
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-__global__ void __maxnreg__(200)
+// 320 threads: ten warps, so some SM sub-partitions (16K registers each) hold
+// three of them, which caps a thread at 168 registers.
+__global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qkv, const AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -269,28 +271,28 @@ __global__ void __maxnreg__(200)
             l_run *= alpha;
           }
 #pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
-            uint32_t r[32];
-            const uint32_t ta = tmem_base + lane_off + colO + uint32_t(c * 32);
-            tmem_ld32_sync(ta, r);
+          for (int c = 0; c < kD / 16; ++c) {
+            uint32_t r[16];
+            const uint32_t ta = tmem_base + lane_off + colO + uint32_t(c * 16);
+            tmem_ld16_sync(ta, r);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(ta, r);
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st16(ta, r);
           }
         }
       }
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < kBKV / 64; ++c) {
-        uint32_t pk[32];
+      for (int c = 0; c < kBKV / 32; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_run));
-          const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_run));
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, -m_run));
+          const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, -m_run));
           lsum += p0 + p1;
           pk[i] = pack_f16x2(p0, p1);
         }
-        tmem_st32(tmem_base + lane_off + colS + uint32_t(c * 32), pk);  // P over S's first 64 columns
+        tmem_st16(tmem_base + lane_off + colS + uint32_t(c * 16), pk);  // P over S's first 64 columns
       }
       l_run += lsum;
       tmem_st_wait();
