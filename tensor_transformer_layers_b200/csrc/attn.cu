@@ -12,7 +12,9 @@
 //   warps 0-3  softmax of tile 0, warps 4-7 softmax of tile 1: thread i of a
 //              warpgroup owns query row i (its TMEM lane), so the row max and
 //              row sum are per-thread reductions over the 128 scores it loads;
-//              p = 2^(s*log2(e)/sqrt(d) - m) with the hardware ex2; P is packed
+//              p = 2^(s*log2(e)/sqrt(d) - m), three quarters with the hardware
+//              ex2 and one quarter with a polynomial on the FMA pipe (the MUFU
+//              unit is the softmax's bottleneck); P is packed
 //              to fp16 pairs and written back over the first 64 columns of its
 //              own S buffer; O is rescaled in TMEM only when the running max
 //              grows by more than 8 (log2 units) - otherwise the stale max is
@@ -240,12 +242,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       float s[kBKV];
+      {
+        // all four loads in flight before one wait
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        const uint32_t ta = tmem_base + lane_off + colS;
+        tmem_ld32(ta, r0);
+        tmem_ld32(ta + 32, r1);
+        tmem_ld32(ta + 64, r2);
+        tmem_ld32(ta + 96, r3);
+        tmem_ld_wait();
+        reg_fence32(r0);
+        reg_fence32(r1);
+        reg_fence32(r2);
+        reg_fence32(r3);
 #pragma unroll
-      for (int c = 0; c < kBKV / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32_sync(tmem_base + lane_off + colS + uint32_t(c * 32), r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(r0[i]);
+          s[32 + i] = __uint_as_float(r1[i]);
+          s[64 + i] = __uint_as_float(r2[i]);
+          s[96 + i] = __uint_as_float(r3[i]);
+        }
       }
       const int kv0 = j * kBKV;
       if (kv0 + kBKV > p.M) {  // ragged last key tile: keys >= M do not exist
@@ -287,8 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
+          // every fourth exponential on the FMA pipe, the rest on the MUFU unit
           const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, -m_run));
-          const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, -m_run));
+          const float x1 = fmaf(s[c * 32 + 2 * i + 1], sl2, -m_run);
+          const float p1 = (i & 1) ? exp2_poly(x1) : ex2_approx(x1);
           lsum += p0 + p1;
           pk[i] = pack_f16x2(p0, p1);
         }
@@ -336,7 +354,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+    y[i] = exp2_poly(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184;
+  exp2_poly_kernel<<<unsigned(blocks), 256, 0, s>>>(x, y, n);
+  count_launch();
+  return note_cuda_error("exp2_poly: launch", cudaGetLastError());
+}
 
 cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
