@@ -269,9 +269,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBKV; ++i)
           if (kv0 + i >= p.M) s[i] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // Row max with eight independent chains (a single chain of 128 dependent
+      // max operations would put its full latency on the critical path).
+      float mx8[8];
 #pragma unroll
-      for (int i = 0; i < kBKV; ++i) mx = fmaxf(mx, s[i]);
+      for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+      for (int i = 8; i < kBKV; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= sl2;
       if (j == 0) {
         m_run = mx;
@@ -297,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      float lsum = 0.f;
+      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // row sum, eight chains
 #pragma unroll
       for (int c = 0; c < kBKV / 32; ++c) {
         uint32_t pk[16];
@@ -307,12 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, -m_run));
           const float x1 = fmaf(s[c * 32 + 2 * i + 1], sl2, -m_run);
           const float p1 = (i & 1) ? exp2_poly(x1) : ex2_approx(x1);
-          lsum += p0 + p1;
+          ls8[i & 7] += p0 + p1;
           pk[i] = pack_f16x2(p0, p1);
         }
         tmem_st16(tmem_base + lane_off + colS + uint32_t(c * 16), pk);  // P over S's first 64 columns
       }
-      l_run += lsum;
+      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
