@@ -11,10 +11,11 @@
 // tiles t = 0, 1, 320 threads:
 //   warps 0-3  softmax of tile 0, warps 4-7 softmax of tile 1: thread i of a
 //              warpgroup owns query row i (its TMEM lane), so the row max and
-//              row sum are per-thread reductions over the 128 scores it loads;
-//              p = 2^(s*log2(e)/sqrt(d) - m), three quarters with the hardware
-//              ex2 and one quarter with a polynomial on the FMA pipe (the MUFU
-//              unit is the softmax's bottleneck); P is packed
+//              row sum are per-thread reductions over the 128 scores of its
+//              row.  Two passes over the S columns in TMEM (the first for the
+//              row max, the second 32 scores at a time) keep ~100 registers per
+//              thread; p = 2^(s*log2(e)/sqrt(d) - m) with the hardware ex2 and
+//              the element-wise arithmetic on packed fp32 pairs; P is packed
 //              to fp16 pairs and written back over the first 64 columns of its
 //              own S buffer; O is rescaled in TMEM only when the running max
 //              grows by more than 8 (log2 units) - otherwise the stale max is
@@ -241,41 +242,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float s[kBKV];
-      {
-        // all four loads in flight before one wait
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t ta = tmem_base + lane_off + colS;
-        tmem_ld32(ta, r0);
-        tmem_ld32(ta + 32, r1);
-        tmem_ld32(ta + 64, r2);
-        tmem_ld32(ta + 96, r3);
-        tmem_ld_wait();
-        reg_fence32(r0);
-        reg_fence32(r1);
-        reg_fence32(r2);
-        reg_fence32(r3);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(r0[i]);
-          s[32 + i] = __uint_as_float(r1[i]);
-          s[64 + i] = __uint_as_float(r2[i]);
-          s[96 + i] = __uint_as_float(r3[i]);
-        }
-      }
+      const uint32_t ta = tmem_base + lane_off + colS;
       const int kv0 = j * kBKV;
-      if (kv0 + kBKV > p.M) {  // ragged last key tile: keys >= M do not exist
-#pragma unroll
-        for (int i = 0; i < kBKV; ++i)
-          if (kv0 + i >= p.M) s[i] = -INFINITY;
-      }
-      // Row max with eight independent chains (a single chain of 128 dependent
-      // max operations would put its full latency on the critical path).
+      const bool ragged = kv0 + kBKV > p.M;  // last key tile: keys >= M do not exist
+      // Pass 1: row max.  Two loads in flight per wait; eight independent max chains.
       float mx8[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-      for (int i = 8; i < kBKV; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], s[i]);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t ra[32], rb[32];
+        tmem_ld32(ta + uint32_t(h * 64), ra);
+        tmem_ld32(ta + uint32_t(h * 64 + 32), rb);
+        tmem_ld_wait();
+        reg_fence32(ra);
+        reg_fence32(rb);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          float va = __uint_as_float(ra[i]), vb = __uint_as_float(rb[i]);
+          if (ragged) {
+            if (kv0 + h * 64 + i >= p.M) va = -INFINITY;
+            if (kv0 + h * 64 + 32 + i >= p.M) vb = -INFINITY;
+          }
+          mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(va, vb));
+        }
+      }
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= sl2;
@@ -295,30 +286,48 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < kD / 16; ++c) {
             uint32_t r[16];
-            const uint32_t ta = tmem_base + lane_off + colO + uint32_t(c * 16);
-            tmem_ld16_sync(ta, r);
+            const uint32_t to = tmem_base + lane_off + colO + uint32_t(c * 16);
+            tmem_ld16_sync(to, r);
 #pragma unroll
             for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st16(ta, r);
+            tmem_st16(to, r);
           }
         }
       }
-      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // row sum, eight chains
+      // Pass 2: p = 2^(s*scale - m), 32 scores at a time, on packed fp32 pairs.
+      // P chunk c goes to columns [16c, 16c+16), which only hold scores already read.
+      const uint64_t scale2 = f32x2(sl2, sl2);
+      const uint64_t negm2 = f32x2(-m_run, -m_run);
+      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < kBKV / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32_sync(ta + uint32_t(c * 32), r);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          // every fourth exponential on the FMA pipe, the rest on the MUFU unit
-          const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, -m_run));
-          const float x1 = fmaf(s[c * 32 + 2 * i + 1], sl2, -m_run);
-          const float p1 = (i & 1) ? exp2_poly(x1) : ex2_approx(x1);
-          ls8[i & 7] += p0 + p1;
+          float x0, x1;
+          f32x2_split(fma_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), scale2, negm2),
+                      x0, x1);
+          if (ragged) {
+            if (kv0 + c * 32 + 2 * i >= p.M) x0 = -INFINITY;
+            if (kv0 + c * 32 + 2 * i + 1 >= p.M) x1 = -INFINITY;
+          }
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          ls2[i & 3] = add_f32x2(ls2[i & 3], f32x2(p0, p1));
           pk[i] = pack_f16x2(p0, p1);
         }
-        tmem_st16(tmem_base + lane_off + colS + uint32_t(c * 16), pk);  // P over S's first 64 columns
+        tmem_st16(ta + uint32_t(c * 16), pk);
       }
-      l_run += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+      {
+        float a0, a1, b0, b1, c0, c1, d0, d1;
+        f32x2_split(ls2[0], a0, a1);
+        f32x2_split(ls2[1], b0, b1);
+        f32x2_split(ls2[2], c0, c1);
+        f32x2_split(ls2[3], d0, d1);
+        l_run += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
