@@ -245,26 +245,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ta = tmem_base + lane_off + colS;
       const int kv0 = j * kBKV;
       const bool ragged = kv0 + kBKV > p.M;  // last key tile: keys >= M do not exist
-      // Pass 1: row max.  Two loads in flight per wait; eight independent max chains.
+      // Pass 1: row max.  All four loads in flight before one wait; eight
+      // independent max chains.
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t ra[32], rb[32];
-        tmem_ld32(ta + uint32_t(h * 64), ra);
-        tmem_ld32(ta + uint32_t(h * 64 + 32), rb);
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(ta, r0);
+        tmem_ld32(ta + 32, r1);
+        tmem_ld32(ta + 64, r2);
+        tmem_ld32(ta + 96, r3);
         tmem_ld_wait();
-        reg_fence32(ra);
-        reg_fence32(rb);
+        reg_fence32(r0);
+        reg_fence32(r1);
+        reg_fence32(r2);
+        reg_fence32(r3);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          float va = __uint_as_float(ra[i]), vb = __uint_as_float(rb[i]);
+          float v0 = __uint_as_float(r0[i]), v1 = __uint_as_float(r1[i]);
+          float v2 = __uint_as_float(r2[i]), v3 = __uint_as_float(r3[i]);
           if (ragged) {
-            if (kv0 + h * 64 + i >= p.M) va = -INFINITY;
-            if (kv0 + h * 64 + 32 + i >= p.M) vb = -INFINITY;
+            if (kv0 + i >= p.M) v0 = -INFINITY;
+            if (kv0 + 32 + i >= p.M) v1 = -INFINITY;
+            if (kv0 + 64 + i >= p.M) v2 = -INFINITY;
+            if (kv0 + 96 + i >= p.M) v3 = -INFINITY;
           }
-          mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(va, vb));
+          mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(fmaxf(v0, v1), fmaxf(v2, v3)));
         }
       }
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
@@ -299,15 +306,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t scale2 = f32x2(sl2, sl2);
       const uint64_t negm2 = f32x2(-m_run, -m_run);
       uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t rc[32], rn[32];  // current chunk, next chunk (its load overlaps this chunk's math)
+      tmem_ld32(ta, rc);
+      tmem_ld_wait();
+      reg_fence32(rc);
 #pragma unroll
       for (int c = 0; c < kBKV / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32_sync(ta + uint32_t(c * 32), r);
+        if (c + 1 < kBKV / 32) tmem_ld32(ta + uint32_t((c + 1) * 32), rn);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           float x0, x1;
-          f32x2_split(fma_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), scale2, negm2),
+          f32x2_split(fma_f32x2(f32x2(__uint_as_float(rc[2 * i]), __uint_as_float(rc[2 * i + 1])), scale2, negm2),
                       x0, x1);
           if (ragged) {
             if (kv0 + c * 32 + 2 * i >= p.M) x0 = -INFINITY;
@@ -318,7 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ls2[i & 3] = add_f32x2(ls2[i & 3], f32x2(p0, p1));
           pk[i] = pack_f16x2(p0, p1);
         }
+        // P chunk c -> columns [16c, 16c+16): scores there were read by chunks <= c
         tmem_st16(ta + uint32_t(c * 16), pk);
+        if (c + 1 < kBKV / 32) {
+          tmem_ld_wait();
+          reg_fence32(rn);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rc[i] = rn[i];
+        }
       }
       {
         float a0, a1, b0, b1, c0, c1, d0, d1;
