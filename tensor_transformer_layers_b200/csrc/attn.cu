@@ -20,7 +20,8 @@
 //              own S buffer; O is rescaled in TMEM only when the running max
 //              grows by more than 8 (log2 units) - otherwise the stale max is
 //              kept for both O and the row sum, which leaves O/l unchanged.
-//   warp 8     TMA producer: Q0, Q1 once, then K and V tiles into a 2-stage ring.
+//   warp 8     TMA producer: Q0, Q1 once, then K tiles into a 3-stage ring and
+//              V tiles into a 2-stage ring, K one tile ahead of V.
 //   warp 9     TMEM allocator + MMA issuer, in the order
 //                S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
 //              so that while one warpgroup computes its softmax the tensor core
@@ -55,14 +56,17 @@ constexpr int kTiles = 2;           // query tiles per CTA
 constexpr int kBKV = 128;           // keys per KV tile
 constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 fp16 (16 KB)
 constexpr int kQBytes = 2 * kBox;   // one Q tile: d in two 64-column boxes
-constexpr int kKVBytes = 4 * kBox;  // K tile (2 boxes) + V tile (2 boxes)
-constexpr int kStages = 2;
+constexpr int kKBytes = 2 * kBox;   // one K tile (d in two boxes)
+constexpr int kVBytes = 2 * kBox;   // one V tile
+constexpr int kKStages = 3;         // K is needed a step before V: deeper ring
+constexpr int kVStages = 2;
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kQOff = 0;
-constexpr int kKVOff = kTiles * kQBytes;
-constexpr int kBarOff = kKVOff + kStages * kKVBytes;
+constexpr int kKOff = kTiles * kQBytes;
+constexpr int kVOff = kKOff + kKStages * kKBytes;
+constexpr int kBarOff = kVOff + kVStages * kVBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kColS0 = 0, kColO0 = 256;  // tile t: S at kColS0 + 128 t, O at kColO0 + 128 t
 constexpr uint32_t kIdescS = idesc_f32acc(kBQ, kBKV, false, false);  // fp16 Q, K
@@ -79,13 +83,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2] per query tile
-  uint64_t* p_full = bars + 7;    // [2] per query tile
-  uint64_t* o_done = bars + 9;    // [2] per query tile (after the last P.V)
-  uint64_t* drain = bars + 11;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* k_full = bars + 1;    // [3]
+  uint64_t* k_empty = bars + 4;   // [3]
+  uint64_t* v_full = bars + 7;    // [2]
+  uint64_t* v_empty = bars + 9;   // [2]
+  uint64_t* s_full = bars + 11;   // [2] per query tile
+  uint64_t* p_full = bars + 13;   // [2] per query tile
+  uint64_t* o_done = bars + 15;   // [2] per query tile (after the last P.V)
+  uint64_t* drain = bars + 17;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -100,9 +106,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 4);  // the four warps of that tile's softmax warpgroup
       mbar_init(&o_done[s], 1);
@@ -131,29 +141,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sq, &qkv, q_full, qcol, row, shard);
         tma_load_3d(sq + kBox, &qkv, q_full, qcol + 64, row, shard);
       }
+      // Order K_0, then (K_{j+1}, V_j) for each j: the MMA order is
+      // S(j) [K_j], PV(j) [V_j], S(j+1) [K_{j+1}], so K runs one tile ahead.
       bool ok = true;
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
+      int k_issued = 0, v_issued = 0;
+      auto load_k = [&](int j) -> bool {
+        const int st = j % kKStages;
+        if (!mbar_wait(&k_empty[st], ((j / kKStages) & 1) ^ 1u, abort_flag)) return false;
+        uint8_t* sk = smem + kKOff + st * kKBytes;
+        mbar_arrive_expect_tx(&k_full[st], kKBytes);
+        tma_load_3d(sk, &qkv, &k_full[st], kcol, j * kBKV, shard);
+        tma_load_3d(sk + kBox, &qkv, &k_full[st], kcol + 64, j * kBKV, shard);
+        ++k_issued;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
         const int st = j & 1;
-        if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        uint8_t* sk = smem + kKVOff + st * kKVBytes;
-        mbar_arrive_expect_tx(&kv_full[st], kKVBytes);
-        tma_load_3d(sk, &qkv, &kv_full[st], kcol, j * kBKV, shard);
-        tma_load_3d(sk + kBox, &qkv, &kv_full[st], kcol + 64, j * kBKV, shard);
-        tma_load_3d(sk + 2 * kBox, &qkv, &kv_full[st], vcol, j * kBKV, shard);
-        tma_load_3d(sk + 3 * kBox, &qkv, &kv_full[st], vcol + 64, j * kBKV, shard);
-        ++issued;
+        if (!mbar_wait(&v_empty[st], ((j >> 1) & 1) ^ 1u, abort_flag)) return false;
+        uint8_t* sv = smem + kVOff + st * kVBytes;
+        mbar_arrive_expect_tx(&v_full[st], kVBytes);
+        tma_load_3d(sv, &qkv, &v_full[st], vcol, j * kBKV, shard);
+        tma_load_3d(sv + kBox, &qkv, &v_full[st], vcol + 64, j * kBKV, shard);
+        ++v_issued;
+        return true;
+      };
+      ok = load_k(0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv && !load_k(j + 1)) ok = false;
+        if (ok && !load_v(j)) ok = false;
       }
       if (!ok) {
         report_timeout(p.err, abort_flag);
         const volatile int no_abort = 0;
         mbar_wait(q_full, 0, &no_abort);
-        // the last (up to) two tiles issued may still be landing
-        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j)
-          mbar_wait(&kv_full[j & 1], (j >> 1) & 1, &no_abort);
+        // the last loads issued may still be landing
+        for (int j = k_issued - kKStages < 0 ? 0 : k_issued - kKStages; j < k_issued; ++j)
+          mbar_wait(&k_full[j % kKStages], (j / kKStages) & 1, &no_abort);
+        for (int j = v_issued - 2 < 0 ? 0 : v_issued - 2; j < v_issued; ++j)
+          mbar_wait(&v_full[j & 1], (j >> 1) & 1, &no_abort);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -162,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sq0 = smem_u32(smem + kQOff);
       auto issue_s = [&](int t, int j) {
         const uint32_t sq = sq0 + uint32_t(t * kQBytes);
-        const uint32_t sk = smem_u32(smem + kKVOff + (j & 1) * kKVBytes);
+        const uint32_t sk = smem_u32(smem + kKOff + (j % kKStages) * kKBytes);
         const uint32_t d = tmem_base + kColS0 + uint32_t(t * 128);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -172,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {
-        const uint32_t sv = smem_u32(smem + kKVOff + (j & 1) * kKVBytes + 2 * kBox);
+        const uint32_t sv = smem_u32(smem + kVOff + (j & 1) * kVBytes);
         const uint32_t d = tmem_base + kColO0 + uint32_t(t * 128);
         const uint32_t a = tmem_base + kColS0 + uint32_t(t * 128);
 #pragma unroll
@@ -182,17 +207,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (j | kk) != 0 ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
+      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
+        umma_commit(&k_empty[0]);  // K_0 no longer read once these complete
       }
       for (int j = 0; j < n_kv && ok; ++j) {
-        const int st = j & 1;
         const bool more = j + 1 < n_kv;
         // tile 0
-        if (!mbar_wait(&p_full[0], j & 1, abort_flag)) {
+        if (!mbar_wait(&p_full[0], j & 1, abort_flag) || !mbar_wait(&v_full[j & 1], (j >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -200,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_pv(0, j);
         if (!more) umma_commit(&o_done[0]);
         if (more) {
-          if (!mbar_wait(&kv_full[st ^ 1], ((j + 1) >> 1) & 1, abort_flag)) {
+          if (!mbar_wait(&k_full[(j + 1) % kKStages], ((j + 1) / kKStages) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -215,8 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_pv(1, j);
         if (!more) umma_commit(&o_done[1]);
-        umma_commit(&kv_empty[st]);  // K_j and V_j no longer read once these complete
-        if (more) issue_s(1, j + 1);
+        umma_commit(&v_empty[j & 1]);  // V_j no longer read once these complete
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(&k_empty[(j + 1) % kKStages]);  // K_{j+1} done
+        }
       }
       if (!ok) {
         report_timeout(p.err, abort_flag);
