@@ -8,30 +8,35 @@
 // computed with an online softmax over 128-key tiles.
 //
 // Structure: one CTA per (shard, head, 256 query rows) = two 128-row query
-// tiles t = 0, 1, 320 threads:
-//   warps 0-3  softmax of tile 0, warps 4-7 softmax of tile 1: thread i of a
-//              warpgroup owns query row i (its TMEM lane), so the row max and
-//              row sum are per-thread reductions over the 128 scores of its
-//              row.  Two passes over the S columns in TMEM (the first for the
-//              row max, the second 32 scores at a time) keep ~100 registers per
-//              thread; p = 2^(s*log2(e)/sqrt(d) - m) with the hardware ex2 and
-//              the element-wise arithmetic on packed fp32 pairs; P is packed
-//              to fp16 pairs and written back over the first 64 columns of its
-//              own S buffer; O is rescaled in TMEM only when the running max
-//              grows by more than 8 (log2 units) - otherwise the stale max is
-//              kept for both O and the row sum, which leaves O/l unchanged.
-//   warp 8     TMA producer: Q0, Q1 once, then K tiles into a 3-stage ring and
-//              V tiles into a 2-stage ring, K one tile ahead of V.
-//   warp 9     TMEM allocator + MMA issuer, in the order
+// tiles t = 0, 1, 576 threads:
+//   warps 0-15 softmax, eight per tile.  TMEM lets warp w reach lanes
+//              32*(w%4)..+31, so warps w and w+4 share the same 32 query rows:
+//              each takes one half (64 columns) of those rows' scores.  The
+//              two halves exchange their partial row maxima through shared
+//              memory behind a per-tile mbarrier; every thread then applies
+//              the same running max.  p = 2^(s*log2(e)/sqrt(d) - m) with the
+//              hardware ex2, element-wise arithmetic on packed fp32 pairs; the
+//              P of a half (fp16 pairs) is written over the first 32 columns of
+//              that half's own S region; O is rescaled in TMEM only when the
+//              running max grows by more than 8 (log2 units) - otherwise the
+//              stale max is kept for both O and the row sum, which leaves O/l
+//              unchanged.  Each half keeps its own partial row sum; the two are
+//              added at the end, and each half normalises and stores its 64
+//              output columns.
+//   warp 16    TMA producer: Q0, Q1 once, then K and V tiles into two 2-stage
+//              rings, K one tile ahead of V.
+//   warp 17    TMEM allocator + MMA issuer, in the order
 //                S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
-//              so that while one warpgroup computes its softmax the tensor core
-//              works on the other tile.  S = Q K^T reads both operands from
-//              shared memory (K-major); O += P V reads P from TMEM and V from
-//              shared memory as an MN-major operand.  tcgen05 MMAs of one
-//              thread execute in issue order, so S_t(j+1) cannot overwrite P_t(j)
-//              before PV_t(j) has read it, and when S_t(j) is signalled complete
-//              PV_t(j-1) has finished updating O_t (safe to rescale).
-// TMEM columns: S0/P0 [0,128), S1/P1 [128,256), O0 [256,384), O1 [384,512).
+//              so that while one tile's softmax runs the tensor core works on
+//              the other tile.  S = Q K^T reads both operands from shared
+//              memory (K-major); O += P V reads P from TMEM (keys 0-63 from the
+//              first S half, 64-127 from the second) and V from shared memory as
+//              an MN-major operand.  tcgen05 MMAs of one thread execute in issue
+//              order, so S_t(j+1) cannot overwrite P_t(j) before PV_t(j) has read
+//              it, and when S_t(j) is signalled complete PV_t(j-1) has finished
+//              updating O_t (safe to rescale).
+// TMEM columns: S0 [0,128) with P0 in [0,32) + [64,96), S1 [128,256) likewise,
+// O0 [256,384), O1 [384,512).
 //
 // Precision: Q, K, V arrive in fp16 and P is rounded to fp16 (11-bit
 // significand; |Q|, |K|, |V| of a unit-variance projection stay far below the
@@ -58,15 +63,18 @@ constexpr int kBox = 128 * 64 * 2;  // one TMA box: 128 rows x 64 fp16 (16 KB)
 constexpr int kQBytes = 2 * kBox;   // one Q tile: d in two 64-column boxes
 constexpr int kKBytes = 2 * kBox;   // one K tile (d in two boxes)
 constexpr int kVBytes = 2 * kBox;   // one V tile
-constexpr int kKStages = 3;         // K is needed a step before V: deeper ring
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreads = 576;
+constexpr int kSoftmaxWarps = 16;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr int kQOff = 0;
 constexpr int kKOff = kTiles * kQBytes;
 constexpr int kVOff = kKOff + kKStages * kKBytes;
-constexpr int kBarOff = kVOff + kVStages * kVBytes;
+constexpr int kXchOff = kVOff + kVStages * kVBytes;  // row-max exchange [tile][slot][half][128] + row sums [tile][half][128]
+constexpr int kXchBytes = (kTiles * 2 * 2 + kTiles * 2) * kBQ * 4;
+constexpr int kBarOff = kXchOff + kXchBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kColS0 = 0, kColO0 = 256;  // tile t: S at kColS0 + 128 t, O at kColO0 + 128 t
 constexpr uint32_t kIdescS = idesc_f32acc(kBQ, kBKV, false, false);  // fp16 Q, K
@@ -75,8 +83,8 @@ constexpr float kRescaleThreshold = 8.0f;                           // log2 unit
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-// 320 threads: ten warps, so some SM sub-partitions (16K registers each) hold
-// three of them, which caps a thread at 168 registers.
+// 576 threads: eighteen warps, so some SM sub-partitions (16K registers each)
+// hold five of them, which caps a thread at about 100 registers.
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qkv, const AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
@@ -91,7 +99,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = bars + 13;   // [2] per query tile
   uint64_t* o_done = bars + 15;   // [2] per query tile (after the last P.V)
   uint64_t* drain = bars + 17;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* xch = bars + 18;      // [2] per query tile: both halves' partial maxima written
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 20);
+  float* xmax = reinterpret_cast<float*>(smem + kXchOff);  // [tile][slot][half][row]
+  float* xsum = xmax + kTiles * 2 * 2 * kBQ;                // [tile][half][row]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -114,8 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 4);  // the four warps of that tile's softmax warpgroup
+      mbar_init(&p_full[s], 8);  // the eight softmax warps of that tile
       mbar_init(&o_done[s], 1);
+      mbar_init(&xch[s], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -202,8 +214,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a = tmem_base + kColS0 + uint32_t(t * 128);
 #pragma unroll
         for (int kk = 0; kk < kBKV / 16; ++kk) {
-          // 16 keys per step: P columns kk*8.. (fp16 pairs); rows kk*16.. of both V boxes
-          umma_ts(d, a + uint32_t(kk * 8), sdesc_sw128(sv + uint32_t(kk * 16 * 128), kBox, 1024), kIdescPV,
+          // 16 keys per step: P of keys 0-63 in columns [0,32), of keys 64-127 in
+          // [64,96) (fp16 pairs); rows kk*16.. of both V boxes
+          const uint32_t pcol = uint32_t((kk >> 2) * 64 + (kk & 3) * 8);
+          umma_ts(d, a + pcol, sdesc_sw128(sv + uint32_t(kk * 16 * 128), kBox, 1024), kIdescPV,
                   (j | kk) != 0 ? 1u : 0u);
         }
       };
@@ -254,63 +268,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 0-7)
-    const int t = warp >> 2;                                     // query tile of this warpgroup
+    // ------------------------------------------------------------ softmax (warps 0-15)
+    const int t = warp >> 3;                                     // query tile
+    const int h = (warp >> 2) & 1;                               // column half of the scores
+    const int rl = (warp & 3) * 32 + lane;                       // row within the tile (= TMEM lane)
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;  // TMEM lane quarter
-    const uint32_t colS = kColS0 + uint32_t(t * 128);
-    const uint32_t colO = kColO0 + uint32_t(t * 128);
-    const int row = qb * (kTiles * kBQ) + t * kBQ + (warp & 3) * 32 + lane;
+    const uint32_t colS = kColS0 + uint32_t(t * 128 + 64 * h);   // this half's S (and P) columns
+    const uint32_t colO = kColO0 + uint32_t(t * 128 + 64 * h);   // this half's O columns
+    const int row = qb * (kTiles * kBQ) + t * kBQ + rl;
     float m_run = -INFINITY;  // running max (log2-scaled units) used for O and l
-    float l_run = 0.f;
+    float l_run = 0.f;        // this half's partial row sum
     bool ok = true;
     const float sl2 = p.scale_log2;
+    const uint32_t ta = tmem_base + lane_off + colS;
     for (int j = 0; j < n_kv; ++j) {
       if (!mbar_wait(&s_full[t], j & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t ta = tmem_base + lane_off + colS;
-      const int kv0 = j * kBKV;
-      const bool ragged = kv0 + kBKV > p.M;  // last key tile: keys >= M do not exist
-      // Pass 1: row max.  All four loads in flight before one wait; eight
-      // independent max chains.
+      const int kv0 = j * kBKV + 64 * h;
+      const bool ragged = kv0 + 64 > p.M;  // keys >= M do not exist
+      // Pass 1: this half's row max (two loads in flight, eight max chains).
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
       {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
+        uint32_t r0[32], r1[32];
         tmem_ld32(ta, r0);
         tmem_ld32(ta + 32, r1);
-        tmem_ld32(ta + 64, r2);
-        tmem_ld32(ta + 96, r3);
         tmem_ld_wait();
         reg_fence32(r0);
         reg_fence32(r1);
-        reg_fence32(r2);
-        reg_fence32(r3);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           float v0 = __uint_as_float(r0[i]), v1 = __uint_as_float(r1[i]);
-          float v2 = __uint_as_float(r2[i]), v3 = __uint_as_float(r3[i]);
           if (ragged) {
             if (kv0 + i >= p.M) v0 = -INFINITY;
             if (kv0 + 32 + i >= p.M) v1 = -INFINITY;
-            if (kv0 + 64 + i >= p.M) v2 = -INFINITY;
-            if (kv0 + 96 + i >= p.M) v3 = -INFINITY;
           }
-          mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(fmaxf(v0, v1), fmaxf(v2, v3)));
+          mx8[i & 7] = fmaxf(mx8[i & 7], fmaxf(v0, v1));
         }
       }
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      mx *= sl2;
+      // Exchange the partial maxima of the two halves (slot j&1: a half can run
+      // at most one step ahead of its partner, so the slot it writes is free).
+      float* slot = xmax + ((t * 2 + (j & 1)) * 2) * kBQ;
+      slot[h * kBQ + rl] = mx;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xch[t]);
+      if (!mbar_wait(&xch[t], j & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      mx = fmaxf(mx, slot[(h ^ 1) * kBQ + rl]) * sl2;
       if (j == 0) {
         m_run = mx;
       } else {
-        // Rescale only rows whose max grew by more than the threshold; the TMEM
-        // accesses are warp-collective, so the whole warp takes the branch if any
-        // lane needs it (other lanes scale by 1).  O_t already holds P_t(j-1) V.
+        // Both halves see the same maxima, so they take the same decision.  Rescale
+        // only rows whose max grew by more than the threshold; the TMEM accesses are
+        // warp-collective, so the whole warp takes the branch if any lane needs it
+        // (other lanes scale by 1).  O_t already holds P_t(j-1) V.
         const bool need = mx > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
           const float alpha = need ? ex2_approx(m_run - mx) : 1.0f;
@@ -319,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             l_run *= alpha;
           }
 #pragma unroll 1
-          for (int c = 0; c < kD / 16; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t r[16];
             const uint32_t to = tmem_base + lane_off + colO + uint32_t(c * 16);
             tmem_ld16_sync(to, r);
@@ -329,23 +348,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      // Pass 2: p = 2^(s*scale - m), 32 scores at a time, on packed fp32 pairs.
-      // P chunk c goes to columns [16c, 16c+16), which only hold scores already read.
+      // Pass 2: p = 2^(s*scale - m), 32 scores at a time on packed fp32 pairs.
+      // P chunk c goes to columns [16c, 16c+16) of this half's region, which only
+      // hold scores this thread has already read.
       const uint64_t scale2 = f32x2(sl2, sl2);
       const uint64_t negm2 = f32x2(-m_run, -m_run);
       uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
-      uint32_t rc[32], rn[32];  // current chunk, next chunk (its load overlaps this chunk's math)
-      tmem_ld32(ta, rc);
-      tmem_ld_wait();
-      reg_fence32(rc);
 #pragma unroll
-      for (int c = 0; c < kBKV / 32; ++c) {
-        if (c + 1 < kBKV / 32) tmem_ld32(ta + uint32_t((c + 1) * 32), rn);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32_sync(ta + uint32_t(c * 32), r);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           float x0, x1;
-          f32x2_split(fma_f32x2(f32x2(__uint_as_float(rc[2 * i]), __uint_as_float(rc[2 * i + 1])), scale2, negm2),
+          f32x2_split(fma_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), scale2, negm2),
                       x0, x1);
           if (ragged) {
             if (kv0 + c * 32 + 2 * i >= p.M) x0 = -INFINITY;
@@ -356,14 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ls2[i & 3] = add_f32x2(ls2[i & 3], f32x2(p0, p1));
           pk[i] = pack_f16x2(p0, p1);
         }
-        // P chunk c -> columns [16c, 16c+16): scores there were read by chunks <= c
         tmem_st16(ta + uint32_t(c * 16), pk);
-        if (c + 1 < kBKV / 32) {
-          tmem_ld_wait();
-          reg_fence32(rn);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) rc[i] = rn[i];
-        }
       }
       {
         float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -380,11 +390,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) ok = mbar_wait(&o_done[t], 0, abort_flag);
     if (ok) {
+      // total row sum = both halves' partial sums (one more exchange phase)
+      float* xs = xsum + t * 2 * kBQ;
+      xs[h * kBQ + rl] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xch[t]);
+      ok = mbar_wait(&xch[t], n_kv & 1, abort_flag);
+      if (ok) l_run += xs[(h ^ 1) * kBQ + rl];
+    }
+    if (ok) {
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
-      uint16_t* orow = p.out + (int64_t(shard) * p.M + row) * int64_t(p.Hs * kD) + head * kD;
+      uint16_t* orow = p.out + (int64_t(shard) * p.M + row) * int64_t(p.Hs * kD) + head * kD + 64 * h;
 #pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
         tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(c * 32), r);
         uint4 o[4];
