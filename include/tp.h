@@ -172,11 +172,6 @@ tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s
 tp_status tp_sdpa_shards(const uint16_t* QKV, int64_t M, int heads, int tp_degree,
                          uint16_t* O, void* stream);
 
-/* Diagnostic: y[i] = 2^x[i] computed by the polynomial that the attention
- * kernel uses for part of its exponentials (fp32 in/out, device pointers), so
- * that its error can be checked against the exact value. */
-tp_status tp_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
-
 /* a8. Standalone partial-sum reduction (the per-element meaning of the
  * block-boundary AllReduce; the unfused alternative of a4):
  *   Y[M x N] = bf16( sum_{r ascending} parts[r] + bias )

@@ -54,7 +54,6 @@ SIGNATURES = {
     "tp_rowwise_linear_sum": (_I, [_P, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
     "tp_sdpa_shards": (_I, [_P, _I64, _I, _I, _P, _P]),
     "tp_reduce_partials": (_I, [_P, _I64, _I64, _I, _P, _P, _P]),
-    "tp_debug_exp2_poly": (_I, [_P, _P, _I64, _P]),
     "tp_mlp_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "tp_mlp_pair": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "tp_attn_workspace_bytes": (_SZ, [_I64, _I64, _I, _I]),
@@ -174,10 +173,6 @@ def tp_sdpa_shards(QKV, M, heads, tp_degree, O, stream=None) -> int:
 
 def tp_reduce_partials(parts, M, N, tp_degree, bias, Y, stream=None) -> int:
     return lib().tp_reduce_partials(_ptr(parts), M, N, tp_degree, _ptr(bias), _ptr(Y), _stream(stream))
-
-
-def tp_debug_exp2_poly(x, y, n, stream=None) -> int:
-    return lib().tp_debug_exp2_poly(_ptr(x), _ptr(y), n, _stream(stream))
 
 
 def tp_mlp_workspace_bytes(M, D, F, tp_degree) -> int:

@@ -506,14 +506,6 @@ tp_status tp_reduce_partials(const float* parts, int64_t M, int64_t N, int tp_de
                                                                                                    : TP_ERR_CUDA;
 }
 
-tp_status tp_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
-  if (!x || !y) return TP_ERR_NULL;
-  if (n < 0) return TP_ERR_BAD_SHAPE;
-  DeviceInfo* di = nullptr;
-  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
-  return launch_exp2_poly(x, y, n, as_stream(stream)) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
-}
-
 // ----------------------------------------------------------------------- MLP pair
 size_t tp_mlp_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree) {
   if (check_mlp_shape(M, D, F, tp_degree) != TP_OK) return 0;

@@ -73,9 +73,6 @@ struct AttnArgs {
 
 cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s);
 
-// y[i] = the attention kernel's FMA-pipe 2^x (exp2_poly), for testing its error.
-cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
-
 // Counts kernel launches (api.cu); every launcher calls it once per launch.
 void count_launch();
 
