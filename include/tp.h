@@ -91,6 +91,13 @@ const char* tp_last_error_message(void);
  * all threads); a telemetry counter for benchmarks. */
 uint64_t tp_kernel_launches(void);
 
+/* Failure-detection check: launches one CTA that waits, through the same
+ * bounded wait every kernel here uses, on an mbarrier that nothing arrives
+ * on.  The wait gives up after wait_ms (1..2000, else TP_ERR_BAD_SHAPE) and
+ * records a timeout, so a following tp_check_device_error() must return
+ * TP_ERR_DEVICE_TIMEOUT while the CUDA context stays usable. */
+tp_status tp_debug_watchdog(uint32_t wait_ms, void* stream);
+
 /* Synchronises `stream`, then reports (and clears) the device error word that
  * the kernels' bounded waits set: TP_OK, or TP_ERR_DEVICE_TIMEOUT.  Returns
  * TP_ERR_CUDA if the synchronisation itself fails. */

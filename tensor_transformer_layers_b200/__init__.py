@@ -44,6 +44,7 @@ SIGNATURES = {
     "tp_abi_version": (_I, []),
     "tp_last_error_message": (ctypes.c_char_p, []),
     "tp_check_device_error": (_I, [_P]),
+    "tp_debug_watchdog": (_I, [ctypes.c_uint32, _P]),
     "tp_shard_weight": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P]),
     "tp_shard_weight_all": (_I, [_P, _I64, _I64, _I, _I, _P, _P]),
     "tp_kernel_launches": (ctypes.c_uint64, []),
@@ -131,6 +132,10 @@ def tp_last_error_message() -> str:
 
 def tp_check_device_error(stream=None) -> int:
     return lib().tp_check_device_error(_stream(stream))
+
+
+def tp_debug_watchdog(wait_ms, stream=None) -> int:
+    return lib().tp_debug_watchdog(wait_ms, _stream(stream))
 
 
 def tp_shard_weight(W, rows, cols, style, tp_degree, rank, out, stream=None) -> int:

@@ -506,6 +506,15 @@ tp_status tp_reduce_partials(const float* parts, int64_t M, int64_t N, int tp_de
                                                                                                    : TP_ERR_CUDA;
 }
 
+tp_status tp_debug_watchdog(uint32_t wait_ms, void* stream) {
+  if (wait_ms < 1 || wait_ms > 2000) return TP_ERR_BAD_SHAPE;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return launch_watchdog_probe(di->err, uint64_t(wait_ms) * 1000000ull, as_stream(stream)) == cudaSuccess
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
 // ----------------------------------------------------------------------- MLP pair
 size_t tp_mlp_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree) {
   if (check_mlp_shape(M, D, F, tp_degree) != TP_OK) return 0;

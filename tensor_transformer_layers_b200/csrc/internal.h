@@ -73,6 +73,10 @@ struct AttnArgs {
 
 cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s);
 
+// One CTA whose bounded wait on an mbarrier that nothing arrives on must run
+// out after limit_ns and set kErrTimeout in *err (watchdog.cu).
+cudaError_t launch_watchdog_probe(int* err, uint64_t limit_ns, cudaStream_t s);
+
 // Counts kernel launches (api.cu); every launcher calls it once per launch.
 void count_launch();
 

@@ -13,6 +13,10 @@ namespace tp {
 // 10 ms), so a second means something is wrong.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
+// Backstop for the same waits that does not depend on the timer: at most this
+// many polling rounds (32 try_waits each).
+constexpr uint32_t kWaitMaxRounds = 1u << 21;
+
 // Device error word bits (OR-ed in by any CTA whose wait ran out).
 constexpr int kErrTimeout = 1;
 
@@ -62,19 +66,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Waits until the phase with the given parity has completed.  Bounded: gives
-// up (returns false) after kWaitLimitNs, or as soon as *abort is set by
-// another role of the CTA.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+// up (returns false) after `limit_ns` of %globaltimer or kWaitMaxRounds polling
+// rounds, whichever comes first, or as soon as *abort is set by another role
+// of the CTA.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, const volatile int* abort,
+                                              uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
+#pragma unroll 1
+  for (uint32_t round = 0; round < kWaitMaxRounds; ++round) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
+  return false;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // Records a timeout: device error word + the CTA-local abort flag.

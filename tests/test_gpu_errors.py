@@ -48,3 +48,25 @@ def test_rejected_calls_write_nothing():
     assert tp.tp_mlp_pair(d["X"], M, D, F, d["W_up"], d["b_up"], d["W_down"], d["b_down"], 2, Y, ws, nb) == 0
     assert tp.tp_check_device_error() == 0
     assert not np.all(from_dev(Y) == CANARY)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    # A wait on an mbarrier that nothing arrives on must give up after its limit,
+    # leave TP_ERR_DEVICE_TIMEOUT for the host and keep the context usable.
+    import time
+    assert tp.tp_check_device_error() == 0
+    t0 = time.perf_counter()
+    assert tp.tp_debug_watchdog(50) == 0
+    st = tp.tp_check_device_error()
+    dt = time.perf_counter() - t0
+    assert tp.STATUS[st] == "TP_ERR_DEVICE_TIMEOUT"
+    assert 0.04 < dt < 30.0
+    assert tp.tp_check_device_error() == 0  # the error word was cleared
+    # the library still works afterwards
+    M, D, F = 64, 128, 512
+    d = {k: to_dev(v) for k, v in syn.mlp_inputs(M, D, F, 0).items()}
+    Y = tp.mlp_pair(d["X"], d["W_up"], d["b_up"], d["W_down"], d["b_down"], 2)
+    torch.cuda.synchronize()
+    assert tp.tp_check_device_error() == 0
+    assert np.all(np.isfinite(syn.bf16_bits_to_f64(from_dev(Y))))
+    assert tp.tp_debug_watchdog(0) == S["TP_ERR_BAD_SHAPE"]
