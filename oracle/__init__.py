@@ -101,20 +101,50 @@ def slice_rowwise(W: np.ndarray, tp_degree: int, rank: int) -> np.ndarray:
     return W[:, rank * step:(rank + 1) * step].copy()
 
 
+def packed_block_sizes(dim: int, blocks: list[int], tp_degree: int) -> list[int]:
+    """Absolute block sizes of a packed dimension ("Fused projections" section).
+
+    ``blocks`` are proportional integers whose sum must divide the packed
+    dimension ([1, 1] for equal SwiGLU gate/up halves, [1, 1, 1, 3, 3] for a
+    fused Q, K, V, gate, up with mlp_ratio 3); absolute sizes, as stored on a
+    Linear, are the case where the sum equals the dimension.  Every block must
+    be divisible by the degree on its own, not only their sum ("Constraints and
+    validation" section)."""
+    if not blocks or any(b < 1 for b in blocks):
+        raise ValueError("packed blocks must be positive")
+    total = sum(blocks)
+    if dim % total != 0:
+        raise ValueError(f"sum of blocks {total} does not divide the packed dimension {dim}")
+    sizes = [b * (dim // total) for b in blocks]
+    for s in sizes:
+        check_divisible(s, tp_degree, "packed block")
+    return sizes
+
+
 def slice_packed_colwise(W: np.ndarray, blocks: list[int], tp_degree: int, rank: int) -> np.ndarray:
     """Packed colwise ("Fused projections" section): W's dim 0 is split into
-    consecutive blocks of the given sizes; each block is sliced colwise on its
-    own and the per-block slices are stacked in block order."""
+    consecutive blocks (proportions ``blocks``); each block is sliced colwise on
+    its own and the per-block slices are stacked in block order."""
     check_degree(tp_degree, rank)
-    if sum(blocks) != W.shape[0]:
-        raise ValueError("packed blocks do not add up to the packed dimension")
-    for b in blocks:
-        check_divisible(b, tp_degree, "packed block")
+    sizes = packed_block_sizes(W.shape[0], blocks, tp_degree)
     parts, start = [], 0
-    for b in blocks:
+    for b in sizes:
         parts.append(slice_colwise(W[start:start + b], tp_degree, rank))
         start += b
     return np.concatenate(parts, axis=0)
+
+
+def slice_packed_rowwise(W: np.ndarray, blocks: list[int], tp_degree: int, rank: int) -> np.ndarray:
+    """Packed rowwise: W's dim 1 is split into consecutive blocks; each block is
+    sliced rowwise on its own and the per-block slices are concatenated along
+    dim 1 in block order."""
+    check_degree(tp_degree, rank)
+    sizes = packed_block_sizes(W.shape[1], blocks, tp_degree)
+    parts, start = [], 0
+    for b in sizes:
+        parts.append(slice_rowwise(W[:, start:start + b], tp_degree, rank))
+        start += b
+    return np.concatenate(parts, axis=1)
 
 
 def slice_qkv_heads(W_qkv: np.ndarray, heads: int, tp_degree: int, rank: int) -> np.ndarray:
@@ -199,6 +229,51 @@ def mlp_sharded_summed(X, W_up, b_up, W_down, b_down, tp_degree, act=gelu_tanh):
         H_r = mlp_colwise_shard(X, W_up, b_up, tp_degree, r, act)
         parts.append(mlp_rowwise_partial(H_r, W_down, tp_degree, r))
     return reduce_partials(parts, b_down)
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU MLP pair: packed colwise [gate; up] (blocks [1, 1]) -> silu(gate) * up
+# -> rowwise FFN-out.  The packed form is the pages' SwiGLU example in the
+# "Fused projections" section; SiLU(x) = x * sigmoid(x) (Elfwing et al., 2018;
+# SwiGLU: Shazeer, 2020).
+# ---------------------------------------------------------------------------
+
+def silu(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def swiglu_unsharded(X, W_in, b_in, W_out, b_out):
+    """W_in = [W_gate; W_up] (2F x D), b_in = [b_gate; b_up] or None."""
+    F = W_in.shape[0] // 2
+    G = linear(X, W_in[:F], None if b_in is None else b_in[:F])
+    U = linear(X, W_in[F:], None if b_in is None else b_in[F:])
+    return linear(silu(G) * U, W_out, b_out)
+
+
+def swiglu_sharded_summed(X, W_in, b_in, W_out, b_out, tp_degree):
+    check_degree(tp_degree)
+    parts = []
+    for r in range(tp_degree):
+        Wr = slice_packed_colwise(W_in, [1, 1], tp_degree, r)  # [gate_r; up_r]
+        Fr = Wr.shape[0] // 2
+        br = None if b_in is None else slice_packed_colwise(b_in, [1, 1], tp_degree, r)
+        G = linear(X, Wr[:Fr], None if br is None else br[:Fr])
+        U = linear(X, Wr[Fr:], None if br is None else br[Fr:])
+        parts.append(linear(silu(G) * U, slice_rowwise(W_out, tp_degree, r)))
+    return reduce_partials(parts, b_out)
+
+
+# ---------------------------------------------------------------------------
+# rowwise_split_input (style table): a rowwise projection whose input is
+# replicated; each rank takes its slice of the input's features itself.
+# ---------------------------------------------------------------------------
+
+def rowwise_split_input(X, W, b, tp_degree):
+    """sum_r X[:, r-th K/T block] . W_r^T (+ b once)."""
+    check_degree(tp_degree)
+    parts = [linear(slice_rowwise(X, tp_degree, r), slice_rowwise(W, tp_degree, r)) for r in range(tp_degree)]
+    return reduce_partials(parts, b)
 
 
 # ---------------------------------------------------------------------------

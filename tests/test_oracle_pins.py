@@ -447,3 +447,90 @@ def test_block_rows_returns_exact_attention_and_mlp_of_rounded_input():
     assert np.allclose(A, A_full[rows], atol=1e-12)
     Y_want = o.mlp_unsharded(o.round_bf16(A_full[rows]), f["W_up"], f["b_up"], f["W_down"], f["b_down"])
     assert np.allclose(Y, Y_want, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Packed styles, SwiGLU pair, rowwise_split_input ("Fused projections" and the
+# style table's third row).
+# ---------------------------------------------------------------------------
+
+def test_packed_fixtures():
+    g = json.load(open(GOLDEN))
+    f = g["packed_colwise_fused_qkv_gate_up"]
+    W = np.arange(f["rows"])[:, None] * np.ones((1, 2), dtype=np.int64)
+    for r in range(f["tp_degree"]):
+        assert list(o.slice_packed_colwise(W, f["blocks"], f["tp_degree"], r)[:, 0]) == f[str(r)]
+    f = g["packed_rowwise_absolute"]
+    W = np.arange(f["cols"])[None, :]
+    for r in range(f["tp_degree"]):
+        assert list(o.slice_packed_rowwise(W, f["blocks"], f["tp_degree"], r)[0]) == f[str(r)]
+
+
+def test_packed_block_rules():
+    assert o.packed_block_sizes(36, [1, 1, 1, 3, 3], 2) == [4, 4, 4, 12, 12]
+    assert o.packed_block_sizes(12, [4, 8], 2) == [4, 8]         # absolute sizes
+    assert o.packed_block_sizes(12, [1, 2], 2) == [4, 8]         # proportional form of the same
+    with pytest.raises(ValueError):
+        o.packed_block_sizes(10, [1, 2], 1)                      # sum 3 does not divide 10
+    with pytest.raises(ValueError):
+        o.packed_block_sizes(18, [1, 1, 1, 3, 3], 3)             # blocks 2,2,2,6,6: 2 % 3 != 0
+    assert o.packed_block_sizes(12, [2, 1], 4) == [8, 4]         # each block divisible
+    with pytest.raises(ValueError):
+        o.packed_block_sizes(12, [5, 1], 4)                      # 10, 2: the sum 12 is divisible, the blocks are not
+
+
+def test_packed_equals_plain_for_one_block():
+    W = _rng(30).integers(0, 9, size=(12, 8))
+    for r in range(4):
+        assert np.array_equal(o.slice_packed_colwise(W, [1], 4, r), o.slice_colwise(W, 4, r))
+        assert np.array_equal(o.slice_packed_rowwise(W, [1], 4, r), o.slice_rowwise(W, 4, r))
+
+
+def test_silu_values():
+    x = np.array([0.0, 1.0, -1.0, 20.0, -20.0])
+    want = np.array([0.0, 1 / (1 + math.exp(-1)), -1 / (1 + math.exp(1)), 20 / (1 + math.exp(-20)),
+                     -20 / (1 + math.exp(20))])
+    assert np.allclose(o.silu(x), want, rtol=1e-15, atol=1e-300)
+    assert abs(o.silu(np.array([20.0]))[0] - 20.0) < 1e-6
+
+
+@pytest.mark.parametrize("T", [1, 2, 4])
+def test_swiglu_sharded_equals_unsharded(T):
+    rng = _rng(31 + T)
+    M, D, F = 5, 16, 32
+    X = rng.standard_normal((M, D))
+    W_in = rng.standard_normal((2 * F, D)) / 4
+    b_in = rng.standard_normal(2 * F) * 0.1
+    W_out = rng.standard_normal((D, F)) / 6
+    b_out = rng.standard_normal(D) * 0.1
+    full = o.swiglu_unsharded(X, W_in, b_in, W_out, b_out)
+    tp = o.swiglu_sharded_summed(X, W_in, b_in, W_out, b_out, T)
+    assert np.max(np.abs(tp - full)) <= 1e-12 * np.max(np.abs(full))
+
+
+def test_swiglu_closed_form():
+    # gate rows = 0 -> silu(0) = 0 -> output = b_out; up irrelevant.
+    rng = _rng(33)
+    M, D, F = 3, 8, 8
+    X = rng.standard_normal((M, D))
+    W_in = np.concatenate([np.zeros((F, D)), rng.standard_normal((F, D))])
+    b_out = rng.standard_normal(D)
+    Y = o.swiglu_sharded_summed(X, W_in, None, rng.standard_normal((D, F)), b_out, 2)
+    assert np.allclose(Y, np.tile(b_out, (M, 1)), atol=1e-14)
+    # gate = large positive constant c -> silu(c) ~ c, so H ~ c * up
+    c = 30.0
+    W_g = np.zeros((F, D))
+    b_in = np.concatenate([np.full(F, c), np.zeros(F)])
+    W_u = rng.standard_normal((F, D))
+    W_out = rng.standard_normal((D, F))
+    Y = o.swiglu_sharded_summed(X, np.concatenate([W_g, W_u]), b_in, W_out, None, 2)
+    assert np.allclose(Y, c * (X @ W_u.T) @ W_out.T, rtol=1e-9)
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 6])
+def test_rowwise_split_input_is_the_full_projection(T):
+    rng = _rng(40 + T)
+    X = rng.integers(-3, 4, size=(4, 12)).astype(np.float64)
+    W = rng.integers(-3, 4, size=(7, 12)).astype(np.float64)
+    b = rng.integers(-3, 4, size=7).astype(np.float64)
+    assert np.array_equal(o.rowwise_split_input(X, W, b, T), X @ W.T + b)
