@@ -11,11 +11,14 @@ duration is measured with CUDA events inside the timed region (a GPU test
 checks that the sequence is bit-identical to ``tp_mlp_pair``).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                       [--workload flux_mlp|flux_attn|wide_block|flux_reduce]
+                       [--workload flux_mlp|flux_attn|wide_block|flux_reduce|flux_swiglu|
+                                   flux_split_input]
 The default workload (flux_mlp) is the headline line.  The others time the
 remaining rows the same way: flux_attn (QKV head split, QKV GEMM, SDPA,
 out-projection), wide_block (attention then MLP pair at tp_degree 8, every
-row) and flux_reduce (the standalone partial-sum reduction, GB/s).
+row), flux_reduce (the standalone partial-sum reduction, GB/s), flux_swiglu
+(the SwiGLU pair: packed gate/up slicing, SwiGLU colwise GEMM, rowwise GEMM)
+and flux_split_input (rowwise_split_input on an FFN-out-sized projection).
 Under torchrun (N > 1) every rank runs the same workload on its own tokens
 (independent replicas: the layer pair has no exchange step when all shards of
 a layer live on one GPU), so per-GPU work is fixed ("weak" scaling) and the
@@ -500,7 +503,162 @@ class ReduceWorkload(MlpWorkload):
                 "M": c["M"], "N": c["N"], "tp_degree": c["T"], "global_batch_tokens": c["M"] * world}
 
 
-WORKLOADS = {w.key: w for w in (MlpWorkload, AttnWorkload, BlockWorkload, ReduceWorkload)}
+class SwigluWorkload(MlpWorkload):
+    """flux_swiglu: the SwiGLU pair with gate and up packed (blocks [1, 1]):
+    packed colwise slicing, the SwiGLU colwise GEMM, the rowwise GEMM."""
+    key = "flux_swiglu"
+    metric = "TP SwiGLU MLP-pair bf16 TFLOP/s on 1 B200"
+
+    def __init__(self, cfg=None):
+        import synthetic as syn
+        self.cfg = cfg or syn.CONFIGS["flux_swiglu"]
+
+    def host_inputs(self, rank):
+        import synthetic as syn
+        c = self.cfg
+        d = syn.swiglu_inputs(c["M"], c["D"], c["F"], c["seed"])
+        if rank:
+            d["X"] = syn.normal_bf16((c["M"], c["D"]), 1.0, seed=c["seed"] + 1000 * rank, tid=syn.TID["X"])
+        return d
+
+    def work(self):
+        c = self.cfg
+        return 6.0 * c["M"] * c["D"] * c["F"]  # 2 M D (2F) for gate+up, 2 M F D for the out-projection
+
+    def kernels(self, tp, g, dev):
+        import torch
+        M, D, F, T = self.cfg["M"], self.cfg["D"], self.cfg["F"], self.cfg["T"]
+        Fs = F // T
+        b = {"w_in": torch.empty((T, 2 * Fs, D), dtype=torch.int16, device=dev),
+             "b_in": torch.empty((T, 2 * Fs), dtype=torch.int16, device=dev),
+             "w_out": torch.empty((T, D, Fs), dtype=torch.int16, device=dev),
+             "H": torch.empty((T, M, Fs), dtype=torch.int16, device=dev),
+             "Y": torch.empty((M, D), dtype=torch.int16, device=dev)}
+        ck = tp._check
+        self.bufs = b
+        return [
+            Kernel("slice_w_in", "GB/s", 2.0 * 2 * F * D * 2,
+                   lambda: ck(tp.tp_shard_packed_all(g["W_in"], 2 * F, D, tp.TP_COLWISE, [1, 1], T, b["w_in"]),
+                              "slice W_in")),
+            Kernel("slice_b_in", "GB/s", 2.0 * 2 * F * 2,
+                   lambda: ck(tp.tp_shard_packed_all(g["b_in"], 1, 2 * F, tp.TP_ROWWISE, [1, 1], T, b["b_in"]),
+                              "slice b_in")),
+            Kernel("slice_w_out", "GB/s", 2.0 * D * F * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["W_out"], D, F, tp.TP_ROWWISE, T, b["w_out"]),
+                              "slice W_out")),
+            Kernel("colwise_swiglu", "TFLOP/s", 2.0 * M * D * 2 * F,
+                   lambda: ck(tp.tp_colwise_swiglu(g["X"], M, D, b["w_in"], b["b_in"], Fs, T, b["H"]),
+                              "colwise swiglu")),
+            Kernel("rowwise_gemm", "TFLOP/s", 2.0 * M * F * D,
+                   lambda: ck(tp.tp_rowwise_linear_sum(b["H"], M, Fs, b["w_out"], D, g["b_out"], T, b["Y"]),
+                              "rowwise")),
+        ]
+
+    def one_shot(self, tp, gi, dev):
+        import torch
+        M, D, F, T = self.cfg["M"], self.cfg["D"], self.cfg["F"], self.cfg["T"]
+        if not hasattr(self, "_ws"):
+            self._ws = torch.empty(tp.tp_swiglu_workspace_bytes(M, D, F, T), dtype=torch.uint8, device=dev)
+            self._y = torch.empty((M, D), dtype=torch.int16, device=dev)
+        tp._check(tp.tp_swiglu_mlp_pair(gi["X"], M, D, F, gi["W_in"], gi["b_in"], gi["W_out"], gi["b_out"], T,
+                                        self._y, self._ws, self._ws.numel()), "tp_swiglu_mlp_pair")
+        return self._y
+
+    e2e_call = "tp_swiglu_mlp_pair with X, W_in, b_in, W_out, b_out copied from pinned host memory and Y copied back"
+
+    def oracle_run(self, d, rows):
+        import oracle as o
+        import synthetic as syn
+        c = self.cfg
+        f = _f64(d, ["W_in", "b_in", "W_out", "b_out"])
+        X = syn.bf16_bits_to_f64(d["X"][:rows])
+        t0 = time.perf_counter()
+        o.swiglu_sharded_summed(X, f["W_in"], f["b_in"], f["W_out"], f["b_out"], c["T"])
+        return time.perf_counter() - t0, 6.0 * rows * c["D"] * c["F"]
+
+    oracle_fn = "swiglu_sharded_summed"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": (f"flux_swiglu: TP SwiGLU pair (gate/up packed colwise with blocks [1, 1], "
+                             f"silu(gate) * up fused in the colwise epilogue, rowwise out-projection with the "
+                             f"cross-shard sum fused); M={c['M']}, D={c['D']}, F={c['F']} (mlp_ratio 3)"),
+                "M": c["M"], "D": c["D"], "F": c["F"], "tp_degree": c["T"],
+                "global_batch_tokens": c["M"] * world}
+
+
+class SplitInputWorkload(MlpWorkload):
+    """flux_split_input: rowwise_split_input, the replicated input sliced by TMA
+    coordinates inside the rowwise GEMM (FFN-out sized)."""
+    key = "flux_split_input"
+    metric = "TP rowwise_split_input bf16 TFLOP/s on 1 B200"
+
+    def __init__(self, cfg=None):
+        import synthetic as syn
+        c = syn.CONFIGS["flux_mlp"]
+        self.cfg = cfg or dict(M=c["M"], K=c["F"], N=c["D"], T=c["T"], seed=5)
+
+    def host_inputs(self, rank):
+        import numpy as np
+        import synthetic as syn
+        c = self.cfg
+        return {"X": syn.normal_bf16((c["M"], c["K"]), 1.0, c["seed"] + 1000 * rank, syn.TID["X"]),
+                "W": syn.normal_bf16((c["N"], c["K"]), 1.0 / np.sqrt(c["K"]), c["seed"], syn.TID["W_down"]),
+                "b": syn.normal_bf16((c["N"],), 0.02, c["seed"], syn.TID["b_down"])}
+
+    def work(self):
+        c = self.cfg
+        return 2.0 * c["M"] * c["K"] * c["N"]
+
+    def kernels(self, tp, g, dev):
+        import torch
+        M, K, N, T = self.cfg["M"], self.cfg["K"], self.cfg["N"], self.cfg["T"]
+        b = {"w": torch.empty((T, N, K // T), dtype=torch.int16, device=dev),
+             "Y": torch.empty((M, N), dtype=torch.int16, device=dev)}
+        ck = tp._check
+        self.bufs = b
+        return [
+            Kernel("slice_w", "GB/s", 2.0 * N * K * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["W"], N, K, tp.TP_ROWWISE_SPLIT_INPUT, T, b["w"]),
+                              "slice W")),
+            Kernel("split_input_gemm", "TFLOP/s", self.work(),
+                   lambda: ck(tp.tp_rowwise_split_input_linear(g["X"], M, K, b["w"], N, g["b"], T, b["Y"]),
+                              "split input")),
+        ]
+
+    def one_shot(self, tp, gi, dev):
+        M, K, N, T = self.cfg["M"], self.cfg["K"], self.cfg["N"], self.cfg["T"]
+        ck = tp._check
+        ck(tp.tp_shard_weight_all(gi["W"], N, K, tp.TP_ROWWISE_SPLIT_INPUT, T, self.bufs["w"]), "slice W")
+        ck(tp.tp_rowwise_split_input_linear(gi["X"], M, K, self.bufs["w"], N, gi["b"], T, self.bufs["Y"]),
+           "split input")
+        return self.bufs["Y"]
+
+    e2e_call = ("tp_shard_weight_all + tp_rowwise_split_input_linear with X, W, b copied from pinned host memory "
+                "and Y copied back")
+
+    def oracle_run(self, d, rows):
+        import oracle as o
+        import synthetic as syn
+        c = self.cfg
+        W = syn.bf16_bits_to_f64(d["W"])
+        b = syn.bf16_bits_to_f64(d["b"])
+        X = syn.bf16_bits_to_f64(d["X"][:rows])
+        t0 = time.perf_counter()
+        o.rowwise_split_input(X, W, b, c["T"])
+        return time.perf_counter() - t0, 2.0 * rows * c["K"] * c["N"]
+
+    oracle_fn = "rowwise_split_input"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": (f"flux_split_input: rowwise_split_input (replicated input, each shard reads its "
+                             f"K/T columns in place), M={c['M']}, K={c['K']}, N={c['N']}"),
+                "M": c["M"], "K": c["K"], "N": c["N"], "tp_degree": c["T"], "global_batch_tokens": c["M"] * world}
+
+
+WORKLOADS = {w.key: w for w in (MlpWorkload, AttnWorkload, BlockWorkload, ReduceWorkload, SwigluWorkload,
+                                SplitInputWorkload)}
 
 
 def workload_cfg():

@@ -15,6 +15,11 @@
  *     Q/K/V give each rank a subset of the heads;
  *   - section "Fused projections": a Linear that packs several tensors along
  *     the sharded dimension is sharded block by block (Q/K/V: blocks [1,1,1]);
+ *   - section "Fused projections" also gives the SwiGLU gate/up pair packed
+ *     with blocks [1, 1], proportional blocks (e.g. [1, 1, 1, 3, 3]) or
+ *     absolute sizes stored on the Linear, and packed rowwise;
+ *   - style table, third row: "rowwise_split_input", a rowwise projection
+ *     whose input is replicated, each rank slicing its part of the input;
  *   - section "Constraints and validation": the degree must divide the head
  *     count and every packed block, checked before any weight is split.
  *
@@ -64,12 +69,15 @@ typedef enum {
   TP_ERR_DEVICE_TIMEOUT = 10,    /* a kernel's bounded wait ran out (see tp_check_device_error) */
   TP_ERR_BAD_STYLE = 11,         /* unknown tp_style */
   TP_ERR_BAD_HANDLE = 12,        /* NULL or foreign handle */
-  TP_ERR_SCRATCH_LIMIT = 13      /* problem too large for the no-allocation entry point's fixed scratch */
+  TP_ERR_SCRATCH_LIMIT = 13,     /* problem too large for the no-allocation entry point's fixed scratch */
+  TP_ERR_BAD_BLOCKS = 14         /* packed blocks: count outside 1..64, a block < 1, or sum not dividing the dim */
 } tp_status;
 
 typedef enum {
-  TP_COLWISE = 0, /* slice output features: rows [r*N/T, (r+1)*N/T) of W[N x K] */
-  TP_ROWWISE = 1  /* slice input features: columns [r*K/T, (r+1)*K/T) of every row */
+  TP_COLWISE = 0,             /* slice output features: rows [r*N/T, (r+1)*N/T) of W[N x K] */
+  TP_ROWWISE = 1,             /* slice input features: columns [r*K/T, (r+1)*K/T) of every row */
+  TP_ROWWISE_SPLIT_INPUT = 2  /* weight sliced as TP_ROWWISE; the replicated input is sliced by
+                                 tp_rowwise_split_input_linear itself */
 } tp_style;
 
 /* Storage type of a 16-bit activation output. */
@@ -108,7 +116,8 @@ tp_status tp_check_device_error(void* stream);
  * Bit-exact copies; a coalesced 128-bit vectorised HBM copy kernel.
  * ------------------------------------------------------------------------- */
 
-/* out = slice `rank` of W[rows x cols] in `style`.
+/* out = slice `rank` of W[rows x cols] in `style` (TP_ROWWISE_SPLIT_INPUT
+ * slices like TP_ROWWISE).
  *   colwise: out is [rows/T x cols] = W[rank*rows/T : (rank+1)*rows/T, :]
  *   rowwise: out is [rows x cols/T] = W[:, rank*cols/T : (rank+1)*cols/T]
  * Errors: NULL, BAD_STYLE, BAD_DEGREE, BAD_RANK, BAD_SHAPE (rows or cols < 1),
@@ -143,6 +152,30 @@ tp_status tp_shard_qkv_heads(const uint16_t* W_qkv, int64_t D, int heads, int tp
 tp_status tp_shard_qkv_heads_all(const uint16_t* W_qkv, int64_t D, int heads, int tp_degree,
                                  uint16_t* out, void* stream);
 
+/* Packed colwise / rowwise ("Fused projections").  W's packed dimension
+ * (dim 0 = rows for TP_COLWISE, dim 1 = cols for TP_ROWWISE) is the
+ * concatenation of nblocks blocks.  blocks[] (HOST memory, 1 <= nblocks <= 64)
+ * are positive proportional integers whose sum divides the packed dimension
+ * P; block b has size S_b = blocks[b] * P / sum (absolute sizes, as stored on
+ * a Linear, are the case sum == P).  Each block is sliced on its own and the
+ * slices follow one another in block order:
+ *   colwise: out is [P/T x cols]: rows [start_b + rank*S_b/T, +S_b/T) of each block;
+ *   rowwise: out is [rows x P/T]: those columns of each block.
+ * The bias of a packed colwise layer is sliced as a 1 x n matrix with
+ * TP_ROWWISE.  Errors, all before any launch: NULL, BAD_STYLE (only
+ * TP_COLWISE / TP_ROWWISE), BAD_DEGREE, BAD_RANK, BAD_SHAPE, BAD_BLOCKS,
+ * INDIVISIBLE (some S_b % T != 0, even when P % T == 0), ALIGNMENT (cols % 8;
+ * rowwise: every S_b/T % 8).  One copy launch per block. */
+tp_status tp_shard_packed(const uint16_t* W, int64_t rows, int64_t cols, int style,
+                          const int64_t* blocks, int nblocks, int tp_degree, int rank,
+                          uint16_t* out, void* stream);
+
+/* All T packed shards, stacked in rank order: out is [T x (shard shape)].
+ * Same checks as tp_shard_packed (without `rank`); one launch per block. */
+tp_status tp_shard_packed_all(const uint16_t* W, int64_t rows, int64_t cols, int style,
+                              const int64_t* blocks, int nblocks, int tp_degree,
+                              uint16_t* out, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Step-level calls (each one kernel), on already-sharded operands.
  * ------------------------------------------------------------------------- */
@@ -168,6 +201,31 @@ tp_status tp_colwise_linear(const uint16_t* X, int64_t M, int64_t K,
 tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s,
                                 const uint16_t* W_shards, int64_t N, const uint16_t* bias,
                                 int tp_degree, uint16_t* Y, void* stream);
+
+/* SwiGLU colwise GEMM for every shard (the gate/up pair packed with blocks
+ * [1, 1], section "Fused projections"):
+ *   out[r] = silu(X W_gate,r^T + bg_r) * (X W_up,r^T + bu_r),   r = 0..T-1
+ * W_shards: [T x 2F_s x K], shard r = [W_gate,r; W_up,r] (F_s rows each: what
+ * tp_shard_packed_all(..., TP_COLWISE, {1, 1}, ...) produces); b_shards:
+ * [T x 2F_s] = [bg_r, bu_r] per shard, or NULL; out: [T x M x F_s] bf16.
+ * silu(x) = x * sigmoid(x).  Both halves accumulate in one tcgen05 tile
+ * (gate and up columns side by side in tensor memory) and the product is
+ * formed in the epilogue, so neither half is ever written out.
+ * Requires K % 8 == 0 and F_s % 8 == 0 (ALIGNMENT).  M == 0 is a no-op. */
+tp_status tp_colwise_swiglu(const uint16_t* X, int64_t M, int64_t K,
+                            const uint16_t* W_shards, const uint16_t* b_shards, int64_t F_s,
+                            int tp_degree, uint16_t* out, void* stream);
+
+/* rowwise_split_input (style table, third row): a rowwise projection whose
+ * input is replicated.  Each shard takes its own K/T columns of X:
+ *   Y[M x N] = bf16( sum_r X[:, r*K/T : (r+1)*K/T] . W_shards[r]^T + bias )
+ * X: [M x K] (the replicated input, read in place: the slice is a TMA
+ * coordinate, not a copy); W_shards: [T x N x K/T] (TP_ROWWISE slices of
+ * W[N x K]); bias [N] or NULL, added once.  K % T == 0 (INDIVISIBLE);
+ * K/T % 8 == 0 and N % 8 == 0 (ALIGNMENT). */
+tp_status tp_rowwise_split_input_linear(const uint16_t* X, int64_t M, int64_t K,
+                                        const uint16_t* W_shards, int64_t N, const uint16_t* bias,
+                                        int tp_degree, uint16_t* Y, void* stream);
 
 /* a6. Per-shard scaled dot-product attention, non-causal, scale 1/sqrt(128):
  * QKV: fp16 [T x M x 3*Hs*128] with Hs = heads/T; inside a row: Q heads,
@@ -203,6 +261,17 @@ tp_status tp_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F,
                       const uint16_t* W_down, const uint16_t* b_down,
                       int tp_degree, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
 
+/* SwiGLU MLP pair: Y = bf16( sum_r (silu(X W_gate,r^T + bg_r) * (X W_up,r^T + bu_r)) W_out,r^T + b_out ).
+ * X[M x D]; W_in[2F x D] = [W_gate; W_up] (packed colwise, blocks [1, 1]);
+ * b_in[2F] = [b_gate, b_up] or NULL; W_out[D x F] (rowwise); b_out[D] or
+ * NULL; Y[M x D].  F % T == 0 (INDIVISIBLE); D and F/T multiples of 8
+ * (ALIGNMENT).  Workspace: tp_swiglu_workspace_bytes(). */
+size_t tp_swiglu_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree);
+tp_status tp_swiglu_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F,
+                             const uint16_t* W_in, const uint16_t* b_in,
+                             const uint16_t* W_out, const uint16_t* b_out,
+                             int tp_degree, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
 /* Attention block: Y = bf16( sum_r O_r W_o,r^T ), O_r = per-shard SDPA of the
  * head-split QKV projection X W_qkv,r^T.  X[M x D], W_qkv[3D x D], W_o[D x D],
  * Y[M x D]; D == heads*128; heads % T == 0.  No biases.
@@ -219,6 +288,11 @@ tp_status tp_attn_block(const uint16_t* X, int64_t M, int64_t D,
 tp_status tp_mlp_prepare(const uint16_t* W_up, const uint16_t* b_up,
                          const uint16_t* W_down, const uint16_t* b_down,
                          int64_t D, int64_t F, int tp_degree, void* stream, void** handle);
+/* The SwiGLU pair's load-once form; arguments as tp_swiglu_mlp_pair.  The
+ * handle runs through tp_mlp_run with tp_mlp_run_workspace_bytes. */
+tp_status tp_swiglu_prepare(const uint16_t* W_in, const uint16_t* b_in,
+                            const uint16_t* W_out, const uint16_t* b_out,
+                            int64_t D, int64_t F, int tp_degree, void* stream, void** handle);
 size_t tp_mlp_run_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree);
 tp_status tp_mlp_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y,
                      void* ws, size_t ws_bytes, void* stream);

@@ -39,6 +39,7 @@ TID = {
     "X": 0, "W_up": 1, "b_up": 2, "W_down": 3, "b_down": 4,
     "W_qkv": 5, "W_o": 6,
     "W_up2": 7, "b_up2": 8, "W_down2": 9, "b_down2": 10,
+    "W_in": 11, "b_in": 12, "W_out": 13, "b_out": 14,
 }
 
 _CHUNK = 1 << 22
@@ -157,11 +158,25 @@ def block_inputs(M: int, D: int, F: int, seed: int) -> dict:
     return d
 
 
-# The five layer configurations exercised by the tests and the benchmark.
+def swiglu_inputs(M: int, D: int, F: int, seed: int) -> dict:
+    """Inputs of a SwiGLU pair: X[M,D], W_in[2F,D] = [W_gate; W_up], b_in[2F],
+    W_out[D,F], b_out[D] (same scales as the GELU pair)."""
+    return {
+        "X": normal_bf16((M, D), 1.0, seed, TID["X"]),
+        "W_in": normal_bf16((2 * F, D), 1.0 / np.sqrt(D), seed, TID["W_in"]),
+        "b_in": normal_bf16((2 * F,), 0.02, seed, TID["b_in"]),
+        "W_out": normal_bf16((D, F), 1.0 / np.sqrt(F), seed, TID["W_out"]),
+        "b_out": normal_bf16((D,), 0.02, seed, TID["b_out"]),
+    }
+
+
+# The layer configurations exercised by the tests and the benchmark.
 CONFIGS = {
     "tiny_mlp": dict(kind="mlp", M=64, D=128, F=512, T=2, seed=0),
     "flux_mlp": dict(kind="mlp", M=4608, D=3072, F=12288, T=4, seed=1),
     "flux_attn": dict(kind="attn", M=4608, D=3072, H=24, T=4, seed=2),
     "flux_mlp_sweep": dict(kind="mlp", M=4608, D=3072, F=12288, T=(1, 2, 4, 8), seed=1),
     "wide_block": dict(kind="block", M=16384, D=6144, H=48, F=24576, T=8, seed=3),
+    # SwiGLU pair, gate and up packed with blocks [1, 1], mlp_ratio 3 (F = 3 D)
+    "flux_swiglu": dict(kind="swiglu", M=4608, D=3072, F=9216, T=4, seed=4),
 }

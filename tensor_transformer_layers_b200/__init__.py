@@ -6,9 +6,9 @@ sizes through ctypes.  Nothing here computes: every step of every layer runs
 in the CUDA kernels of ``libtp.so``.  If the library is missing this module
 raises on first use; there is no fallback.
 
-The convenience wrappers at the end (``mlp_pair``, ``attn_block``,
-``MlpPair``, ``AttnBlock``) only allocate outputs and workspaces with torch
-and call the C entry points.
+The convenience wrappers at the end (``mlp_pair``, ``swiglu_mlp_pair``,
+``attn_block``, ``MlpPair``, ``AttnBlock``) only allocate outputs and
+workspaces with torch and call the C entry points.
 """
 from __future__ import annotations
 
@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libtp.so")
 
 TP_COLWISE = 0
 TP_ROWWISE = 1
+TP_ROWWISE_SPLIT_INPUT = 2
 TP_OUT_BF16 = 0
 TP_OUT_F16 = 1
 
@@ -30,7 +31,7 @@ STATUS = {
     4: "TP_ERR_INDIVISIBLE", 5: "TP_ERR_HEADS_INDIVISIBLE", 6: "TP_ERR_BAD_SHAPE",
     7: "TP_ERR_ALIGNMENT", 8: "TP_ERR_WORKSPACE", 9: "TP_ERR_CUDA",
     10: "TP_ERR_DEVICE_TIMEOUT", 11: "TP_ERR_BAD_STYLE", 12: "TP_ERR_BAD_HANDLE",
-    13: "TP_ERR_SCRATCH_LIMIT",
+    13: "TP_ERR_SCRATCH_LIMIT", 14: "TP_ERR_BAD_BLOCKS",
 }
 
 _P = ctypes.c_void_p
@@ -67,6 +68,13 @@ SIGNATURES = {
     "tp_attn_run": (_I, [_P, _P, _I64, _P, _P, _SZ, _P]),
     "tp_destroy": (None, [_P]),
     "tp_mlp_pair_sharded_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _P]),
+    "tp_shard_packed": (_I, [_P, _I64, _I64, _I, ctypes.POINTER(_I64), _I, _I, _I, _P, _P]),
+    "tp_shard_packed_all": (_I, [_P, _I64, _I64, _I, ctypes.POINTER(_I64), _I, _I, _P, _P]),
+    "tp_colwise_swiglu": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _P, _P]),
+    "tp_rowwise_split_input_linear": (_I, [_P, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
+    "tp_swiglu_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
+    "tp_swiglu_mlp_pair": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "tp_swiglu_prepare": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _P, ctypes.POINTER(_P)]),
 }
 
 _lib = None
@@ -240,6 +248,50 @@ def tp_mlp_pair_sharded_noalloc(X, M, D, F, W_up_shards, b_up_shards, W_down_sha
                                              _stream(stream))
 
 
+def _blocks(blocks):
+    """Host int64 array for a packed call (None stays NULL)."""
+    if blocks is None:
+        return None, 0
+    blocks = [int(b) for b in blocks]
+    return (_I64 * max(len(blocks), 1))(*blocks), len(blocks)
+
+
+def tp_shard_packed(W, rows, cols, style, blocks, tp_degree, rank, out, stream=None) -> int:
+    arr, n = _blocks(blocks)
+    return lib().tp_shard_packed(_ptr(W), rows, cols, style, arr, n, tp_degree, rank, _ptr(out), _stream(stream))
+
+
+def tp_shard_packed_all(W, rows, cols, style, blocks, tp_degree, out, stream=None) -> int:
+    arr, n = _blocks(blocks)
+    return lib().tp_shard_packed_all(_ptr(W), rows, cols, style, arr, n, tp_degree, _ptr(out), _stream(stream))
+
+
+def tp_colwise_swiglu(X, M, K, W_shards, b_shards, F_s, tp_degree, out, stream=None) -> int:
+    return lib().tp_colwise_swiglu(_ptr(X), M, K, _ptr(W_shards), _ptr(b_shards), F_s, tp_degree, _ptr(out),
+                                   _stream(stream))
+
+
+def tp_rowwise_split_input_linear(X, M, K, W_shards, N, bias, tp_degree, Y, stream=None) -> int:
+    return lib().tp_rowwise_split_input_linear(_ptr(X), M, K, _ptr(W_shards), N, _ptr(bias), tp_degree, _ptr(Y),
+                                               _stream(stream))
+
+
+def tp_swiglu_workspace_bytes(M, D, F, tp_degree) -> int:
+    return lib().tp_swiglu_workspace_bytes(M, D, F, tp_degree)
+
+
+def tp_swiglu_mlp_pair(X, M, D, F, W_in, b_in, W_out, b_out, tp_degree, Y, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_swiglu_mlp_pair(_ptr(X), M, D, F, _ptr(W_in), _ptr(b_in), _ptr(W_out), _ptr(b_out), tp_degree,
+                                    _ptr(Y), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def tp_swiglu_prepare(W_in, b_in, W_out, b_out, D, F, tp_degree, stream=None):
+    h = _P()
+    st = lib().tp_swiglu_prepare(_ptr(W_in), _ptr(b_in), _ptr(W_out), _ptr(b_out), D, F, tp_degree,
+                                 _stream(stream), ctypes.byref(h))
+    return st, h.value
+
+
 # --------------------------------------------------------------------------- convenience
 def _u16(t: torch.Tensor) -> torch.Tensor:
     """bf16 bit patterns travel as 16-bit tensors; accept bfloat16 or int16/uint16 storage."""
@@ -266,6 +318,19 @@ def mlp_pair(X, W_up, b_up, W_down, b_down, tp_degree: int, stream=None) -> torc
     return Y
 
 
+def swiglu_mlp_pair(X, W_in, b_in, W_out, b_out, tp_degree: int, stream=None) -> torch.Tensor:
+    """One-shot SwiGLU pair, W_in = [W_gate; W_up]; returns Y [M, D] (bf16)."""
+    _u16(X), _u16(W_in), _u16(W_out)
+    M, D = X.shape
+    F = W_in.shape[0] // 2
+    Y = torch.empty((M, D), dtype=torch.bfloat16, device=X.device)
+    nb = tp_swiglu_workspace_bytes(M, D, F, tp_degree)
+    ws = _workspace(nb, X.device)
+    _check(tp_swiglu_mlp_pair(X, M, D, F, W_in, b_in, W_out, b_out, tp_degree, Y, ws, nb, stream),
+           "tp_swiglu_mlp_pair")
+    return Y
+
+
 def attn_block(X, W_qkv, W_o, heads: int, tp_degree: int, stream=None) -> torch.Tensor:
     """One-shot attention block; returns Y [M, D] (bf16)."""
     _u16(X), _u16(W_qkv), _u16(W_o)
@@ -278,14 +343,23 @@ def attn_block(X, W_qkv, W_o, heads: int, tp_degree: int, stream=None) -> torch.
 
 
 class MlpPair:
-    """Shards once (tp_mlp_prepare), runs many times (tp_mlp_run)."""
+    """Shards once (tp_mlp_prepare, or tp_swiglu_prepare with
+    activation="swiglu" and W_up = [W_gate; W_up]), runs many times (tp_mlp_run)."""
 
-    def __init__(self, W_up, b_up, W_down, b_down, tp_degree: int, stream=None):
+    def __init__(self, W_up, b_up, W_down, b_down, tp_degree: int, stream=None, activation: str = "gelu"):
         self.D = W_up.shape[1]
-        self.F = W_up.shape[0]
         self.T = tp_degree
-        st, self.handle = tp_mlp_prepare(W_up, b_up, W_down, b_down, self.D, self.F, tp_degree, stream)
-        _check(st, "tp_mlp_prepare")
+        self.handle = None
+        if activation == "gelu":
+            self.F = W_up.shape[0]
+            st, self.handle = tp_mlp_prepare(W_up, b_up, W_down, b_down, self.D, self.F, tp_degree, stream)
+            _check(st, "tp_mlp_prepare")
+        elif activation == "swiglu":
+            self.F = W_up.shape[0] // 2
+            st, self.handle = tp_swiglu_prepare(W_up, b_up, W_down, b_down, self.D, self.F, tp_degree, stream)
+            _check(st, "tp_swiglu_prepare")
+        else:
+            raise ValueError(f"unknown activation {activation!r}")
         self._ws = None
 
     def workspace(self, M, device):

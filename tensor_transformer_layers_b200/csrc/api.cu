@@ -31,6 +31,7 @@ constexpr int kMaxDevices = 64;
 constexpr uint64_t kMlpMagic = 0x54504D4C50484E44ull;   // "TPMLPHND"
 constexpr uint64_t kAttnMagic = 0x5450415454484E44ull;  // "TPATTHND"
 constexpr int64_t kMaxDim = int64_t(1) << 31;           // TMA coordinates are 32-bit
+constexpr int kMaxPackedBlocks = 64;
 
 struct DeviceInfo {
   bool ready = false;
@@ -98,10 +99,10 @@ int current_device_context(int* num_sms, int** err) {
 }
 
 static CUresult make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
-                            uint64_t d2, uint32_t box0, uint32_t box1) {
+                            uint64_t d2, uint32_t box0, uint32_t box1, uint32_t box2 = 1) {
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};  // bytes, dims 1 and 2
-  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t box[3] = {box0, box1, box2};
   const cuuint32_t estride[3] = {1, 1, 1};
   return g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -110,6 +111,11 @@ static CUresult make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void
 CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
                           uint32_t box1) {
   return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d0, d1, d2, box0, box1);
+}
+
+CUresult make_map_3d_bf16_box(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                              uint32_t box0, uint32_t box1, uint32_t box2) {
+  return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d0, d1, d2, box0, box1, box2);
 }
 
 CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
@@ -129,7 +135,7 @@ tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, c
   if (M == 0) return TP_OK;
   const GemmOperand A{X, uint64_t(K), uint64_t(M), 1};
   const GemmOperand B{W, uint64_t(K), uint64_t(Ns), uint64_t(T)};
-  GemmArgs a;
+  GemmArgs a{};
   a.M = int(M);
   a.N = int(Ns);
   a.k_blocks = int((K + 63) / 64);
@@ -153,7 +159,7 @@ tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, 
   if (M == 0) return TP_OK;
   const GemmOperand Aop{A, uint64_t(Ks), uint64_t(M), uint64_t(T)};
   const GemmOperand Bop{W, uint64_t(Ks), uint64_t(N), uint64_t(T)};
-  GemmArgs a;
+  GemmArgs a{};
   a.M = int(M);
   a.N = int(N);
   a.k_blocks = int((Ks + 63) / 64);
@@ -167,6 +173,49 @@ tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, 
   a.bias_gstride = 0;
   a.gelu = 0;
   a.out_f16 = 0;
+  a.err = di->err;
+  return launch_gemm(Aop, Bop, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+// SwiGLU colwise: out[g] = silu(X W_gate,g^T + bg) * (X W_up,g^T + bu), W[g] = [gate; up].
+tp_status run_colwise_swiglu(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, const uint16_t* W,
+                             const uint16_t* b, int64_t Fs, int T, uint16_t* out, cudaStream_t s) {
+  if (M == 0) return TP_OK;
+  const GemmOperand A{X, uint64_t(K), uint64_t(M), 1};
+  const GemmOperand B{W, uint64_t(K), uint64_t(2 * Fs), uint64_t(T)};
+  GemmArgs a{};
+  a.M = int(M);
+  a.N = int(Fs);
+  a.k_blocks = int((K + 63) / 64);
+  a.kshards = 1;
+  a.groups = T;
+  a.out = out;
+  a.out_gstride = M * Fs;
+  a.ldo = Fs;
+  a.bias = b;
+  a.bias_gstride = 2 * Fs;
+  a.swiglu = 1;
+  a.up_off = Fs;
+  a.err = di->err;
+  return launch_gemm(A, B, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+// rowwise_split_input: Y = sum_r X[:, r*Ks:(r+1)*Ks] . W[r]^T + bias, X read in place.
+tp_status run_rowwise_split(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t Ks, const uint16_t* W, int64_t N,
+                            const uint16_t* bias, int T, uint16_t* Y, cudaStream_t s) {
+  if (M == 0) return TP_OK;
+  const GemmOperand Aop{X, uint64_t(Ks), uint64_t(M), uint64_t(T)};  // memory [M][T][Ks]
+  const GemmOperand Bop{W, uint64_t(Ks), uint64_t(N), uint64_t(T)};
+  GemmArgs a{};
+  a.M = int(M);
+  a.N = int(N);
+  a.k_blocks = int((Ks + 63) / 64);
+  a.kshards = T;
+  a.groups = 1;
+  a.a_split_input = 1;
+  a.out = Y;
+  a.ldo = N;
+  a.bias = bias;
   a.err = di->err;
   return launch_gemm(Aop, Bop, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
@@ -210,6 +259,60 @@ tp_status slice_all_qkv(const uint16_t* Wqkv, int64_t D, int T, uint16_t* out, c
              : TP_ERR_CUDA;
 }
 
+// Packed slicing ("Fused projections").  sizes[] are absolute block sizes
+// along the packed dimension (validated).  rank < 0: all shards, stacked.
+tp_status slice_packed(const uint16_t* W, int64_t rows, int64_t cols, int style, const int64_t* sizes, int nb,
+                       int T, int rank, uint16_t* out, cudaStream_t s) {
+  const int64_t P = style == TP_COLWISE ? rows : cols;
+  const int64_t Ps = P / T;  // shard extent along the packed dimension
+  int64_t start = 0, off = 0;
+  for (int b = 0; b < nb; ++b) {
+    const int64_t q = sizes[b] / T;  // this block's share per shard
+    cudaError_t e;
+    if (style == TP_COLWISE) {
+      if (rank >= 0)
+        e = launch_slice_copy(W + (start + rank * q) * cols, out + off * cols, 1, q, cols, cols, 0, 0, s);
+      else
+        e = launch_slice_copy(W + start * cols, out + off * cols, T, q, cols, cols, q * cols, Ps * cols, s);
+    } else {
+      if (rank >= 0)
+        e = launch_slice_copy(W + start + rank * q, out + off, 1, rows, q, cols, 0, 0, s, 1, 0, 0, Ps);
+      else
+        e = launch_slice_copy(W + start, out + off, T, rows, q, cols, q, rows * Ps, s, 1, 0, 0, Ps);
+    }
+    if (e != cudaSuccess) return TP_ERR_CUDA;
+    start += sizes[b];
+    off += q;
+  }
+  return TP_OK;
+}
+
+// Validates a packed call and turns proportional blocks into absolute sizes.
+tp_status check_packed(const uint16_t* W, int64_t rows, int64_t cols, int style, const int64_t* blocks, int nblocks,
+                       int T, const uint16_t* out, int64_t* sizes) {
+  if (!W || !out || !blocks) return TP_ERR_NULL;
+  if (style != TP_COLWISE && style != TP_ROWWISE) return TP_ERR_BAD_STYLE;
+  if (T < 1) return TP_ERR_BAD_DEGREE;
+  if (rows < 1 || cols < 1 || rows >= kMaxDim || cols >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (nblocks < 1 || nblocks > kMaxPackedBlocks) return TP_ERR_BAD_BLOCKS;
+  const int64_t P = style == TP_COLWISE ? rows : cols;
+  int64_t sum = 0;
+  for (int b = 0; b < nblocks; ++b) {
+    if (blocks[b] < 1 || blocks[b] > P) return TP_ERR_BAD_BLOCKS;
+    sum += blocks[b];
+  }
+  if (sum > P || P % sum != 0) return TP_ERR_BAD_BLOCKS;
+  for (int b = 0; b < nblocks; ++b) {
+    sizes[b] = blocks[b] * (P / sum);
+    if (sizes[b] % T != 0) return TP_ERR_INDIVISIBLE;
+  }
+  if (!al16(W) || !al16(out) || cols % 8 != 0) return TP_ERR_ALIGNMENT;
+  if (style == TP_ROWWISE)
+    for (int b = 0; b < nblocks; ++b)
+      if ((sizes[b] / T) % 8 != 0) return TP_ERR_ALIGNMENT;
+  return TP_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Shape checks shared by the layer calls.
 // ---------------------------------------------------------------------------
@@ -232,14 +335,16 @@ tp_status check_attn_shape(int64_t M, int64_t D, int heads, int T) {
 struct MlpLayout {
   size_t w_up, b_up, w_down, h, total;
 };
-MlpLayout mlp_layout(int64_t M, int64_t D, int64_t F, bool with_weights) {
+// swiglu: the colwise weight is [gate; up], twice the rows of W_up.
+MlpLayout mlp_layout(int64_t M, int64_t D, int64_t F, bool with_weights, bool swiglu = false) {
   MlpLayout L{};
   size_t off = 0;
+  const size_t in_rows = size_t(F) * (swiglu ? 2 : 1);
   if (with_weights) {
     L.w_up = off;
-    off += up256(size_t(F) * D * 2);
+    off += up256(in_rows * D * 2);
     L.b_up = off;
-    off += up256(size_t(F) * 2);
+    off += up256(in_rows * 2);
     L.w_down = off;
     off += up256(size_t(D) * F * 2);
   }
@@ -275,12 +380,13 @@ tp_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   return TP_OK;
 }
 
-// The MLP pair on sharded weights (a2..a4).
+// The MLP pair on sharded weights (a2..a4); swiglu: w_up_sh holds [gate_r; up_r].
 tp_status mlp_forward(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t D, int64_t F, int T,
                       const uint16_t* w_up_sh, const uint16_t* b_up_sh, const uint16_t* w_down_sh,
-                      const uint16_t* b_down, uint16_t* H, uint16_t* Y, cudaStream_t s) {
+                      const uint16_t* b_down, uint16_t* H, uint16_t* Y, cudaStream_t s, bool swiglu = false) {
   const int64_t Fs = F / T;
-  tp_status st = run_colwise(di, X, M, D, w_up_sh, b_up_sh, Fs, T, 1, 0, H, s);
+  tp_status st = swiglu ? run_colwise_swiglu(di, X, M, D, w_up_sh, b_up_sh, Fs, T, H, s)
+                        : run_colwise(di, X, M, D, w_up_sh, b_up_sh, Fs, T, 1, 0, H, s);
   if (st != TP_OK) return st;
   return run_rowwise(di, H, M, Fs, w_down_sh, D, b_down, T, Y, s);
 }
@@ -303,8 +409,9 @@ struct MlpHandle {
   int device;
   int64_t D, F;
   int T;
-  uint16_t* w_up;    // [T][F/T][D]
-  uint16_t* b_up;    // [T][F/T] or null
+  bool swiglu;       // colwise weight holds [gate_r; up_r] per shard
+  uint16_t* w_up;    // [T][F/T][D], SwiGLU: [T][2F/T][D]
+  uint16_t* b_up;    // [T][F/T] or null, SwiGLU: [T][2F/T]
   uint16_t* w_down;  // [T][D][F/T]
   uint16_t* b_down;  // [D] or null (replicated)
 };
@@ -340,6 +447,9 @@ const char* tp_status_string(int s) {
     case TP_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait timed out";
     case TP_ERR_BAD_STYLE: return "unknown sharding style";
     case TP_ERR_BAD_HANDLE: return "invalid handle";
+    case TP_ERR_BAD_BLOCKS:
+      return "packed blocks invalid: count outside 1..64, a block < 1, or their sum does not divide the packed "
+             "dimension";
     case TP_ERR_SCRATCH_LIMIT:
       return "size exceeds the 64 MiB static scratch of tp_mlp_pair_sharded_noalloc (F * 256 bytes must fit)";
     default: return "unknown status";
@@ -371,6 +481,7 @@ tp_status tp_check_device_error(void* stream) {
 tp_status tp_shard_weight(const uint16_t* W, int64_t rows, int64_t cols, int style, int tp_degree, int rank,
                           uint16_t* out, void* stream) {
   if (!W || !out) return TP_ERR_NULL;
+  if (style == TP_ROWWISE_SPLIT_INPUT) style = TP_ROWWISE;  // same weight slice
   if (style != TP_COLWISE && style != TP_ROWWISE) return TP_ERR_BAD_STYLE;
   if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
   if (rank < 0 || rank >= tp_degree) return TP_ERR_BAD_RANK;
@@ -395,6 +506,7 @@ tp_status tp_shard_weight(const uint16_t* W, int64_t rows, int64_t cols, int sty
 tp_status tp_shard_weight_all(const uint16_t* W, int64_t rows, int64_t cols, int style, int tp_degree, uint16_t* out,
                               void* stream) {
   if (!W || !out) return TP_ERR_NULL;
+  if (style == TP_ROWWISE_SPLIT_INPUT) style = TP_ROWWISE;  // same weight slice
   if (style != TP_COLWISE && style != TP_ROWWISE) return TP_ERR_BAD_STYLE;
   if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
   if (rows < 1 || cols < 1) return TP_ERR_BAD_SHAPE;
@@ -454,6 +566,27 @@ tp_status tp_shard_qkv_heads_all(const uint16_t* W_qkv, int64_t D, int heads, in
   return slice_all_qkv(W_qkv, D, tp_degree, out, as_stream(stream));
 }
 
+tp_status tp_shard_packed(const uint16_t* W, int64_t rows, int64_t cols, int style, const int64_t* blocks,
+                          int nblocks, int tp_degree, int rank, uint16_t* out, void* stream) {
+  int64_t sizes[kMaxPackedBlocks];
+  tp_status st = check_packed(W, rows, cols, style, blocks, nblocks, tp_degree, out, sizes);
+  if (st != TP_OK) return st;
+  if (rank < 0 || rank >= tp_degree) return TP_ERR_BAD_RANK;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return slice_packed(W, rows, cols, style, sizes, nblocks, tp_degree, rank, out, as_stream(stream));
+}
+
+tp_status tp_shard_packed_all(const uint16_t* W, int64_t rows, int64_t cols, int style, const int64_t* blocks,
+                              int nblocks, int tp_degree, uint16_t* out, void* stream) {
+  int64_t sizes[kMaxPackedBlocks];
+  tp_status st = check_packed(W, rows, cols, style, blocks, nblocks, tp_degree, out, sizes);
+  if (st != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return slice_packed(W, rows, cols, style, sizes, nblocks, tp_degree, -1, out, as_stream(stream));
+}
+
 // ----------------------------------------------------------------------- step-level calls
 tp_status tp_colwise_linear(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W_shards,
                             const uint16_t* b_shards, int64_t N_s, int tp_degree, int gelu, int out_dtype,
@@ -481,6 +614,32 @@ tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s
   DeviceInfo* di = nullptr;
   if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
   return run_rowwise(di, A_shards, M, K_s, W_shards, N, bias, tp_degree, Y, as_stream(stream));
+}
+
+tp_status tp_colwise_swiglu(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W_shards,
+                            const uint16_t* b_shards, int64_t F_s, int tp_degree, uint16_t* out, void* stream) {
+  if (!X || !W_shards || !out) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || K < 1 || F_s < 1 || M >= kMaxDim || K >= kMaxDim || 2 * F_s * tp_degree >= kMaxDim)
+    return TP_ERR_BAD_SHAPE;
+  if (!al16(X) || !al16(W_shards) || !al16(out) || (b_shards && !al16(b_shards))) return TP_ERR_ALIGNMENT;
+  if (K % 8 != 0 || F_s % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_colwise_swiglu(di, X, M, K, W_shards, b_shards, F_s, tp_degree, out, as_stream(stream));
+}
+
+tp_status tp_rowwise_split_input_linear(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W_shards, int64_t N,
+                                        const uint16_t* bias, int tp_degree, uint16_t* Y, void* stream) {
+  if (!X || !W_shards || !Y) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || K < 1 || N < 1 || M >= kMaxDim || K >= kMaxDim || N >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (K % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  if (!al16(X) || !al16(W_shards) || !al16(Y) || (bias && !al16(bias))) return TP_ERR_ALIGNMENT;
+  if ((K / tp_degree) % 8 != 0 || N % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_rowwise_split(di, X, M, K / tp_degree, W_shards, N, bias, tp_degree, Y, as_stream(stream));
 }
 
 tp_status tp_sdpa_shards(const uint16_t* QKV, int64_t M, int heads, int tp_degree, uint16_t* O, void* stream) {
@@ -554,6 +713,71 @@ tp_status tp_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F, const 
   return mlp_forward(di, X, M, D, F, tp_degree, w_up_sh, b_up_sh, w_down_sh, b_down, H, Y, s);
 }
 
+size_t tp_swiglu_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree) {
+  if (check_mlp_shape(M, D, F, tp_degree) != TP_OK) return 0;
+  return mlp_layout(M, D, F, true, true).total;
+}
+
+tp_status tp_swiglu_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F, const uint16_t* W_in,
+                             const uint16_t* b_in, const uint16_t* W_out, const uint16_t* b_out, int tp_degree,
+                             uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (!X || !W_in || !W_out || !Y) return TP_ERR_NULL;
+  tp_status st = check_mlp_shape(M, D, F, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(X) || !al16(W_in) || !al16(W_out) || !al16(Y) || (b_in && !al16(b_in)) || (b_out && !al16(b_out)))
+    return TP_ERR_ALIGNMENT;
+  if (M == 0) return TP_OK;
+  const MlpLayout L = mlp_layout(M, D, F, true, true);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* w_in_sh = reinterpret_cast<uint16_t*>(w + L.w_up);
+  uint16_t* b_in_sh = b_in ? reinterpret_cast<uint16_t*>(w + L.b_up) : nullptr;
+  uint16_t* w_out_sh = reinterpret_cast<uint16_t*>(w + L.w_down);
+  const int64_t halves[2] = {F, F};  // [gate; up], packed colwise with blocks [1, 1]
+  if ((st = slice_packed(W_in, 2 * F, D, TP_COLWISE, halves, 2, tp_degree, -1, w_in_sh, s)) != TP_OK) return st;
+  if (b_in && (st = slice_packed(b_in, 1, 2 * F, TP_ROWWISE, halves, 2, tp_degree, -1, b_in_sh, s)) != TP_OK)
+    return st;
+  if ((st = slice_all_rowwise(W_out, D, F, tp_degree, w_out_sh, s)) != TP_OK) return st;
+  return mlp_forward(di, X, M, D, F, tp_degree, w_in_sh, b_in_sh, w_out_sh, b_out,
+                     reinterpret_cast<uint16_t*>(w + L.h), Y, s, true);
+}
+
+tp_status tp_swiglu_prepare(const uint16_t* W_in, const uint16_t* b_in, const uint16_t* W_out, const uint16_t* b_out,
+                            int64_t D, int64_t F, int tp_degree, void* stream, void** handle) {
+  if (!W_in || !W_out || !handle) return TP_ERR_NULL;
+  tp_status st = check_mlp_shape(0, D, F, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(W_in) || !al16(W_out) || (b_in && !al16(b_in)) || (b_out && !al16(b_out))) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  MlpHandle* h = new MlpHandle{};
+  h->magic = kMlpMagic;
+  cudaGetDevice(&h->device);
+  h->D = D;
+  h->F = F;
+  h->T = tp_degree;
+  h->swiglu = true;
+  const int64_t halves[2] = {F, F};
+  bool ok = cudaMalloc(&h->w_up, size_t(2 * F) * D * 2) == cudaSuccess &&
+            cudaMalloc(&h->w_down, size_t(D) * F * 2) == cudaSuccess &&
+            (!b_in || cudaMalloc(&h->b_up, size_t(2 * F) * 2) == cudaSuccess) &&
+            (!b_out || cudaMalloc(&h->b_down, size_t(D) * 2) == cudaSuccess);
+  ok = ok && slice_packed(W_in, 2 * F, D, TP_COLWISE, halves, 2, tp_degree, -1, h->w_up, s) == TP_OK &&
+       slice_all_rowwise(W_out, D, F, tp_degree, h->w_down, s) == TP_OK &&
+       (!b_in || slice_packed(b_in, 1, 2 * F, TP_ROWWISE, halves, 2, tp_degree, -1, h->b_up, s) == TP_OK) &&
+       (!b_out || cudaMemcpyAsync(h->b_down, b_out, size_t(D) * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess);
+  if (!ok) {
+    tp_destroy(h);
+    return TP_ERR_CUDA;
+  }
+  *handle = h;
+  return TP_OK;
+}
+
 tp_status tp_mlp_prepare(const uint16_t* W_up, const uint16_t* b_up, const uint16_t* W_down, const uint16_t* b_down,
                          int64_t D, int64_t F, int tp_degree, void* stream, void** handle) {
   if (!W_up || !W_down || !handle) return TP_ERR_NULL;
@@ -600,7 +824,8 @@ tp_status tp_mlp_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y, vo
   DeviceInfo* di = nullptr;
   if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
   uint16_t* H = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.h);
-  return mlp_forward(di, X, M, h->D, h->F, h->T, h->w_up, h->b_up, h->w_down, h->b_down, H, Y, as_stream(stream));
+  return mlp_forward(di, X, M, h->D, h->F, h->T, h->w_up, h->b_up, h->w_down, h->b_down, H, Y, as_stream(stream),
+                     h->swiglu);
 }
 
 // ----------------------------------------------------------------------- attention block

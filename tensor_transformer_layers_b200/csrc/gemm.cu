@@ -19,6 +19,16 @@
 //   warps 2-5 epilogue: tcgen05.ld 32 columns at a time (thread = output row),
 //             bias, optional tanh-form GELU, rounding to bf16 (or fp16 for the
 //             Q/K/V that feed attention), 16-byte global stores.
+// Two more forms of the same kernels:
+//   SwiGLU colwise (a gate/up pair packed with blocks [1, 1], section "Fused
+//            projections"): the B tile's first 128 rows are gate rows and its
+//            last 128 the matching up rows, fetched from the two blocks of the
+//            shard [gate_r; up_r] as they lie; the epilogue pairs accumulator
+//            column j with column 128 + j and writes silu(g) * u, so the output
+//            tile is 128 columns wide;
+//   rowwise_split_input (style table): A is the replicated input and shard s
+//            reads its own K range of it; the A map is {K_s, T, M}, so the
+//            slice of the input is a TMA coordinate, not a copy.
 // * gemm_tc_kernel: one CTA per SM, 128x256 tile, M=128 N=256 K=16 MMAs,
 //   4 stages of 48 KB (A 128x64 + B 256x64).  Used for M < 256.
 // * gemm_pair_kernel: CTA pairs (cluster of 2, tcgen05 cta_group::2), 256x256
@@ -71,6 +81,12 @@ __device__ __forceinline__ float gelu_tanh(float x) {
   // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))  (Hendrycks & Gimpel, 2016)
   const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
   return 0.5f * x * (1.0f + tanh_approx(u));
+}
+
+// SiLU(x) = x * sigmoid(x) = x / (1 + 2^(-x log2 e))  (Elfwing et al., 2018).
+// For x -> -inf the power overflows to +inf and the reciprocal to 0.
+__device__ __forceinline__ float silu(float x) {
+  return x * rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * x));
 }
 
 struct TileCoord {
@@ -150,6 +166,60 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& p, uint32_t taddr,
   }
 }
 
+// SwiGLU drain of one accumulator: columns [0, 128) hold gate, [128, 256) the
+// matching up.  Output columns col_base + j, j < 128, masked by p.N; gate bias
+// at bias[col], up bias at bias[up_off + col].
+__device__ __forceinline__ void epilogue_swiglu(const GemmArgs& p, uint32_t taddr, int row, int g, int col_base) {
+  uint16_t* orow = p.out + int64_t(g) * p.out_gstride + int64_t(row) * p.ldo;
+  const uint16_t* bias = p.bias ? p.bias + int64_t(g) * p.bias_gstride : nullptr;
+  const int n_left = p.N - col_base;
+  const int chunks = n_left >= 128 ? 8 : (n_left + 15) / 16;  // warp-uniform
+  for (int c = 0; c < chunks; ++c) {
+    uint32_t rg[16], ru[16];
+    __syncwarp();
+    tmem_ld16x2_sync(taddr + uint32_t(c * 16), rg, taddr + uint32_t(128 + c * 16), ru);
+    const int col0 = col_base + c * 16;
+    float gv[16], uv[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      gv[j] = __uint_as_float(rg[j]);
+      uv[j] = __uint_as_float(ru[j]);
+    }
+    if (bias != nullptr) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (col0 + 8 * h < p.N) {
+          const uint4 bg = __ldg(reinterpret_cast<const uint4*>(bias + col0) + h);
+          const uint4 bu = __ldg(reinterpret_cast<const uint4*>(bias + p.up_off + col0) + h);
+          const uint32_t wg[4] = {bg.x, bg.y, bg.z, bg.w};
+          const uint32_t wu[4] = {bu.x, bu.y, bu.z, bu.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            gv[8 * h + 2 * j] += bf16_lo(wg[j]);
+            gv[8 * h + 2 * j + 1] += bf16_hi(wg[j]);
+            uv[8 * h + 2 * j] += bf16_lo(wu[j]);
+            uv[8 * h + 2 * j + 1] += bf16_hi(wu[j]);
+          }
+        }
+      }
+    }
+    uint4 o[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      o[h].x = pack_bf16x2(silu(gv[8 * h + 0]) * uv[8 * h + 0], silu(gv[8 * h + 1]) * uv[8 * h + 1]);
+      o[h].y = pack_bf16x2(silu(gv[8 * h + 2]) * uv[8 * h + 2], silu(gv[8 * h + 3]) * uv[8 * h + 3]);
+      o[h].z = pack_bf16x2(silu(gv[8 * h + 4]) * uv[8 * h + 4], silu(gv[8 * h + 5]) * uv[8 * h + 5]);
+      o[h].w = pack_bf16x2(silu(gv[8 * h + 6]) * uv[8 * h + 6], silu(gv[8 * h + 7]) * uv[8 * h + 7]);
+    }
+    if (row < p.M) {
+      uint4* op = reinterpret_cast<uint4*>(orow + col0);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (col0 + 8 * h < p.N) op[h] = o[h];
+    }
+  }
+}
+
 // ============================================================================
 // Single-CTA kernel
 // ============================================================================
@@ -168,8 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int out_bn = p.swiglu ? BN1 / 2 : BN1;  // output columns per tile
   const int m_tiles = (p.M + BM1 - 1) / BM1;
-  const int n_tiles = (p.N + BN1 - 1) / BN1;
+  const int n_tiles = (p.N + out_bn - 1) / out_bn;
   const int tiles = m_tiles * n_tiles * p.groups;
   const int k_iters = p.k_blocks * p.kshards;
 
@@ -217,8 +288,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kb = it - s * p.k_blocks;
           uint8_t* sa = smem + stage * kStageBytes1;
           mbar_arrive_expect_tx(&full[stage], kStageBytes1);
-          tma_load_3d(sa, &amap, &full[stage], kb * BK, tc.mb * BM1, p.a_follows_shard ? s : 0);
-          tma_load_3d(sa + kABytes1, &bmap, &full[stage], kb * BK, tc.nb * BN1, tc.g + s);
+          if (p.a_split_input)
+            tma_load_3d(sa, &amap, &full[stage], kb * BK, s, tc.mb * BM1);
+          else
+            tma_load_3d(sa, &amap, &full[stage], kb * BK, tc.mb * BM1, p.a_follows_shard ? s : 0);
+          if (p.swiglu) {  // two 128-row boxes: gate rows, then the matching up rows
+            tma_load_3d(sa + kABytes1, &bmap, &full[stage], kb * BK, tc.nb * 128, tc.g + s);
+            tma_load_3d(sa + kABytes1 + 128 * BK * 2, &bmap, &full[stage], kb * BK, int(p.up_off) + tc.nb * 128,
+                        tc.g + s);
+          } else {
+            tma_load_3d(sa + kABytes1, &bmap, &full[stage], kb * BK, tc.nb * BN1, tc.g + s);
+          }
           ++issued;
           if (++stage == kStages1) {
             stage = 0;
@@ -294,8 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      epilogue_rows(p, tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols), tc.mb * BM1 + q * 32 + lane,
-                    tc.g, tc.nb * BN1);
+      const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
+      if (p.swiglu)
+        epilogue_swiglu(p, taddr, tc.mb * BM1 + q * 32 + lane, tc.g, tc.nb * out_bn);
+      else
+        epilogue_rows(p, taddr, tc.mb * BM1 + q * 32 + lane, tc.g, tc.nb * out_bn);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -334,8 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();  // 0 = leader, 1 = peer
   const int pair = blockIdx.x >> 1;
   const int n_pairs = gridDim.x >> 1;
+  const int out_bn = p.swiglu ? BN2 / 2 : BN2;  // output columns per tile
   const int m_tiles = (p.M + BM2 - 1) / BM2;
-  const int n_tiles = (p.N + BN2 - 1) / BN2;
+  const int n_tiles = (p.N + out_bn - 1) / out_bn;
   const int tiles = m_tiles * n_tiles * p.groups;
   const int k_iters = p.k_blocks * p.kshards;
 
@@ -385,8 +469,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* sa = smem + stage * kStageBytes2;
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes2);  // both CTAs' bytes
-          tma_load_3d_pair(sa, &amap, fb, kb * BK, tc.mb * BM2 + int(rank) * 128, p.a_follows_shard ? s : 0);
-          tma_load_3d_pair(sa + kHalfBytes, &bmap, fb, kb * BK, tc.nb * BN2 + int(rank) * 128, tc.g + s);
+          const int a_row = tc.mb * BM2 + int(rank) * 128;
+          if (p.a_split_input)
+            tma_load_3d_pair(sa, &amap, fb, kb * BK, s, a_row);
+          else
+            tma_load_3d_pair(sa, &amap, fb, kb * BK, a_row, p.a_follows_shard ? s : 0);
+          // B: this CTA's 128 rows of the 256-row tile; SwiGLU: the even CTA
+          // fetches the gate rows, the odd one the matching up rows.
+          const int b_row = p.swiglu ? int(rank) * int(p.up_off) + tc.nb * 128 : tc.nb * BN2 + int(rank) * 128;
+          tma_load_3d_pair(sa + kHalfBytes, &bmap, fb, kb * BK, b_row, tc.g + s);
           ++issued;
           if (++stage == kStages2) {
             stage = 0;
@@ -466,8 +557,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      epilogue_rows(p, tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols),
-                    tc.mb * BM2 + int(rank) * 128 + q * 32 + lane, tc.g, tc.nb * BN2);
+      const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
+      const int row = tc.mb * BM2 + int(rank) * 128 + q * 32 + lane;
+      if (p.swiglu)
+        epilogue_swiglu(p, taddr, row, tc.g, tc.nb * out_bn);
+      else
+        epilogue_rows(p, taddr, row, tc.g, tc.nb * out_bn);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader + uint32_t(acc * sizeof(uint64_t)));
@@ -518,6 +613,13 @@ int max_active_pairs(int num_sms) {
   return g_max_pairs[dev];
 }
 
+// A's map: {K_s, rows, z}, or {K_s, z, rows} for a split input (memory
+// [rows][z][K_s]), with a box of 64 x box_rows rows either way.
+CUresult make_a_map(CUtensorMap* map, const GemmOperand& A, const GemmArgs& a, uint32_t box_rows) {
+  if (a.a_split_input) return make_map_3d_bf16_box(map, A.base, A.k, A.z, A.rows, BK, 1, box_rows);
+  return make_map_3d_bf16(map, A.base, A.k, A.rows, A.z, BK, box_rows);
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms,
@@ -526,12 +628,13 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
   CUtensorMap amap, bmap;
   if (a.M >= BM2) {
     // CTA-pair kernel: each CTA loads 128-row halves of both operands.
-    if (make_map_3d_bf16(&amap, A.base, A.k, A.rows, A.z, BK, 128) != CUDA_SUCCESS ||
+    if (make_a_map(&amap, A, a, 128) != CUDA_SUCCESS ||
         make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, 128) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+      return note_cuda_error("gemm (CTA pairs): tensor map encode", cudaErrorInvalidValue);
     cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
     if (e != cudaSuccess) return note_cuda_error("gemm (CTA pairs): set shared memory size", e);
-    const int64_t tiles = int64_t((a.M + BM2 - 1) / BM2) * ((a.N + BN2 - 1) / BN2) * a.groups;
+    const int out_bn = a.swiglu ? BN2 / 2 : BN2;
+    const int64_t tiles = int64_t((a.M + BM2 - 1) / BM2) * ((a.N + out_bn - 1) / out_bn) * a.groups;
     int pairs = max_active_pairs(num_sms);
     if (tiles < pairs) pairs = int(tiles);
     cudaLaunchConfig_t cfg = {};
@@ -551,11 +654,11 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
     if (e == cudaSuccess) e = cudaGetLastError();
     return note_cuda_error("gemm (CTA pairs): launch", e);
   }
-  if (make_map_3d_bf16(&amap, A.base, A.k, A.rows, A.z, BK, BM1) != CUDA_SUCCESS ||
-      make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, BN1) != CUDA_SUCCESS)
+  if (make_a_map(&amap, A, a, BM1) != CUDA_SUCCESS ||
+      make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, a.swiglu ? BN1 / 2 : BN1) != CUDA_SUCCESS)
     return note_cuda_error("gemm: tensor map encode", cudaErrorInvalidValue);
   const int m_tiles = (a.M + BM1 - 1) / BM1;
-  const int n_tiles = (a.N + BN1 - 1) / BN1;
+  const int n_tiles = (a.N + (a.swiglu ? BN1 / 2 : BN1) - 1) / (a.swiglu ? BN1 / 2 : BN1);
   const int64_t tiles = int64_t(m_tiles) * n_tiles * a.groups;
   const int grid = int(tiles < num_sms ? tiles : num_sms);
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes1);

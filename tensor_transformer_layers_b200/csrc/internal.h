@@ -11,14 +11,16 @@ namespace tp {
 // ----------------------------------------------------------------------------
 // a1: blocked 2-D copy.  For b in [0, nblocks), b2 in [0, nblocks2),
 // r in [0, rows), c in [0, cols):
-//   dst[b*dst_bstride + b2*dst_bstride2 + r*cols + c]
+//   dst[b*dst_bstride + b2*dst_bstride2 + r*dst_ld + c]
 //     = src[b*src_bstride + b2*src_bstride2 + r*src_ld + c]
-// (element units).  cols, src_ld, the strides and both pointers must be
-// multiples of 8 elements / 16 bytes (checked by the caller).
+// (element units; dst_ld < 0 means dst_ld = cols).  cols, src_ld, dst_ld, the
+// strides and both pointers must be multiples of 8 elements / 16 bytes
+// (checked by the caller).
 // ----------------------------------------------------------------------------
 cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblocks, int64_t rows, int64_t cols,
                               int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t s,
-                              int64_t nblocks2 = 1, int64_t src_bstride2 = 0, int64_t dst_bstride2 = 0);
+                              int64_t nblocks2 = 1, int64_t src_bstride2 = 0, int64_t dst_bstride2 = 0,
+                              int64_t dst_ld = -1);
 
 // ----------------------------------------------------------------------------
 // a8: Y[M x N] = bf16(sum_r parts[r] + bias)
@@ -32,6 +34,13 @@ cudaError_t launch_reduce_partials(const float* parts, int64_t M, int64_t N, int
 // A map: 3-D bf16 {K_s, M, ZA}; B map: 3-D bf16 {K_s, Nrows, ZB}.
 //   colwise: groups = T, kshards = 1, zb = g, za = 0.
 //   rowwise: groups = 1, kshards = T, zb = s, za = s.
+//   rowwise_split_input: as rowwise, but A is one replicated [M x T*K_s]
+//     input and shard s reads its columns [s*K_s, (s+1)*K_s): the A map is
+//     built {K_s, T, M} (a_split_input = 1) and loaded at (k, s, row).
+//   SwiGLU colwise (swiglu = 1): B_g = [gate_g; up_g] with up_g starting
+//     up_off rows in; each 256-column accumulator holds 128 gate and the 128
+//     matching up columns, and the epilogue writes silu(gate + bg) * (up + bu)
+//     to a 128-column output tile (N = output columns = gate rows).
 // ----------------------------------------------------------------------------
 struct GemmArgs {
   int M;                 // output rows
@@ -47,11 +56,15 @@ struct GemmArgs {
   int64_t bias_gstride;  // elements between groups' biases
   int gelu;              // 1: tanh-form GELU after bias
   int out_f16;           // 1: store fp16 instead of bf16
+  int swiglu;            // 1: SwiGLU epilogue over [gate; up] weight rows (see above)
+  int a_split_input;     // 1: A map is {K_s, T, M}, loaded at (k, s, row)
+  int64_t up_off;        // SwiGLU: rows from gate_g to up_g in B (and bias elements)
   int* err;              // device error word
 };
 
 // A bf16 operand seen as a 3-D tensor {k (contiguous), rows, z}: the GEMM
 // builds its TMA maps from this (box sizes depend on the kernel it picks).
+// With a_split_input the A operand's memory is [rows][z][k] instead.
 struct GemmOperand {
   const void* base;
   uint64_t k, rows, z;
@@ -92,6 +105,8 @@ int current_device_context(int* num_sms, int** err);
 // Host helpers (api.cu).
 CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                           uint32_t box0, uint32_t box1);
+CUresult make_map_3d_bf16_box(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                              uint32_t box0, uint32_t box1, uint32_t box2);
 CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
                          uint32_t box1);
 

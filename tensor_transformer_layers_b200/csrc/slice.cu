@@ -3,10 +3,12 @@
 // A colwise shard (rows [r*N/T, (r+1)*N/T) of a row-major W[N x K]) is one
 // contiguous span; a rowwise shard (columns [r*K/T, (r+1)*K/T) of every row)
 // is N row segments of K/T elements at stride K; the packed head split of a
-// fused QKV weight is three contiguous spans.  All three are instances of a
-// blocked 2-D copy, done here with 16-byte loads/stores.  Each thread keeps
-// four 16-byte loads in flight before storing, and loads/stores use the
-// streaming cache policy: the data is touched exactly once.
+// fused QKV weight is three contiguous spans; a packed block (section "Fused
+// projections") is one of these per block, written at the block's offset
+// inside the shard (a destination row stride for packed rowwise).  All are
+// instances of a blocked 2-D copy, done here with 16-byte loads/stores.  Each
+// thread keeps four 16-byte loads in flight before storing, and loads/stores
+// use the streaming cache policy: the data is touched exactly once.
 #include "internal.h"
 
 namespace tp {
@@ -17,14 +19,15 @@ constexpr int kUnroll = 4;
 
 __global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                               uint32_t rows, uint32_t c8, int64_t src_ld8,
-                                                              int64_t src_b8, int64_t dst_b8, int64_t src_b8_2,
-                                                              int64_t dst_b8_2) {
+                                                              int64_t dst_ld8, int64_t src_b8, int64_t dst_b8,
+                                                              int64_t src_b8_2, int64_t dst_b8_2) {
   const uint32_t total = rows * c8;  // chunks in this block (host guarantees < 2^31)
   const uint4* s = src + int64_t(blockIdx.y) * src_b8 + int64_t(blockIdx.z) * src_b8_2;
   uint4* d = dst + int64_t(blockIdx.y) * dst_b8 + int64_t(blockIdx.z) * dst_b8_2;
   const uint32_t stride = gridDim.x * kThreads;
   for (uint32_t base = blockIdx.x * kThreads + threadIdx.x; base < total; base += stride * kUnroll) {
     uint4 v[kUnroll];
+    int64_t doff[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const uint32_t j = base + u * stride;
@@ -32,12 +35,13 @@ __global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __res
         const uint32_t r = j / c8;
         const uint32_t c = j - r * c8;
         v[u] = __ldcs(s + int64_t(r) * src_ld8 + c);
+        doff[u] = int64_t(r) * dst_ld8 + c;
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const uint32_t j = base + u * stride;
-      if (j < total) __stcs(d + j, v[u]);
+      if (j < total) __stcs(d + doff[u], v[u]);
     }
   }
 }
@@ -46,11 +50,12 @@ __global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __res
 
 cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblocks, int64_t rows, int64_t cols,
                               int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t st,
-                              int64_t nblocks2, int64_t src_bstride2, int64_t dst_bstride2) {
+                              int64_t nblocks2, int64_t src_bstride2, int64_t dst_bstride2, int64_t dst_ld) {
   if (nblocks <= 0 || nblocks2 <= 0 || rows <= 0 || cols <= 0) return cudaSuccess;
-  // A contiguous source (row segments back to back) is copied as one long span,
-  // split into virtual rows so the 32-bit chunk index never overflows.
-  if (src_ld == cols) {
+  if (dst_ld < 0) dst_ld = cols;
+  // A contiguous copy (row segments back to back on both sides) is one long
+  // span, split into virtual rows so the 32-bit chunk index never overflows.
+  if (src_ld == cols && dst_ld == cols) {
     int64_t n8 = rows * cols / 8;
     int64_t vc8 = 1;
     for (int64_t cand : {int64_t(4096), int64_t(1024), int64_t(256), int64_t(64), int64_t(8), int64_t(1)})
@@ -58,6 +63,7 @@ cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblock
     rows = n8 / vc8;
     cols = vc8 * 8;
     src_ld = cols;
+    dst_ld = cols;
   }
   const int64_t c8 = cols / 8;
   // Split very tall copies into pieces whose chunk count fits 31 bits.
@@ -70,9 +76,9 @@ cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblock
     if (blocks < 1) blocks = 1;
     dim3 grid(static_cast<unsigned>(blocks), static_cast<unsigned>(nblocks), static_cast<unsigned>(nblocks2));
     slice_copy_kernel<<<grid, kThreads, 0, st>>>(reinterpret_cast<const uint4*>(src + r0 * src_ld),
-                                                 reinterpret_cast<uint4*>(dst + r0 * cols), uint32_t(nr),
-                                                 uint32_t(c8), src_ld / 8, src_bstride / 8, dst_bstride / 8,
-                                                 src_bstride2 / 8, dst_bstride2 / 8);
+                                                 reinterpret_cast<uint4*>(dst + r0 * dst_ld), uint32_t(nr),
+                                                 uint32_t(c8), src_ld / 8, dst_ld / 8, src_bstride / 8,
+                                                 dst_bstride / 8, src_bstride2 / 8, dst_bstride2 / 8);
     count_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return note_cuda_error("slice: launch", e);

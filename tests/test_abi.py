@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings():
-    for code in range(14):
+    for code in range(15):
         assert tp.tp_status_string(code) not in ("", "unknown status")
     assert tp.tp_status_string(99) == "unknown status"
 
@@ -49,6 +49,9 @@ def test_workspace_sizes():
     assert tp.tp_attn_workspace_bytes(M, D, 24, T) == up(3 * D * D * 2) + up(D * D * 2) + up(M * 3 * D * 2) + up(M * D * 2)
     assert tp.tp_attn_run_workspace_bytes(M, D, 24, T) == up(M * 3 * D * 2) + up(M * D * 2)
     # invalid shapes report 0
+    assert tp.tp_swiglu_workspace_bytes(M, D, F, T) == (up(2 * F * D * 2) + up(2 * F * 2) + up(D * F * 2)
+                                                        + up(M * F * 2))
+    assert tp.tp_swiglu_workspace_bytes(M, D, F, 5) == 0
     assert tp.tp_mlp_workspace_bytes(M, D, F, 5) == 0
     assert tp.tp_attn_workspace_bytes(M, D, 24, 5) == 0
     assert tp.tp_attn_workspace_bytes(M, 3000, 24, 4) == 0
@@ -115,3 +118,49 @@ def test_layer_checks():
     st, h = tp.tp_attn_prepare(A, A, 768, 6, 4, stream=0)
     assert st == S["TP_ERR_HEADS_INDIVISIBLE"] and not h
     tp.tp_destroy(None)
+
+
+@pytest.mark.parametrize("args,want", [
+    # (W, rows, cols, style, blocks, T, rank, out)
+    ((0, 36, 8, tp.TP_COLWISE, [1, 1, 1, 3, 3], 2, 0, A), "TP_ERR_NULL"),
+    ((A, 36, 8, tp.TP_COLWISE, None, 2, 0, A), "TP_ERR_NULL"),
+    ((A, 36, 8, tp.TP_ROWWISE_SPLIT_INPUT, [1, 1], 2, 0, A), "TP_ERR_BAD_STYLE"),
+    ((A, 36, 8, tp.TP_COLWISE, [1, 1, 1, 3, 3], 0, 0, A), "TP_ERR_BAD_DEGREE"),
+    ((A, 0, 8, tp.TP_COLWISE, [1], 1, 0, A), "TP_ERR_BAD_SHAPE"),
+    ((A, 36, 8, tp.TP_COLWISE, [], 2, 0, A), "TP_ERR_BAD_BLOCKS"),
+    ((A, 36, 8, tp.TP_COLWISE, [1, 0, 1], 2, 0, A), "TP_ERR_BAD_BLOCKS"),
+    ((A, 36, 8, tp.TP_COLWISE, [1, -1, 2], 2, 0, A), "TP_ERR_BAD_BLOCKS"),
+    ((A, 36, 8, tp.TP_COLWISE, [1, 1, 3], 2, 0, A), "TP_ERR_BAD_BLOCKS"),      # sum 5 does not divide 36
+    ((A, 36, 8, tp.TP_COLWISE, [1] * 65, 1, 0, A), "TP_ERR_BAD_BLOCKS"),       # more than 64 blocks
+    ((A, 18, 8, tp.TP_COLWISE, [1, 1, 1, 3, 3], 3, 0, A), "TP_ERR_INDIVISIBLE"),  # blocks 2,2,2,6,6 by 3
+    ((A, 12, 8, tp.TP_COLWISE, [5, 1], 4, 0, A), "TP_ERR_INDIVISIBLE"),      # 12 % 4 == 0, 10 % 4 != 0
+    ((A, 36, 12, tp.TP_COLWISE, [1, 1, 1, 3, 3], 2, 0, A), "TP_ERR_ALIGNMENT"),
+    ((A, 8, 48, tp.TP_ROWWISE, [1, 5], 2, 0, A), "TP_ERR_ALIGNMENT"),        # per-shard widths 4 and 20
+    ((A, 36, 8, tp.TP_COLWISE, [1, 1, 1, 3, 3], 2, 2, A), "TP_ERR_BAD_RANK"),
+])
+def test_shard_packed_checks(args, want):
+    W, rows, cols, style, blocks, T, rank, out = args
+    assert tp.tp_shard_packed(W, rows, cols, style, blocks, T, rank, out, stream=0) == S[want]
+    if want != "TP_ERR_BAD_RANK":
+        assert tp.tp_shard_packed_all(W, rows, cols, style, blocks, T, out, stream=0) == S[want]
+
+
+def test_swiglu_and_split_input_checks():
+    ws = 1 << 30
+    assert tp.tp_swiglu_mlp_pair(A, 64, 128, 512, A, A, A, A, 3, A, A, ws, stream=0) == S["TP_ERR_INDIVISIBLE"]
+    assert tp.tp_swiglu_mlp_pair(A, 64, 128, 520, A, A, A, A, 4, A, A, ws, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_swiglu_mlp_pair(None, 64, 128, 512, A, A, A, A, 2, A, A, ws, stream=0) == S["TP_ERR_NULL"]
+    assert tp.tp_swiglu_mlp_pair(A, 64, 128, 512, A, A, A, A, 2, A, A, 100, stream=0) == S["TP_ERR_WORKSPACE"]
+    assert tp.tp_swiglu_mlp_pair(A, 0, 128, 512, A, A, A, A, 2, A, None, 0, stream=0) == 0
+    st, h = tp.tp_swiglu_prepare(A, A, A, A, 128, 512, 3, stream=0)
+    assert st == S["TP_ERR_INDIVISIBLE"] and not h
+    assert tp.tp_colwise_swiglu(A, 64, 100, A, None, 64, 2, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_colwise_swiglu(A, 64, 128, A, None, 60, 2, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_colwise_swiglu(A, 64, 128, A, None, 64, 0, A, stream=0) == S["TP_ERR_BAD_DEGREE"]
+    assert tp.tp_colwise_swiglu(A, -1, 128, A, None, 64, 2, A, stream=0) == S["TP_ERR_BAD_SHAPE"]
+    assert tp.tp_rowwise_split_input_linear(A, 64, 100, A, 64, None, 3, A, stream=0) == S["TP_ERR_INDIVISIBLE"]
+    assert tp.tp_rowwise_split_input_linear(A, 64, 60, A, 64, None, 3, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_rowwise_split_input_linear(A, 64, 128, A, 60, None, 2, A, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_rowwise_split_input_linear(None, 64, 128, A, 64, None, 2, A, stream=0) == S["TP_ERR_NULL"]
+    # the split-input style slices its weight like rowwise
+    assert tp.tp_shard_weight(A, 8, 24, tp.TP_ROWWISE_SPLIT_INPUT, 5, 0, A, stream=0) == S["TP_ERR_INDIVISIBLE"]
