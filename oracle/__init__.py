@@ -335,6 +335,61 @@ def attn_rows(X, W_qkv, W_o, heads, rows, tp_degree=1):
 
 
 # ---------------------------------------------------------------------------
+# Dual-stream joint attention: the image stream (to_q/k/v, to_out) and the
+# text stream (add_q/k/v_proj, to_add_out) are sharded alike (the page's note
+# that the encoder-stream projections follow the image-stream pattern); the
+# two streams' Q, K, V are concatenated along tokens (image first, then text)
+# and attended jointly; each stream's rows go through its own out-projection.
+# ---------------------------------------------------------------------------
+
+def joint_attn_unsharded(X_img, X_txt, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, heads):
+    """Returns (Y_img, Y_txt)."""
+    D = W_qkv_img.shape[1]
+    check_heads(D, heads, 1)
+    QKV = np.concatenate([linear(X_img, W_qkv_img), linear(X_txt, W_qkv_txt)], axis=0)
+    O = _heads_attention(QKV[:, :D], QKV[:, D:2 * D], QKV[:, 2 * D:], heads)
+    Mi = X_img.shape[0]
+    return linear(O[:Mi], W_o_img), linear(O[Mi:], W_o_txt)
+
+
+def joint_attn_sharded_summed(X_img, X_txt, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, heads, tp_degree):
+    D = W_qkv_img.shape[1]
+    check_degree(tp_degree)
+    check_heads(D, heads, tp_degree)
+    Dr, Mi = D // tp_degree, X_img.shape[0]
+    parts_img, parts_txt = [], []
+    for r in range(tp_degree):
+        QKV_r = np.concatenate([linear(X_img, slice_qkv_heads(W_qkv_img, heads, tp_degree, r)),
+                                linear(X_txt, slice_qkv_heads(W_qkv_txt, heads, tp_degree, r))], axis=0)
+        O_r = _heads_attention(QKV_r[:, :Dr], QKV_r[:, Dr:2 * Dr], QKV_r[:, 2 * Dr:], heads // tp_degree)
+        parts_img.append(linear(O_r[:Mi], slice_rowwise(W_o_img, tp_degree, r)))
+        parts_txt.append(linear(O_r[Mi:], slice_rowwise(W_o_txt, tp_degree, r)))
+    return reduce_partials(parts_img), reduce_partials(parts_txt)
+
+
+def joint_attn_rows(X_img, X_txt, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, heads, rows_img, rows_txt,
+                    tp_degree=1):
+    """(Y_img[rows_img], Y_txt[rows_txt]): K and V need every token of both
+    streams; queries are independent, so these rows equal the full output's."""
+    D = W_qkv_img.shape[1]
+    check_heads(D, heads, tp_degree)
+    Dr = D // tp_degree
+    rows_img, rows_txt = np.asarray(rows_img, dtype=np.int64), np.asarray(rows_txt, dtype=np.int64)
+    parts_img, parts_txt = [], []
+    for r in range(tp_degree):
+        Wi = slice_qkv_heads(W_qkv_img, heads, tp_degree, r)
+        Wt = slice_qkv_heads(W_qkv_txt, heads, tp_degree, r)
+        Q = np.concatenate([linear(X_img[rows_img], Wi[:Dr]), linear(X_txt[rows_txt], Wt[:Dr])], axis=0)
+        K = np.concatenate([linear(X_img, Wi[Dr:2 * Dr]), linear(X_txt, Wt[Dr:2 * Dr])], axis=0)
+        V = np.concatenate([linear(X_img, Wi[2 * Dr:]), linear(X_txt, Wt[2 * Dr:])], axis=0)
+        O_r = _heads_attention(Q, K, V, heads // tp_degree)
+        n = len(rows_img)
+        parts_img.append(linear(O_r[:n], slice_rowwise(W_o_img, tp_degree, r)))
+        parts_txt.append(linear(O_r[n:], slice_rowwise(W_o_txt, tp_degree, r)))
+    return reduce_partials(parts_img), reduce_partials(parts_txt)
+
+
+# ---------------------------------------------------------------------------
 # Composed block: Y = mlp_pair(attn_block(X)) (no residual, no norm).
 # ---------------------------------------------------------------------------
 

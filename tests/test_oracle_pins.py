@@ -534,3 +534,63 @@ def test_rowwise_split_input_is_the_full_projection(T):
     W = rng.integers(-3, 4, size=(7, 12)).astype(np.float64)
     b = rng.integers(-3, 4, size=7).astype(np.float64)
     assert np.array_equal(o.rowwise_split_input(X, W, b, T), X @ W.T + b)
+
+
+# ---------------------------------------------------------------------------
+# Dual-stream joint attention (image stream + text stream, one joint SDPA).
+# ---------------------------------------------------------------------------
+
+def _joint_inputs(seed, Mi=6, Mt=3, D=256):
+    rng = _rng(seed)
+    w = lambda *s: rng.standard_normal(s) / np.sqrt(s[-1])  # noqa: E731
+    return (rng.standard_normal((Mi, D)), rng.standard_normal((Mt, D)), w(3 * D, D), w(3 * D, D), w(D, D),
+            w(D, D))
+
+
+def test_joint_with_shared_weights_is_attention_over_the_concatenation():
+    Xi, Xt, Wq, _, Wo, _ = _joint_inputs(50)
+    Yi, Yt = o.joint_attn_unsharded(Xi, Xt, Wq, Wq, Wo, Wo, heads=2)
+    Y = o.attn_unsharded(np.concatenate([Xi, Xt]), Wq, Wo, heads=2)
+    assert np.allclose(np.concatenate([Yi, Yt]), Y, rtol=1e-13, atol=1e-13)
+
+
+def test_joint_without_text_is_the_image_attention():
+    Xi, Xt, Wqi, Wqt, Woi, Wot = _joint_inputs(51)
+    Yi, Yt = o.joint_attn_unsharded(Xi, Xt[:0], Wqi, Wqt, Woi, Wot, heads=2)
+    assert Yt.shape == (0, Xi.shape[1])
+    assert np.allclose(Yi, o.attn_unsharded(Xi, Wqi, Woi, heads=2), rtol=1e-13, atol=1e-13)
+
+
+def test_joint_uniform_scores_average_both_streams():
+    # Q = 0 in both streams: every score is 0, so each query averages V over ALL
+    # joint tokens.  Attending each stream on its own would average per stream.
+    Xi, Xt, Wqi, Wqt, Woi, Wot = _joint_inputs(52)
+    D = Xi.shape[1]
+    Wqi[:D] = 0
+    Wqt[:D] = 0
+    Yi, Yt = o.joint_attn_unsharded(Xi, Xt, Wqi, Wqt, Woi, Wot, heads=2)
+    V = np.concatenate([Xi @ Wqi[2 * D:].T, Xt @ Wqt[2 * D:].T])
+    vbar = V.mean(axis=0)
+    assert np.allclose(Yi, np.tile(vbar @ Woi.T, (Xi.shape[0], 1)), rtol=1e-12, atol=1e-12)
+    assert np.allclose(Yt, np.tile(vbar @ Wot.T, (Xt.shape[0], 1)), rtol=1e-12, atol=1e-12)
+    # the per-stream average differs, so this pin separates the two readings
+    assert not np.allclose(V[:Xi.shape[0]].mean(axis=0), vbar)
+
+
+def test_joint_token_order_does_not_matter():
+    Xi, Xt, Wqi, Wqt, Woi, Wot = _joint_inputs(53)
+    Yi, Yt = o.joint_attn_unsharded(Xi, Xt, Wqi, Wqt, Woi, Wot, heads=2)
+    Yt2, Yi2 = o.joint_attn_unsharded(Xt, Xi, Wqt, Wqi, Wot, Woi, heads=2)
+    assert np.allclose(Yi, Yi2, rtol=1e-12, atol=1e-13) and np.allclose(Yt, Yt2, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_joint_sharded_equals_unsharded_and_rows(T):
+    Xi, Xt, Wqi, Wqt, Woi, Wot = _joint_inputs(54 + T)
+    Yi, Yt = o.joint_attn_unsharded(Xi, Xt, Wqi, Wqt, Woi, Wot, heads=2)
+    Si, St = o.joint_attn_sharded_summed(Xi, Xt, Wqi, Wqt, Woi, Wot, 2, T)
+    assert np.allclose(Si, Yi, rtol=1e-12, atol=1e-12) and np.allclose(St, Yt, rtol=1e-12, atol=1e-12)
+    Ri, Rt = o.joint_attn_rows(Xi, Xt, Wqi, Wqt, Woi, Wot, 2, [0, 5], [2], tp_degree=T)
+    assert np.allclose(Ri, Yi[[0, 5]], rtol=1e-12, atol=1e-12) and np.allclose(Rt, Yt[[2]], rtol=1e-12, atol=1e-12)
+    with pytest.raises(ValueError):
+        o.joint_attn_sharded_summed(Xi, Xt, Wqi, Wqt, Woi, Wot, 2, 4)  # 4 does not divide 2 heads
