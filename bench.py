@@ -12,13 +12,14 @@ checks that the sequence is bit-identical to ``tp_mlp_pair``).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                        [--workload flux_mlp|flux_attn|wide_block|flux_reduce|flux_swiglu|
-                                   flux_split_input]
+                                   flux_split_input|flux_joint_attn]
 The default workload (flux_mlp) is the headline line.  The others time the
 remaining rows the same way: flux_attn (QKV head split, QKV GEMM, SDPA,
 out-projection), wide_block (attention then MLP pair at tp_degree 8, every
 row), flux_reduce (the standalone partial-sum reduction, GB/s), flux_swiglu
 (the SwiGLU pair: packed gate/up slicing, SwiGLU colwise GEMM, rowwise GEMM)
-and flux_split_input (rowwise_split_input on an FFN-out-sized projection).
+flux_split_input (rowwise_split_input on an FFN-out-sized projection) and
+flux_joint_attn (dual-stream joint attention, 4096 image + 512 text tokens).
 Under torchrun (N > 1) every rank runs the same workload on its own tokens
 (independent replicas: the layer pair has no exchange step when all shards of
 a layer live on one GPU), so per-GPU work is fixed ("weak" scaling) and the
@@ -375,6 +376,117 @@ class AttnWorkload(MlpWorkload):
                 "global_batch_tokens": c["M"] * world}
 
 
+class JointAttnWorkload(AttnWorkload):
+    """flux_joint_attn: dual-stream joint attention (image and text streams'
+    head-split QKV, one SDPA over 4096 + 512 tokens, per-stream rowwise
+    out-projections)."""
+    key = "flux_joint_attn"
+    metric = "TP dual-stream joint-attention TFLOP/s (QKV fp16, bf16 weights) on 1 B200"
+
+    def __init__(self, cfg=None):
+        import synthetic as syn
+        self.cfg = dict(cfg or syn.CONFIGS["flux_joint_attn"])
+        self.cfg["M"] = self.cfg["M_img"] + self.cfg["M_txt"]  # joint tokens (the oracle legs sample these)
+
+    def host_inputs(self, rank):
+        import synthetic as syn
+        c = self.cfg
+        d = syn.joint_attn_inputs(c["M_img"], c["M_txt"], c["D"], c["seed"])
+        if rank:
+            d["X_img"] = syn.normal_bf16((c["M_img"], c["D"]), 1.0, c["seed"] + 1000 * rank, syn.TID["X"])
+            d["X_txt"] = syn.normal_bf16((c["M_txt"], c["D"]), 1.0, c["seed"] + 1000 * rank, syn.TID["X_txt"])
+        return d
+
+    def work(self):
+        Mi, Mt, D = self.cfg["M_img"], self.cfg["M_txt"], self.cfg["D"]
+        M = Mi + Mt
+        return 2.0 * M * D * 3 * D + 4.0 * M * M * D + 2.0 * M * D * D
+
+    def kernels(self, tp, g, dev):
+        import torch
+        c = self.cfg
+        Mi, Mt, D, H, T = c["M_img"], c["M_txt"], c["D"], c["H"], c["T"]
+        M, Ds = Mi + Mt, D // T
+        b = {"wq_img": torch.empty((T, 3 * Ds, D), dtype=torch.int16, device=dev),
+             "wq_txt": torch.empty((T, 3 * Ds, D), dtype=torch.int16, device=dev),
+             "wo_img": torch.empty((T, D, Ds), dtype=torch.int16, device=dev),
+             "wo_txt": torch.empty((T, D, Ds), dtype=torch.int16, device=dev),
+             "QKV": torch.empty((T, M, 3 * Ds), dtype=torch.int16, device=dev),
+             "O": torch.empty((T, M, Ds), dtype=torch.int16, device=dev),
+             "Y_img": torch.empty((Mi, D), dtype=torch.int16, device=dev),
+             "Y_txt": torch.empty((Mt, D), dtype=torch.int16, device=dev)}
+        self.bufs = b
+        ck = tp._check
+        qkv_txt = b["QKV"].view(T, M * 3 * Ds)[:, Mi * 3 * Ds:]  # rows [Mi, M) of every shard's block
+        o_txt = b["O"].view(T, M * Ds)[:, Mi * Ds:]
+        return [
+            Kernel("slice_w_qkv_img", "GB/s", 2.0 * 3 * D * D * 2,
+                   lambda: ck(tp.tp_shard_qkv_heads_all(g["W_qkv_img"], D, H, T, b["wq_img"]), "slice")),
+            Kernel("slice_w_qkv_txt", "GB/s", 2.0 * 3 * D * D * 2,
+                   lambda: ck(tp.tp_shard_qkv_heads_all(g["W_qkv_txt"], D, H, T, b["wq_txt"]), "slice")),
+            Kernel("slice_w_o_img", "GB/s", 2.0 * D * D * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["W_o_img"], D, D, tp.TP_ROWWISE, T, b["wo_img"]), "slice")),
+            Kernel("slice_w_o_txt", "GB/s", 2.0 * D * D * 2,
+                   lambda: ck(tp.tp_shard_weight_all(g["W_o_txt"], D, D, tp.TP_ROWWISE, T, b["wo_txt"]), "slice")),
+            Kernel("qkv_gemm_img", "TFLOP/s", 2.0 * Mi * D * 3 * D,
+                   lambda: ck(tp.tp_colwise_linear_rows(g["X_img"], Mi, D, b["wq_img"], None, 3 * Ds, T, 0,
+                                                        tp.TP_OUT_F16, b["QKV"], M), "qkv img")),
+            Kernel("qkv_gemm_txt", "TFLOP/s", 2.0 * Mt * D * 3 * D,
+                   lambda: ck(tp.tp_colwise_linear_rows(g["X_txt"], Mt, D, b["wq_txt"], None, 3 * Ds, T, 0,
+                                                        tp.TP_OUT_F16, qkv_txt.data_ptr(), M), "qkv txt")),
+            Kernel("sdpa", "TFLOP/s", 4.0 * M * M * D,
+                   lambda: ck(tp.tp_sdpa_shards(b["QKV"], M, H, T, b["O"]), "sdpa")),
+            Kernel("out_gemm_img", "TFLOP/s", 2.0 * Mi * D * D,
+                   lambda: ck(tp.tp_rowwise_linear_sum_rows(b["O"], Mi, Ds, M, b["wo_img"], D, None, T, b["Y_img"]),
+                              "out img")),
+            Kernel("out_gemm_txt", "TFLOP/s", 2.0 * Mt * D * D,
+                   lambda: ck(tp.tp_rowwise_linear_sum_rows(o_txt.data_ptr(), Mt, Ds, M, b["wo_txt"], D, None, T,
+                                                            b["Y_txt"]), "out txt")),
+        ]
+
+    def one_shot(self, tp, gi, dev):
+        import torch
+        c = self.cfg
+        Mi, Mt, D, H, T = c["M_img"], c["M_txt"], c["D"], c["H"], c["T"]
+        if not hasattr(self, "_ws"):
+            self._ws = torch.empty(tp.tp_joint_attn_workspace_bytes(Mi, Mt, D, H, T), dtype=torch.uint8,
+                                   device=dev)
+            self._y = torch.empty((Mi + Mt, D), dtype=torch.int16, device=dev)
+        tp._check(tp.tp_joint_attn_block(gi["X_img"], Mi, gi["X_txt"], Mt, D, gi["W_qkv_img"], gi["W_qkv_txt"],
+                                         gi["W_o_img"], gi["W_o_txt"], H, T, self._y, self._y[Mi:], self._ws,
+                                         self._ws.numel()), "tp_joint_attn_block")
+        return self._y
+
+    e2e_call = ("tp_joint_attn_block with both streams' X and weights copied from pinned host memory and "
+                "Y_img, Y_txt copied back")
+
+    def oracle_run(self, d, rows):
+        import oracle as o
+        c = self.cfg
+        Mi, Mt, D, H, T = c["M_img"], c["M_txt"], c["D"], c["H"], c["T"]
+        M = Mi + Mt
+        f = _f64(d, ["X_img", "X_txt", "W_qkv_img", "W_qkv_txt", "W_o_img", "W_o_txt"])
+        ri = list(range(min(rows, Mi)))
+        rt = list(range(max(0, rows - Mi)))
+        t0 = time.perf_counter()
+        o.joint_attn_rows(f["X_img"], f["X_txt"], f["W_qkv_img"], f["W_qkv_txt"], f["W_o_img"], f["W_o_txt"], H,
+                          ri, rt, tp_degree=T)
+        n = len(ri) + len(rt)
+        done = 2.0 * M * D * 2 * D + 2.0 * n * D * D + 4.0 * n * M * D + 2.0 * n * D * D
+        return time.perf_counter() - t0, done
+
+    oracle_fn = "joint_attn_rows"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": (f"flux_joint_attn: TP dual-stream joint attention (image and text streams' head-split "
+                             f"QKV colwise, one per-shard SDPA over both streams' tokens, per-stream rowwise "
+                             f"out-projections with the sum fused); M_img={c['M_img']}, M_txt={c['M_txt']}, "
+                             f"D={c['D']}, {c['H']} heads x 128"),
+                "M_img": c["M_img"], "M_txt": c["M_txt"], "D": c["D"], "heads": c["H"], "tp_degree": c["T"],
+                "global_batch_tokens": (c["M_img"] + c["M_txt"]) * world}
+
+
 class BlockWorkload(AttnWorkload):
     """wide_block: attention then MLP pair at tp_degree 8 (every row a1..a7)."""
     key = "wide_block"
@@ -658,7 +770,7 @@ class SplitInputWorkload(MlpWorkload):
 
 
 WORKLOADS = {w.key: w for w in (MlpWorkload, AttnWorkload, BlockWorkload, ReduceWorkload, SwigluWorkload,
-                                SplitInputWorkload)}
+                                SplitInputWorkload, JointAttnWorkload)}
 
 
 def workload_cfg():
@@ -678,7 +790,7 @@ def cpu_baseline(wl, d, budget_s: float = 12.0):
     wl.oracle_run(d, probe)  # warm
     t, _ = wl.oracle_run(d, probe)
     rows = int(min(M, max(probe, probe * budget_s / max(t, 1e-6))))
-    if wl.key in ("flux_attn", "wide_block"):
+    if wl.key in ("flux_attn", "wide_block", "flux_joint_attn"):
         rows = min(rows, 256)  # the K/V projection of every token dominates; more rows add little
     t, done = wl.oracle_run(d, rows)
     return {"value": done / t / _scale(wl.unit), "unit": wl.unit, "cores": blas_threads(), "kind": "oracle",

@@ -20,6 +20,9 @@
  *     absolute sizes stored on the Linear, and packed rowwise;
  *   - style table, third row: "rowwise_split_input", a rowwise projection
  *     whose input is replicated, each rank slicing its part of the input;
+ *   - the note after the style table: the encoder (text) stream's projections
+ *     (add_q_proj, to_add_out, ...) follow the image stream's pattern, which
+ *     with joint attention over both streams' tokens is the dual-stream block;
  *   - section "Constraints and validation": the degree must divide the head
  *     count and every packed block, checked before any weight is split.
  *
@@ -202,6 +205,23 @@ tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s
                                 const uint16_t* W_shards, int64_t N, const uint16_t* bias,
                                 int tp_degree, uint16_t* Y, void* stream);
 
+/* Row-range forms of the two calls above, for layers whose token sets share
+ * one activation buffer (the dual-stream joint attention's Q/K/V and O):
+ *   tp_colwise_linear_rows: out is [T x out_rows x N_s] and rows [0, M) of
+ *     every shard's block are written (pass out + row_offset*N_s to write
+ *     rows [row_offset, row_offset + M)); out_rows >= M (else BAD_SHAPE).
+ *   tp_rowwise_linear_sum_rows: A_shards is [T x a_rows x K_s] and rows
+ *     [0, M) of every shard's block are read (A_shards + row_offset*K_s for
+ *     another range); a_rows >= M (else BAD_SHAPE).
+ * Other arguments and checks as tp_colwise_linear / tp_rowwise_linear_sum. */
+tp_status tp_colwise_linear_rows(const uint16_t* X, int64_t M, int64_t K,
+                                 const uint16_t* W_shards, const uint16_t* b_shards, int64_t N_s,
+                                 int tp_degree, int gelu, int out_dtype, uint16_t* out, int64_t out_rows,
+                                 void* stream);
+tp_status tp_rowwise_linear_sum_rows(const uint16_t* A_shards, int64_t M, int64_t K_s, int64_t a_rows,
+                                     const uint16_t* W_shards, int64_t N, const uint16_t* bias,
+                                     int tp_degree, uint16_t* Y, void* stream);
+
 /* SwiGLU colwise GEMM for every shard (the gate/up pair packed with blocks
  * [1, 1], section "Fused projections"):
  *   out[r] = silu(X W_gate,r^T + bg_r) * (X W_up,r^T + bu_r),   r = 0..T-1
@@ -302,6 +322,31 @@ tp_status tp_attn_prepare(const uint16_t* W_qkv, const uint16_t* W_o, int64_t D,
 size_t tp_attn_run_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree);
 tp_status tp_attn_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y,
                       void* ws, size_t ws_bytes, void* stream);
+
+/* Dual-stream joint attention (the text stream's add_q/k/v_proj and
+ * to_add_out sharded like the image stream's to_q/k/v and to_out):
+ *   QKV_r = [X_img W_qkv_img,r^T ; X_txt W_qkv_txt,r^T]   (image rows first)
+ *   O_r   = per-head SDPA of QKV_r over all M_img + M_txt tokens
+ *   Y_img = bf16( sum_r O_r[:M_img] W_o_img,r^T ),  Y_txt = bf16( sum_r O_r[M_img:] W_o_txt,r^T )
+ * X_img[M_img x D], X_txt[M_txt x D]; W_qkv_*[3D x D] = [Q; K; V] (head split
+ * as tp_shard_qkv_heads); W_o_*[D x D]; Y_img[M_img x D], Y_txt[M_txt x D].
+ * D == heads*128, heads % T == 0, no biases.  Either stream may be empty
+ * (its X and Y may then be NULL; M_txt == 0 gives tp_attn_block's result on
+ * the image stream).  Both streams' Q/K/V go into one buffer and one SDPA
+ * launch; each out-projection reads its stream's rows of O in place.
+ * Workspace: tp_joint_attn_workspace_bytes(). */
+size_t tp_joint_attn_workspace_bytes(int64_t M_img, int64_t M_txt, int64_t D, int heads, int tp_degree);
+tp_status tp_joint_attn_block(const uint16_t* X_img, int64_t M_img, const uint16_t* X_txt, int64_t M_txt,
+                              int64_t D, const uint16_t* W_qkv_img, const uint16_t* W_qkv_txt,
+                              const uint16_t* W_o_img, const uint16_t* W_o_txt, int heads, int tp_degree,
+                              uint16_t* Y_img, uint16_t* Y_txt, void* ws, size_t ws_bytes, void* stream);
+tp_status tp_joint_attn_prepare(const uint16_t* W_qkv_img, const uint16_t* W_qkv_txt,
+                                const uint16_t* W_o_img, const uint16_t* W_o_txt, int64_t D, int heads,
+                                int tp_degree, void* stream, void** handle);
+size_t tp_joint_attn_run_workspace_bytes(int64_t M_img, int64_t M_txt, int64_t D, int heads, int tp_degree);
+tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, const uint16_t* X_txt,
+                            int64_t M_txt, uint16_t* Y_img, uint16_t* Y_txt, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /* Frees a handle from tp_*_prepare (synchronises the device first). NULL is a no-op. */
 void tp_destroy(void* handle);

@@ -40,6 +40,7 @@ TID = {
     "W_qkv": 5, "W_o": 6,
     "W_up2": 7, "b_up2": 8, "W_down2": 9, "b_down2": 10,
     "W_in": 11, "b_in": 12, "W_out": 13, "b_out": 14,
+    "X_txt": 15, "W_qkv_txt": 16, "W_o_txt": 17,
 }
 
 _CHUNK = 1 << 22
@@ -170,6 +171,19 @@ def swiglu_inputs(M: int, D: int, F: int, seed: int) -> dict:
     }
 
 
+def joint_attn_inputs(M_img: int, M_txt: int, D: int, seed: int) -> dict:
+    """Inputs of dual-stream joint attention: the image stream uses the
+    attention block's ids (X, W_qkv, W_o), the text stream its own."""
+    return {
+        "X_img": normal_bf16((M_img, D), 1.0, seed, TID["X"]),
+        "X_txt": normal_bf16((M_txt, D), 1.0, seed, TID["X_txt"]),
+        "W_qkv_img": normal_bf16((3 * D, D), 1.0 / np.sqrt(D), seed, TID["W_qkv"]),
+        "W_qkv_txt": normal_bf16((3 * D, D), 1.0 / np.sqrt(D), seed, TID["W_qkv_txt"]),
+        "W_o_img": normal_bf16((D, D), 1.0 / np.sqrt(D), seed, TID["W_o"]),
+        "W_o_txt": normal_bf16((D, D), 1.0 / np.sqrt(D), seed, TID["W_o_txt"]),
+    }
+
+
 # The layer configurations exercised by the tests and the benchmark.
 CONFIGS = {
     "tiny_mlp": dict(kind="mlp", M=64, D=128, F=512, T=2, seed=0),
@@ -179,4 +193,6 @@ CONFIGS = {
     "wide_block": dict(kind="block", M=16384, D=6144, H=48, F=24576, T=8, seed=3),
     # SwiGLU pair, gate and up packed with blocks [1, 1], mlp_ratio 3 (F = 3 D)
     "flux_swiglu": dict(kind="swiglu", M=4608, D=3072, F=9216, T=4, seed=4),
+    # dual-stream joint attention: 4096 image + 512 text tokens, one SDPA over both
+    "flux_joint_attn": dict(kind="joint", M_img=4096, M_txt=512, D=3072, H=24, T=4, seed=6),
 }

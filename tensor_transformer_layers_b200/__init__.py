@@ -75,6 +75,13 @@ SIGNATURES = {
     "tp_swiglu_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "tp_swiglu_mlp_pair": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "tp_swiglu_prepare": (_I, [_P, _P, _P, _P, _I64, _I64, _I, _P, ctypes.POINTER(_P)]),
+    "tp_joint_attn_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I, _I]),
+    "tp_joint_attn_block": (_I, [_P, _I64, _P, _I64, _I64, _P, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "tp_joint_attn_prepare": (_I, [_P, _P, _P, _P, _I64, _I, _I, _P, ctypes.POINTER(_P)]),
+    "tp_joint_attn_run_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I, _I]),
+    "tp_joint_attn_run": (_I, [_P, _P, _I64, _P, _I64, _P, _P, _P, _SZ, _P]),
+    "tp_colwise_linear_rows": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _I, _P, _I64, _P]),
+    "tp_rowwise_linear_sum_rows": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
 }
 
 _lib = None
@@ -292,6 +299,44 @@ def tp_swiglu_prepare(W_in, b_in, W_out, b_out, D, F, tp_degree, stream=None):
     return st, h.value
 
 
+def tp_colwise_linear_rows(X, M, K, W_shards, b_shards, N_s, tp_degree, gelu, out_dtype, out, out_rows,
+                           stream=None) -> int:
+    return lib().tp_colwise_linear_rows(_ptr(X), M, K, _ptr(W_shards), _ptr(b_shards), N_s, tp_degree,
+                                        int(bool(gelu)), int(out_dtype), _ptr(out), out_rows, _stream(stream))
+
+
+def tp_rowwise_linear_sum_rows(A_shards, M, K_s, a_rows, W_shards, N, bias, tp_degree, Y, stream=None) -> int:
+    return lib().tp_rowwise_linear_sum_rows(_ptr(A_shards), M, K_s, a_rows, _ptr(W_shards), N, _ptr(bias),
+                                            tp_degree, _ptr(Y), _stream(stream))
+
+
+def tp_joint_attn_workspace_bytes(M_img, M_txt, D, heads, tp_degree) -> int:
+    return lib().tp_joint_attn_workspace_bytes(M_img, M_txt, D, heads, tp_degree)
+
+
+def tp_joint_attn_run_workspace_bytes(M_img, M_txt, D, heads, tp_degree) -> int:
+    return lib().tp_joint_attn_run_workspace_bytes(M_img, M_txt, D, heads, tp_degree)
+
+
+def tp_joint_attn_block(X_img, M_img, X_txt, M_txt, D, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, heads, tp_degree,
+                        Y_img, Y_txt, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_joint_attn_block(_ptr(X_img), M_img, _ptr(X_txt), M_txt, D, _ptr(W_qkv_img), _ptr(W_qkv_txt),
+                                     _ptr(W_o_img), _ptr(W_o_txt), heads, tp_degree, _ptr(Y_img), _ptr(Y_txt),
+                                     _ptr(ws), ws_bytes, _stream(stream))
+
+
+def tp_joint_attn_prepare(W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, D, heads, tp_degree, stream=None):
+    h = _P()
+    st = lib().tp_joint_attn_prepare(_ptr(W_qkv_img), _ptr(W_qkv_txt), _ptr(W_o_img), _ptr(W_o_txt), D, heads,
+                                     tp_degree, _stream(stream), ctypes.byref(h))
+    return st, h.value
+
+
+def tp_joint_attn_run(handle, X_img, M_img, X_txt, M_txt, Y_img, Y_txt, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_joint_attn_run(handle, _ptr(X_img), M_img, _ptr(X_txt), M_txt, _ptr(Y_img), _ptr(Y_txt),
+                                   _ptr(ws), ws_bytes, _stream(stream))
+
+
 # --------------------------------------------------------------------------- convenience
 def _u16(t: torch.Tensor) -> torch.Tensor:
     """bf16 bit patterns travel as 16-bit tensors; accept bfloat16 or int16/uint16 storage."""
@@ -340,6 +385,22 @@ def attn_block(X, W_qkv, W_o, heads: int, tp_degree: int, stream=None) -> torch.
     ws = _workspace(nb, X.device)
     _check(tp_attn_block(X, M, D, W_qkv, W_o, heads, tp_degree, Y, ws, nb, stream), "tp_attn_block")
     return Y
+
+
+def joint_attn_block(X_img, X_txt, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, heads: int, tp_degree: int,
+                     stream=None):
+    """One-shot dual-stream joint attention; returns (Y_img, Y_txt) (bf16)."""
+    for t in (X_img, X_txt, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt):
+        _u16(t)
+    Mi, D = X_img.shape
+    Mt = X_txt.shape[0]
+    Yi = torch.empty((Mi, D), dtype=torch.bfloat16, device=X_img.device)
+    Yt = torch.empty((Mt, D), dtype=torch.bfloat16, device=X_img.device)
+    nb = tp_joint_attn_workspace_bytes(Mi, Mt, D, heads, tp_degree)
+    ws = _workspace(nb, X_img.device)
+    _check(tp_joint_attn_block(X_img, Mi, X_txt, Mt, D, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, heads, tp_degree,
+                               Yi, Yt, ws, nb, stream), "tp_joint_attn_block")
+    return Yi, Yt
 
 
 class MlpPair:
@@ -412,6 +473,42 @@ class AttnBlock:
         ws, nb = self.workspace(M, X.device)
         _check(tp_attn_run(self.handle, X, M, Y, ws, nb, stream), "tp_attn_run")
         return Y
+
+    def close(self):
+        if self.handle:
+            tp_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001
+            pass
+
+
+class JointAttnBlock:
+    """Shards once (tp_joint_attn_prepare), runs many times (tp_joint_attn_run)."""
+
+    def __init__(self, W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, heads: int, tp_degree: int, stream=None):
+        self.D = W_qkv_img.shape[1]
+        self.heads = heads
+        self.T = tp_degree
+        self.handle = None
+        st, self.handle = tp_joint_attn_prepare(W_qkv_img, W_qkv_txt, W_o_img, W_o_txt, self.D, heads, tp_degree,
+                                                stream)
+        _check(st, "tp_joint_attn_prepare")
+        self._ws = None
+
+    def __call__(self, X_img, X_txt, stream=None):
+        Mi, Mt = X_img.shape[0], X_txt.shape[0]
+        Yi = torch.empty((Mi, self.D), dtype=torch.bfloat16, device=X_img.device)
+        Yt = torch.empty((Mt, self.D), dtype=torch.bfloat16, device=X_img.device)
+        nb = tp_joint_attn_run_workspace_bytes(Mi, Mt, self.D, self.heads, self.T)
+        if self._ws is None or self._ws.numel() < nb:
+            self._ws = _workspace(nb, X_img.device)
+        _check(tp_joint_attn_run(self.handle, X_img, Mi, X_txt, Mt, Yi, Yt, self._ws, nb, stream),
+               "tp_joint_attn_run")
+        return Yi, Yt
 
     def close(self):
         if self.handle:

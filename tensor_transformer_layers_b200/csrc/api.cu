@@ -30,6 +30,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kMlpMagic = 0x54504D4C50484E44ull;   // "TPMLPHND"
 constexpr uint64_t kAttnMagic = 0x5450415454484E44ull;  // "TPATTHND"
+constexpr uint64_t kJointMagic = 0x54504A4E54484E44ull; // "TPJNTHND"
 constexpr int64_t kMaxDim = int64_t(1) << 31;           // TMA coordinates are 32-bit
 constexpr int kMaxPackedBlocks = 64;
 
@@ -99,9 +100,9 @@ int current_device_context(int* num_sms, int** err) {
 }
 
 static CUresult make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
-                            uint64_t d2, uint32_t box0, uint32_t box1, uint32_t box2 = 1) {
+                            uint64_t d2, uint32_t box0, uint32_t box1, uint32_t box2 = 1, uint64_t d1_stride = 0) {
   const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};  // bytes, dims 1 and 2
+  const cuuint64_t strides[2] = {d0 * 2, d0 * (d1_stride ? d1_stride : d1) * 2};  // bytes, dims 1 and 2
   const cuuint32_t box[3] = {box0, box1, box2};
   const cuuint32_t estride[3] = {1, 1, 1};
   return g_encode(map, dt, 3, const_cast<void*>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -109,8 +110,8 @@ static CUresult make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void
 }
 
 CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
-                          uint32_t box1) {
-  return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d0, d1, d2, box0, box1);
+                          uint32_t box1, uint64_t d1_stride) {
+  return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d0, d1, d2, box0, box1, 1, d1_stride);
 }
 
 CUresult make_map_3d_bf16_box(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
@@ -130,8 +131,10 @@ namespace {
 // ---------------------------------------------------------------------------
 
 // colwise: out[g] = epi(X . W[g]^T + b[g]), g < T.
+// out_rows: rows of each group's output block (0 = M; larger when `out` is a
+// row range of a taller [T][out_rows][Ns] buffer).
 tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, const uint16_t* b,
-                      int64_t Ns, int T, int gelu, int out_f16, uint16_t* out, cudaStream_t s) {
+                      int64_t Ns, int T, int gelu, int out_f16, uint16_t* out, cudaStream_t s, int64_t out_rows = 0) {
   if (M == 0) return TP_OK;
   const GemmOperand A{X, uint64_t(K), uint64_t(M), 1};
   const GemmOperand B{W, uint64_t(K), uint64_t(Ns), uint64_t(T)};
@@ -143,7 +146,7 @@ tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, c
   a.groups = T;
   a.a_follows_shard = 0;
   a.out = out;
-  a.out_gstride = M * Ns;
+  a.out_gstride = (out_rows ? out_rows : M) * Ns;
   a.ldo = Ns;
   a.bias = b;
   a.bias_gstride = Ns;
@@ -153,11 +156,12 @@ tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, c
   return launch_gemm(A, B, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
-// rowwise: Y = sum_r A[r] . W[r]^T + bias.
+// rowwise: Y = sum_r A[r] . W[r]^T + bias.  a_rows: rows of each shard's A
+// block in memory (0 = M; larger when A is a row range of a taller buffer).
 tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, const uint16_t* W, int64_t N,
-                      const uint16_t* bias, int T, uint16_t* Y, cudaStream_t s) {
+                      const uint16_t* bias, int T, uint16_t* Y, cudaStream_t s, int64_t a_rows = 0) {
   if (M == 0) return TP_OK;
-  const GemmOperand Aop{A, uint64_t(Ks), uint64_t(M), uint64_t(T)};
+  const GemmOperand Aop{A, uint64_t(Ks), uint64_t(M), uint64_t(T), uint64_t(a_rows)};
   const GemmOperand Bop{W, uint64_t(Ks), uint64_t(N), uint64_t(T)};
   GemmArgs a{};
   a.M = int(M);
@@ -404,6 +408,24 @@ tp_status attn_forward(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t D, 
   return run_rowwise(di, O, M, Ds, w_o_sh, D, nullptr, T, Y, s);
 }
 
+// Dual-stream joint attention on sharded weights: both streams' head-split
+// QKV land in one [T][Mi+Mt][3*Ds] buffer (image rows first), one SDPA runs
+// over the joint tokens, and each stream's rows of O go through its own
+// rowwise out-projection (read in place as a row range of O).
+tp_status joint_attn_forward(DeviceInfo* di, const uint16_t* X_img, int64_t Mi, const uint16_t* X_txt, int64_t Mt,
+                             int64_t D, int heads, int T, const uint16_t* wq_img, const uint16_t* wq_txt,
+                             const uint16_t* wo_img, const uint16_t* wo_txt, uint16_t* QKV, uint16_t* O,
+                             uint16_t* Y_img, uint16_t* Y_txt, cudaStream_t s) {
+  const int64_t Ds = D / T, M = Mi + Mt;
+  tp_status st = run_colwise(di, X_img, Mi, D, wq_img, nullptr, 3 * Ds, T, 0, 1, QKV, s, M);
+  if (st != TP_OK) return st;
+  if ((st = run_colwise(di, X_txt, Mt, D, wq_txt, nullptr, 3 * Ds, T, 0, 1, QKV + Mi * 3 * Ds, s, M)) != TP_OK)
+    return st;
+  if ((st = run_sdpa(di, QKV, M, heads, T, O, s)) != TP_OK) return st;
+  if ((st = run_rowwise(di, O, Mi, Ds, wo_img, D, nullptr, T, Y_img, s, M)) != TP_OK) return st;
+  return run_rowwise(di, O + Mi * Ds, Mt, Ds, wo_txt, D, nullptr, T, Y_txt, s, M);
+}
+
 struct MlpHandle {
   uint64_t magic;
   int device;
@@ -424,6 +446,47 @@ struct AttnHandle {
   uint16_t* w_qkv;  // [T][3D/T][D]
   uint16_t* w_o;    // [T][D][D/T]
 };
+
+struct JointHandle {
+  uint64_t magic;
+  int device;
+  int64_t D;
+  int heads, T;
+  uint16_t* w_qkv_img;  // [T][3D/T][D]
+  uint16_t* w_qkv_txt;
+  uint16_t* w_o_img;    // [T][D][D/T]
+  uint16_t* w_o_txt;
+};
+
+struct JointLayout {
+  size_t w_qkv_img, w_qkv_txt, w_o_img, w_o_txt, qkv, o, total;
+};
+JointLayout joint_layout(int64_t M, int64_t D, bool with_weights) {
+  JointLayout L{};
+  size_t off = 0;
+  if (with_weights) {
+    const size_t wq = up256(size_t(3) * D * D * 2), wo = up256(size_t(D) * D * 2);
+    L.w_qkv_img = off;
+    off += wq;
+    L.w_qkv_txt = off;
+    off += wq;
+    L.w_o_img = off;
+    off += wo;
+    L.w_o_txt = off;
+    off += wo;
+  }
+  L.qkv = off;
+  off += up256(size_t(M) * 3 * D * 2);
+  L.o = off;
+  off += up256(size_t(M) * D * 2);
+  L.total = off;
+  return L;
+}
+
+tp_status check_joint_shape(int64_t Mi, int64_t Mt, int64_t D, int heads, int T) {
+  if (Mi < 0 || Mt < 0) return TP_ERR_BAD_SHAPE;
+  return check_attn_shape(Mi + Mt, D, heads, T);
+}
 
 }  // namespace
 }  // namespace tp
@@ -614,6 +677,37 @@ tp_status tp_rowwise_linear_sum(const uint16_t* A_shards, int64_t M, int64_t K_s
   DeviceInfo* di = nullptr;
   if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
   return run_rowwise(di, A_shards, M, K_s, W_shards, N, bias, tp_degree, Y, as_stream(stream));
+}
+
+tp_status tp_colwise_linear_rows(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W_shards,
+                                 const uint16_t* b_shards, int64_t N_s, int tp_degree, int gelu, int out_dtype,
+                                 uint16_t* out, int64_t out_rows, void* stream) {
+  if (out_rows < M || out_rows >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (!X || !W_shards || !out) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || K < 1 || N_s < 1 || M >= kMaxDim || K >= kMaxDim || N_s * tp_degree >= kMaxDim)
+    return TP_ERR_BAD_SHAPE;
+  if (!al16(X) || !al16(W_shards) || !al16(out) || (b_shards && !al16(b_shards))) return TP_ERR_ALIGNMENT;
+  if (K % 8 != 0 || N_s % 8 != 0) return TP_ERR_ALIGNMENT;
+  if (out_dtype != TP_OUT_BF16 && out_dtype != TP_OUT_F16) return TP_ERR_BAD_STYLE;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_colwise(di, X, M, K, W_shards, b_shards, N_s, tp_degree, gelu ? 1 : 0, out_dtype == TP_OUT_F16 ? 1 : 0,
+                     out, as_stream(stream), out_rows);
+}
+
+tp_status tp_rowwise_linear_sum_rows(const uint16_t* A_shards, int64_t M, int64_t K_s, int64_t a_rows,
+                                     const uint16_t* W_shards, int64_t N, const uint16_t* bias, int tp_degree,
+                                     uint16_t* Y, void* stream) {
+  if (a_rows < M || a_rows >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (!A_shards || !W_shards || !Y) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || K_s < 1 || N < 1 || M >= kMaxDim || K_s >= kMaxDim || N >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (!al16(A_shards) || !al16(W_shards) || !al16(Y) || (bias && !al16(bias))) return TP_ERR_ALIGNMENT;
+  if (K_s % 8 != 0 || N % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_rowwise(di, A_shards, M, K_s, W_shards, N, bias, tp_degree, Y, as_stream(stream), a_rows);
 }
 
 tp_status tp_colwise_swiglu(const uint16_t* X, int64_t M, int64_t K, const uint16_t* W_shards,
@@ -906,6 +1000,95 @@ tp_status tp_attn_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y, v
                       reinterpret_cast<uint16_t*>(w + L.o), Y, as_stream(stream));
 }
 
+// ----------------------------------------------------------------------- dual-stream joint attention
+size_t tp_joint_attn_workspace_bytes(int64_t M_img, int64_t M_txt, int64_t D, int heads, int tp_degree) {
+  if (check_joint_shape(M_img, M_txt, D, heads, tp_degree) != TP_OK) return 0;
+  return joint_layout(M_img + M_txt, D, true).total;
+}
+
+size_t tp_joint_attn_run_workspace_bytes(int64_t M_img, int64_t M_txt, int64_t D, int heads, int tp_degree) {
+  if (check_joint_shape(M_img, M_txt, D, heads, tp_degree) != TP_OK) return 0;
+  return joint_layout(M_img + M_txt, D, false).total;
+}
+
+tp_status tp_joint_attn_block(const uint16_t* X_img, int64_t M_img, const uint16_t* X_txt, int64_t M_txt, int64_t D,
+                              const uint16_t* W_qkv_img, const uint16_t* W_qkv_txt, const uint16_t* W_o_img,
+                              const uint16_t* W_o_txt, int heads, int tp_degree, uint16_t* Y_img, uint16_t* Y_txt,
+                              void* ws, size_t ws_bytes, void* stream) {
+  if (!W_qkv_img || !W_qkv_txt || !W_o_img || !W_o_txt) return TP_ERR_NULL;
+  if ((M_img > 0 && (!X_img || !Y_img)) || (M_txt > 0 && (!X_txt || !Y_txt))) return TP_ERR_NULL;
+  tp_status st = check_joint_shape(M_img, M_txt, D, heads, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(X_img) || !al16(X_txt) || !al16(Y_img) || !al16(Y_txt) || !al16(W_qkv_img) || !al16(W_qkv_txt) ||
+      !al16(W_o_img) || !al16(W_o_txt))
+    return TP_ERR_ALIGNMENT;
+  if (M_img + M_txt == 0) return TP_OK;
+  const JointLayout L = joint_layout(M_img + M_txt, D, true);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  auto at = [w](size_t off) { return reinterpret_cast<uint16_t*>(w + off); };
+  if ((st = slice_all_qkv(W_qkv_img, D, tp_degree, at(L.w_qkv_img), s)) != TP_OK) return st;
+  if ((st = slice_all_qkv(W_qkv_txt, D, tp_degree, at(L.w_qkv_txt), s)) != TP_OK) return st;
+  if ((st = slice_all_rowwise(W_o_img, D, D, tp_degree, at(L.w_o_img), s)) != TP_OK) return st;
+  if ((st = slice_all_rowwise(W_o_txt, D, D, tp_degree, at(L.w_o_txt), s)) != TP_OK) return st;
+  return joint_attn_forward(di, X_img, M_img, X_txt, M_txt, D, heads, tp_degree, at(L.w_qkv_img), at(L.w_qkv_txt),
+                            at(L.w_o_img), at(L.w_o_txt), at(L.qkv), at(L.o), Y_img, Y_txt, s);
+}
+
+tp_status tp_joint_attn_prepare(const uint16_t* W_qkv_img, const uint16_t* W_qkv_txt, const uint16_t* W_o_img,
+                                const uint16_t* W_o_txt, int64_t D, int heads, int tp_degree, void* stream,
+                                void** handle) {
+  if (!W_qkv_img || !W_qkv_txt || !W_o_img || !W_o_txt || !handle) return TP_ERR_NULL;
+  tp_status st = check_attn_shape(0, D, heads, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(W_qkv_img) || !al16(W_qkv_txt) || !al16(W_o_img) || !al16(W_o_txt)) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  JointHandle* h = new JointHandle{};
+  h->magic = kJointMagic;
+  cudaGetDevice(&h->device);
+  h->D = D;
+  h->heads = heads;
+  h->T = tp_degree;
+  const size_t wq = size_t(3) * D * D * 2, wo = size_t(D) * D * 2;
+  bool ok = cudaMalloc(&h->w_qkv_img, wq) == cudaSuccess && cudaMalloc(&h->w_qkv_txt, wq) == cudaSuccess &&
+            cudaMalloc(&h->w_o_img, wo) == cudaSuccess && cudaMalloc(&h->w_o_txt, wo) == cudaSuccess;
+  ok = ok && slice_all_qkv(W_qkv_img, D, tp_degree, h->w_qkv_img, s) == TP_OK &&
+       slice_all_qkv(W_qkv_txt, D, tp_degree, h->w_qkv_txt, s) == TP_OK &&
+       slice_all_rowwise(W_o_img, D, D, tp_degree, h->w_o_img, s) == TP_OK &&
+       slice_all_rowwise(W_o_txt, D, D, tp_degree, h->w_o_txt, s) == TP_OK;
+  if (!ok) {
+    tp_destroy(h);
+    return TP_ERR_CUDA;
+  }
+  *handle = h;
+  return TP_OK;
+}
+
+tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, const uint16_t* X_txt, int64_t M_txt,
+                            uint16_t* Y_img, uint16_t* Y_txt, void* ws, size_t ws_bytes, void* stream) {
+  JointHandle* h = static_cast<JointHandle*>(handle);
+  if (!h) return TP_ERR_BAD_HANDLE;
+  if (h->magic != kJointMagic) return TP_ERR_BAD_HANDLE;
+  if ((M_img > 0 && (!X_img || !Y_img)) || (M_txt > 0 && (!X_txt || !Y_txt))) return TP_ERR_NULL;
+  tp_status st = check_joint_shape(M_img, M_txt, h->D, h->heads, h->T);
+  if (st != TP_OK) return st;
+  if (!al16(X_img) || !al16(X_txt) || !al16(Y_img) || !al16(Y_txt)) return TP_ERR_ALIGNMENT;
+  if (M_img + M_txt == 0) return TP_OK;
+  const JointLayout L = joint_layout(M_img + M_txt, h->D, false);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  return joint_attn_forward(di, X_img, M_img, X_txt, M_txt, h->D, h->heads, h->T, h->w_qkv_img, h->w_qkv_txt,
+                            h->w_o_img, h->w_o_txt, reinterpret_cast<uint16_t*>(w + L.qkv),
+                            reinterpret_cast<uint16_t*>(w + L.o), Y_img, Y_txt, as_stream(stream));
+}
+
 void tp_destroy(void* handle) {
   if (!handle) return;
   const uint64_t magic = *static_cast<uint64_t*>(handle);
@@ -923,6 +1106,15 @@ void tp_destroy(void* handle) {
     cudaDeviceSynchronize();
     cudaFree(h->w_qkv);
     cudaFree(h->w_o);
+    h->magic = 0;
+    delete h;
+  } else if (magic == kJointMagic) {
+    JointHandle* h = static_cast<JointHandle*>(handle);
+    cudaDeviceSynchronize();
+    cudaFree(h->w_qkv_img);
+    cudaFree(h->w_qkv_txt);
+    cudaFree(h->w_o_img);
+    cudaFree(h->w_o_txt);
     h->magic = 0;
     delete h;
   }

@@ -617,7 +617,7 @@ int max_active_pairs(int num_sms) {
 // [rows][z][K_s]), with a box of 64 x box_rows rows either way.
 CUresult make_a_map(CUtensorMap* map, const GemmOperand& A, const GemmArgs& a, uint32_t box_rows) {
   if (a.a_split_input) return make_map_3d_bf16_box(map, A.base, A.k, A.z, A.rows, BK, 1, box_rows);
-  return make_map_3d_bf16(map, A.base, A.k, A.rows, A.z, BK, box_rows);
+  return make_map_3d_bf16(map, A.base, A.k, A.rows, A.z, BK, box_rows, A.zrows);
 }
 
 }  // namespace
@@ -629,7 +629,7 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
   if (a.M >= BM2) {
     // CTA-pair kernel: each CTA loads 128-row halves of both operands.
     if (make_a_map(&amap, A, a, 128) != CUDA_SUCCESS ||
-        make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, 128) != CUDA_SUCCESS)
+        make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, 128, B.zrows) != CUDA_SUCCESS)
       return note_cuda_error("gemm (CTA pairs): tensor map encode", cudaErrorInvalidValue);
     cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
     if (e != cudaSuccess) return note_cuda_error("gemm (CTA pairs): set shared memory size", e);
@@ -655,7 +655,7 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
     return note_cuda_error("gemm (CTA pairs): launch", e);
   }
   if (make_a_map(&amap, A, a, BM1) != CUDA_SUCCESS ||
-      make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, a.swiglu ? BN1 / 2 : BN1) != CUDA_SUCCESS)
+      make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, a.swiglu ? BN1 / 2 : BN1, B.zrows) != CUDA_SUCCESS)
     return note_cuda_error("gemm: tensor map encode", cudaErrorInvalidValue);
   const int m_tiles = (a.M + BM1 - 1) / BM1;
   const int n_tiles = (a.N + (a.swiglu ? BN1 / 2 : BN1) - 1) / (a.swiglu ? BN1 / 2 : BN1);

@@ -64,10 +64,13 @@ struct GemmArgs {
 
 // A bf16 operand seen as a 3-D tensor {k (contiguous), rows, z}: the GEMM
 // builds its TMA maps from this (box sizes depend on the kernel it picks).
-// With a_split_input the A operand's memory is [rows][z][k] instead.
+// z-slices lie zrows rows apart in memory (0: zrows = rows), so an operand
+// can be a row range of a taller [z][zrows][k] buffer; rows past `rows` read
+// as zeros.  With a_split_input the A operand's memory is [rows][z][k] instead.
 struct GemmOperand {
   const void* base;
   uint64_t k, rows, z;
+  uint64_t zrows = 0;
 };
 
 cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms, cudaStream_t s);
@@ -102,9 +105,10 @@ cudaError_t note_cuda_error(const char* where, cudaError_t e, const char* detail
 // Returns a tp_status value.
 int current_device_context(int* num_sms, int** err);
 
-// Host helpers (api.cu).
+// Host helpers (api.cu).  d1_stride: elements of dim 1 between dim-2 slices
+// (0 = d1, the packed layout).
 CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                          uint32_t box0, uint32_t box1);
+                          uint32_t box0, uint32_t box1, uint64_t d1_stride = 0);
 CUresult make_map_3d_bf16_box(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                               uint32_t box0, uint32_t box1, uint32_t box2);
 CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,

@@ -164,3 +164,27 @@ def test_swiglu_and_split_input_checks():
     assert tp.tp_rowwise_split_input_linear(None, 64, 128, A, 64, None, 2, A, stream=0) == S["TP_ERR_NULL"]
     # the split-input style slices its weight like rowwise
     assert tp.tp_shard_weight(A, 8, 24, tp.TP_ROWWISE_SPLIT_INPUT, 5, 0, A, stream=0) == S["TP_ERR_INDIVISIBLE"]
+
+
+def test_joint_attn_checks():
+    ws = 1 << 30
+    up = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    Mi, Mt, D = 4096, 512, 3072
+    assert tp.tp_joint_attn_workspace_bytes(Mi, Mt, D, 24, 4) == (2 * up(3 * D * D * 2) + 2 * up(D * D * 2)
+                                                                  + up((Mi + Mt) * 3 * D * 2) + up((Mi + Mt) * D * 2))
+    assert tp.tp_joint_attn_run_workspace_bytes(Mi, Mt, D, 24, 4) == up((Mi + Mt) * 3 * D * 2) + up((Mi + Mt) * D * 2)
+    assert tp.tp_joint_attn_workspace_bytes(Mi, -1, D, 24, 4) == 0
+    assert tp.tp_joint_attn_workspace_bytes(Mi, Mt, D, 24, 5) == 0
+    j = tp.tp_joint_attn_block
+    assert j(A, 64, A, 32, 768, A, A, A, A, 6, 4, A, A, A, ws, stream=0) == S["TP_ERR_HEADS_INDIVISIBLE"]
+    assert j(A, 64, A, 32, 700, A, A, A, A, 6, 2, A, A, A, ws, stream=0) == S["TP_ERR_BAD_SHAPE"]
+    assert j(A, 64, A, -2, 768, A, A, A, A, 6, 2, A, A, A, ws, stream=0) == S["TP_ERR_BAD_SHAPE"]
+    assert j(A, 64, A, 32, 768, A, None, A, A, 6, 2, A, A, A, ws, stream=0) == S["TP_ERR_NULL"]
+    assert j(A, 64, None, 32, 768, A, A, A, A, 6, 2, A, A, A, ws, stream=0) == S["TP_ERR_NULL"]
+    assert j(A, 64, A, 32, 768, A, A, A, A, 6, 2, A, A, A, 10, stream=0) == S["TP_ERR_WORKSPACE"]
+    assert j(A, 64, A, 32, 768, A, A, A, A, 6, 2, A + 8, A, A, ws, stream=0) == S["TP_ERR_ALIGNMENT"]
+    # an empty text stream may pass NULL pointers for it; both empty is a no-op
+    assert j(A, 0, None, 0, 768, A, A, A, A, 6, 2, None, None, None, 0, stream=0) == 0
+    st, h = tp.tp_joint_attn_prepare(A, A, A, A, 768, 6, 4, stream=0)
+    assert st == S["TP_ERR_HEADS_INDIVISIBLE"] and not h
+    assert tp.tp_joint_attn_run(None, A, 64, A, 32, A, A, A, ws, stream=0) == S["TP_ERR_BAD_HANDLE"]
