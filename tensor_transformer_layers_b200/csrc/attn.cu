@@ -156,27 +156,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t sq0 = smem_u32(smem + kQOff);
+      // Descriptors are computed once: a descriptor's low field is the start
+      // address >> 4, so moving inside shared memory is an integer add.
+      const uint64_t dq0 = sdesc_sw128(smem_u32(smem + kQOff), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(smem + kKVOff), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(smem + kKVOff + 2 * kBox), kBox, 1024);
       auto issue_s = [&](int t, int j) {
-        const uint32_t sq = sq0 + uint32_t(t * kQBytes);
-        const uint32_t sk = smem_u32(smem + kKVOff + (j & 1) * kKVBytes);
+        const uint64_t dq = dq0 + uint64_t((t * kQBytes) >> 4);
+        const uint64_t dk = dk0 + uint64_t(((j & 1) * kKVBytes) >> 4);
         const uint32_t d = tmem_base + kColS0 + uint32_t(t * 128);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = uint32_t((kk >> 2) * kBox + (kk & 3) * 32);
-          umma_ss(d, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), kIdescS, kk != 0 ? 1u : 0u);
+          const uint64_t off = uint64_t(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+          umma_ss(d, dq + off, dk + off, kIdescS, kk != 0 ? 1u : 0u);
         }
         umma_commit(&s_full[t]);
       };
       auto issue_pv = [&](int t, int j) {
-        const uint32_t sv = smem_u32(smem + kKVOff + (j & 1) * kKVBytes + 2 * kBox);
+        const uint64_t dv = dv0 + uint64_t(((j & 1) * kKVBytes) >> 4);
         const uint32_t d = tmem_base + kColO0 + uint32_t(t * 128);
         const uint32_t a = tmem_base + kColS0 + uint32_t(t * 128);
 #pragma unroll
         for (int kk = 0; kk < kBKV / 16; ++kk) {
           // 16 keys per step: P columns kk*8.. (fp16 pairs); rows kk*16.. of both V boxes
-          umma_ts(d, a + uint32_t(kk * 8), sdesc_sw128(sv + uint32_t(kk * 16 * 128), kBox, 1024), kIdescPV,
-                  (j | kk) != 0 ? 1u : 0u);
+          umma_ts(d, a + uint32_t(kk * 8), dv + uint64_t((kk * 16 * 128) >> 4), kIdescPV, (j | kk) != 0 ? 1u : 0u);
         }
       };
       bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
@@ -253,9 +256,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBKV; ++i)
           if (kv0 + i >= p.M) s[i] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max over 8 independent chains, combined at the end (a shorter
+      // dependency chain than one running max over 128 values)
+      float m8[8];
 #pragma unroll
-      for (int i = 0; i < kBKV; ++i) mx = fmaxf(mx, s[i]);
+      for (int a = 0; a < 8; ++a) m8[a] = s[a];
+#pragma unroll
+      for (int i = 8; i < kBKV; ++i) m8[i & 7] = fmaxf(m8[i & 7], s[i]);
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= sl2;
       if (j == 0) {
         m_run = mx;
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      float lsum = 0.f;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent partial sums
 #pragma unroll
       for (int c = 0; c < kBKV / 32; ++c) {
         uint32_t pk[16];
@@ -289,12 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 16; ++i) {
           const float p0 = ex2_approx(fmaf(s[c * 32 + 2 * i], sl2, -m_run));
           const float p1 = ex2_approx(fmaf(s[c * 32 + 2 * i + 1], sl2, -m_run));
-          lsum += p0 + p1;
+          l4[i & 3] += p0 + p1;
           pk[i] = pack_f16x2(p0, p1);
         }
         tmem_st16(tmem_base + lane_off + colS + uint32_t(c * 16), pk);  // P over S's first 64 columns
       }
-      l_run += lsum;
+      l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
