@@ -119,6 +119,17 @@ CUresult make_map_3d_bf16_box(CUtensorMap* map, const void* base, uint64_t d0, u
   return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, d0, d1, d2, box0, box1, box2);
 }
 
+CUresult make_map_out_u16(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t g, uint64_t row_stride,
+                          uint64_t group_stride) {
+  const cuuint64_t dims[3] = {n, m, g};
+  const cuuint64_t strides[2] = {row_stride * 2, (group_stride ? group_stride : row_stride * m) * 2};
+  const cuuint32_t box[3] = {64, 32, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, base, dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
                          uint32_t box1) {
   return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, d0, d1, d2, box0, box1);

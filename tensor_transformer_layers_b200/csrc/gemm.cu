@@ -18,7 +18,11 @@
 //             while tile i+1's MMAs do;
 //   warps 2-5 epilogue: tcgen05.ld 32 columns at a time (thread = output row),
 //             bias, optional tanh-form GELU, rounding to bf16 (or fp16 for the
-//             Q/K/V that feed attention), 16-byte global stores.
+//             Q/K/V that feed attention); each warp stages its 32 rows x 64
+//             columns in shared memory (128-byte swizzle, two buffers) and
+//             writes them with one TMA store, so global writes are whole lines
+//             instead of 16 bytes from each of 32 rows per instruction; TMA
+//             clips the ragged edges.
 // Two more forms of the same kernels:
 //   SwiGLU colwise (a gate/up pair packed with blocks [1, 1], section "Fused
 //            projections"): the B tile's first 128 rows are gate rows and its
@@ -56,12 +60,17 @@ constexpr int kThreads = 192;
 constexpr int kAccCols = 256;  // fp32 TMEM columns per accumulator (N = 256)
 constexpr int kTmemCols = 2 * kAccCols;
 
+// epilogue staging: per epilogue warp two buffers of 32 rows x 128 bytes
+constexpr int kEpiBuf = 32 * 128;
+constexpr int kEpiBytes = 4 * 2 * kEpiBuf;
+
 // single-CTA kernel
 constexpr int BM1 = 128, BN1 = 256;
 constexpr int kStages1 = 4;
 constexpr int kABytes1 = BM1 * BK * 2;
 constexpr int kStageBytes1 = kABytes1 + BN1 * BK * 2;
-constexpr int kBarOff1 = kStages1 * kStageBytes1;
+constexpr int kEpiOff1 = kStages1 * kStageBytes1;
+constexpr int kBarOff1 = kEpiOff1 + kEpiBytes;
 constexpr int kSmemBytes1 = kBarOff1 + 256 + 1024;  // + barriers + 1 KB alignment slack
 constexpr uint32_t kIdesc1 = idesc_bf16_f32(BM1, BN1, false);
 
@@ -70,7 +79,8 @@ constexpr int BM2 = 256, BN2 = 256;
 constexpr int kStages2 = 6;
 constexpr int kHalfBytes = 128 * BK * 2;
 constexpr int kStageBytes2 = 2 * kHalfBytes;
-constexpr int kBarOff2 = kStages2 * kStageBytes2;
+constexpr int kEpiOff2 = kStages2 * kStageBytes2;
+constexpr int kBarOff2 = kEpiOff2 + kEpiBytes;
 constexpr int kSmemBytes2 = kBarOff2 + 512 + 1024;
 constexpr uint32_t kIdesc2 = idesc_bf16_f32(BM2, BN2, false);
 
@@ -103,120 +113,148 @@ __device__ __forceinline__ TileCoord decode_tile(int t, int m_tiles, int n_tiles
   return c;
 }
 
-// Drains one 128-row x 256-column fp32 accumulator (this warp's 32 lanes) to
-// global memory: bias, GELU, rounding, masked 16-byte stores.
-__device__ __forceinline__ void epilogue_rows(const GemmArgs& p, uint32_t taddr, int row, int g, int col_base) {
-  uint16_t* orow = p.out + int64_t(g) * p.out_gstride + int64_t(row) * p.ldo;
+// Stages 16 output bytes (8 columns) of this thread's row at 16-byte chunk k
+// (0..7) of a 32-row x 128-byte box in the 128-byte swizzle that the output
+// map's TMA store expects (chunk index XOR row index mod 8).
+__device__ __forceinline__ void stage16(uint8_t* buf, int lane, int k, uint4 v) {
+  *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) << 4)) = v;
+}
+
+// Hands a staged 32 x 64 box to the TMA unit.  `row0` is the warp's first
+// row; a box wholly below M is skipped (TMA would clip it anyway).
+__device__ __forceinline__ void store_box(const CUtensorMap* omap, uint8_t* buf, int lane, int col0, int row0, int g,
+                                          int M) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && row0 < M) {
+    tma_store_3d(omap, buf, col0, row0, g);
+    bulk_commit();
+  }
+}
+
+// Waits until the staging buffer about to be reused is no longer read by an
+// earlier TMA store of this warp (two buffers, so one store may stay in flight).
+__device__ __forceinline__ uint8_t* next_buf(uint8_t* stage, uint32_t& nbox, int lane) {
+  uint8_t* buf = stage + (nbox & 1u) * kEpiBuf;
+  ++nbox;
+  if (lane == 0) bulk_wait_read_1();
+  __syncwarp();
+  return buf;
+}
+
+// Drains `width` columns of a 128-row fp32 accumulator (this warp's 32 lanes,
+// TMEM columns from taddr, output columns from col_base, rows from row0) in
+// 64-column boxes: bias, GELU, rounding, staging, TMA store.
+__device__ __forceinline__ void epilogue_rows(const GemmArgs& p, const CUtensorMap* omap, uint32_t taddr, int row0,
+                                              int lane, int g, int col_base, int width, uint8_t* stage,
+                                              uint32_t& nbox) {
   const uint16_t* bias = p.bias ? p.bias + int64_t(g) * p.bias_gstride : nullptr;
   const int n_left = p.N - col_base;
-  const int chunks = n_left >= kAccCols ? kAccCols / 32 : (n_left + 31) / 32;  // warp-uniform
-  for (int c = 0; c < chunks; ++c) {
-    uint32_t r[32];
-    __syncwarp();
-    tmem_ld32_sync(taddr + uint32_t(c * 32), r);
-    const int col0 = col_base + c * 32;
-    float v[32];
+  const int boxes = n_left >= width ? width / 64 : (n_left > 0 ? (n_left + 63) / 64 : 0);  // warp-uniform
+  for (int b = 0; b < boxes; ++b) {
+    uint8_t* buf = next_buf(stage, nbox, lane);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-    if (bias != nullptr) {
-      const uint4* bp = reinterpret_cast<const uint4*>(bias + col0);
+    for (int h = 0; h < 2; ++h) {
+      uint32_t r[32];
+      __syncwarp();
+      tmem_ld32_sync(taddr + uint32_t(b * 64 + h * 32), r);
+      const int col0 = col_base + b * 64 + h * 32;
+      float v[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (col0 + 8 * j < p.N) {
-          const uint4 b = __ldg(bp + j);
-          v[8 * j + 0] += bf16_lo(b.x);
-          v[8 * j + 1] += bf16_hi(b.x);
-          v[8 * j + 2] += bf16_lo(b.y);
-          v[8 * j + 3] += bf16_hi(b.y);
-          v[8 * j + 4] += bf16_lo(b.z);
-          v[8 * j + 5] += bf16_hi(b.z);
-          v[8 * j + 6] += bf16_lo(b.w);
-          v[8 * j + 7] += bf16_hi(b.w);
+      for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+      if (bias != nullptr) {
+        const uint4* bp = reinterpret_cast<const uint4*>(bias + col0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (col0 + 8 * j < p.N) {
+            const uint4 bb = __ldg(bp + j);
+            v[8 * j + 0] += bf16_lo(bb.x);
+            v[8 * j + 1] += bf16_hi(bb.x);
+            v[8 * j + 2] += bf16_lo(bb.y);
+            v[8 * j + 3] += bf16_hi(bb.y);
+            v[8 * j + 4] += bf16_lo(bb.z);
+            v[8 * j + 5] += bf16_hi(bb.z);
+            v[8 * j + 6] += bf16_lo(bb.w);
+            v[8 * j + 7] += bf16_hi(bb.w);
+          }
         }
       }
-    }
-    if (p.gelu) {
+      if (p.gelu) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
-    }
-    uint4 o[4];
-    if (p.out_f16) {
+        for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        o[j].x = pack_f16x2(v[8 * j + 0], v[8 * j + 1]);
-        o[j].y = pack_f16x2(v[8 * j + 2], v[8 * j + 3]);
-        o[j].z = pack_f16x2(v[8 * j + 4], v[8 * j + 5]);
-        o[j].w = pack_f16x2(v[8 * j + 6], v[8 * j + 7]);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        o[j].x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-        o[j].y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-        o[j].z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-        o[j].w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+        uint4 o;
+        if (p.out_f16) {
+          o.x = pack_f16x2(v[8 * j + 0], v[8 * j + 1]);
+          o.y = pack_f16x2(v[8 * j + 2], v[8 * j + 3]);
+          o.z = pack_f16x2(v[8 * j + 4], v[8 * j + 5]);
+          o.w = pack_f16x2(v[8 * j + 6], v[8 * j + 7]);
+        } else {
+          o.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+          o.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+          o.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+          o.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+        }
+        stage16(buf, lane, h * 4 + j, o);
       }
     }
-    if (row < p.M) {
-      uint4* op = reinterpret_cast<uint4*>(orow + col0);
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (col0 + 8 * j < p.N) op[j] = o[j];
-    }
+    store_box(omap, buf, lane, col_base + b * 64, row0, g, p.M);
   }
 }
 
 // SwiGLU drain of one accumulator: columns [0, 128) hold gate, [128, 256) the
-// matching up.  Output columns col_base + j, j < 128, masked by p.N; gate bias
-// at bias[col], up bias at bias[up_off + col].
-__device__ __forceinline__ void epilogue_swiglu(const GemmArgs& p, uint32_t taddr, int row, int g, int col_base) {
-  uint16_t* orow = p.out + int64_t(g) * p.out_gstride + int64_t(row) * p.ldo;
+// matching up.  Output columns col_base + j, j < 128, in two 64-column boxes;
+// gate bias at bias[col], up bias at bias[up_off + col].
+__device__ __forceinline__ void epilogue_swiglu(const GemmArgs& p, const CUtensorMap* omap, uint32_t taddr, int row0,
+                                                int lane, int g, int col_base, uint8_t* stage, uint32_t& nbox) {
   const uint16_t* bias = p.bias ? p.bias + int64_t(g) * p.bias_gstride : nullptr;
   const int n_left = p.N - col_base;
-  const int chunks = n_left >= 128 ? 8 : (n_left + 15) / 16;  // warp-uniform
-  for (int c = 0; c < chunks; ++c) {
-    uint32_t rg[16], ru[16];
-    __syncwarp();
-    tmem_ld16x2_sync(taddr + uint32_t(c * 16), rg, taddr + uint32_t(128 + c * 16), ru);
-    const int col0 = col_base + c * 16;
-    float gv[16], uv[16];
+  const int boxes = n_left >= 128 ? 2 : (n_left > 0 ? (n_left + 63) / 64 : 0);  // warp-uniform
+  for (int b = 0; b < boxes; ++b) {
+    uint8_t* buf = next_buf(stage, nbox, lane);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      gv[j] = __uint_as_float(rg[j]);
-      uv[j] = __uint_as_float(ru[j]);
-    }
-    if (bias != nullptr) {
+    for (int q = 0; q < 4; ++q) {
+      uint32_t rg[16], ru[16];
+      __syncwarp();
+      tmem_ld16x2_sync(taddr + uint32_t(b * 64 + q * 16), rg, taddr + uint32_t(128 + b * 64 + q * 16), ru);
+      const int col0 = col_base + b * 64 + q * 16;
+      float gv[16], uv[16];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (col0 + 8 * h < p.N) {
-          const uint4 bg = __ldg(reinterpret_cast<const uint4*>(bias + col0) + h);
-          const uint4 bu = __ldg(reinterpret_cast<const uint4*>(bias + p.up_off + col0) + h);
-          const uint32_t wg[4] = {bg.x, bg.y, bg.z, bg.w};
-          const uint32_t wu[4] = {bu.x, bu.y, bu.z, bu.w};
+      for (int j = 0; j < 16; ++j) {
+        gv[j] = __uint_as_float(rg[j]);
+        uv[j] = __uint_as_float(ru[j]);
+      }
+      if (bias != nullptr) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            gv[8 * h + 2 * j] += bf16_lo(wg[j]);
-            gv[8 * h + 2 * j + 1] += bf16_hi(wg[j]);
-            uv[8 * h + 2 * j] += bf16_lo(wu[j]);
-            uv[8 * h + 2 * j + 1] += bf16_hi(wu[j]);
+        for (int h = 0; h < 2; ++h) {
+          if (col0 + 8 * h < p.N) {
+            const uint4 bg = __ldg(reinterpret_cast<const uint4*>(bias + col0) + h);
+            const uint4 bu = __ldg(reinterpret_cast<const uint4*>(bias + p.up_off + col0) + h);
+            const uint32_t wg[4] = {bg.x, bg.y, bg.z, bg.w};
+            const uint32_t wu[4] = {bu.x, bu.y, bu.z, bu.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              gv[8 * h + 2 * j] += bf16_lo(wg[j]);
+              gv[8 * h + 2 * j + 1] += bf16_hi(wg[j]);
+              uv[8 * h + 2 * j] += bf16_lo(wu[j]);
+              uv[8 * h + 2 * j + 1] += bf16_hi(wu[j]);
+            }
           }
         }
       }
-    }
-    uint4 o[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      o[h].x = pack_bf16x2(silu(gv[8 * h + 0]) * uv[8 * h + 0], silu(gv[8 * h + 1]) * uv[8 * h + 1]);
-      o[h].y = pack_bf16x2(silu(gv[8 * h + 2]) * uv[8 * h + 2], silu(gv[8 * h + 3]) * uv[8 * h + 3]);
-      o[h].z = pack_bf16x2(silu(gv[8 * h + 4]) * uv[8 * h + 4], silu(gv[8 * h + 5]) * uv[8 * h + 5]);
-      o[h].w = pack_bf16x2(silu(gv[8 * h + 6]) * uv[8 * h + 6], silu(gv[8 * h + 7]) * uv[8 * h + 7]);
+      for (int h = 0; h < 2; ++h) {
+        uint4 o;
+        o.x = pack_bf16x2(silu(gv[8 * h + 0]) * uv[8 * h + 0], silu(gv[8 * h + 1]) * uv[8 * h + 1]);
+        o.y = pack_bf16x2(silu(gv[8 * h + 2]) * uv[8 * h + 2], silu(gv[8 * h + 3]) * uv[8 * h + 3]);
+        o.z = pack_bf16x2(silu(gv[8 * h + 4]) * uv[8 * h + 4], silu(gv[8 * h + 5]) * uv[8 * h + 5]);
+        o.w = pack_bf16x2(silu(gv[8 * h + 6]) * uv[8 * h + 6], silu(gv[8 * h + 7]) * uv[8 * h + 7]);
+        stage16(buf, lane, q * 2 + h, o);
+      }
     }
-    if (row < p.M) {
-      uint4* op = reinterpret_cast<uint4*>(orow + col0);
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        if (col0 + 8 * h < p.N) op[h] = o[h];
-    }
+    store_box(omap, buf, lane, col_base + b * 64, row0, g, p.M);
   }
 }
 
@@ -225,7 +263,7 @@ __device__ __forceinline__ void epilogue_swiglu(const GemmArgs& p, uint32_t tadd
 // ============================================================================
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-                   const GemmArgs p) {
+                   const __grid_constant__ CUtensorMap omap, const GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff1);
@@ -260,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&amap);
     tma_prefetch_desc(&bmap);
+    tma_prefetch_desc(&omap);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, kTmemCols);
@@ -364,6 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // this warp's TMEM lane quarter
+    uint8_t* stage = smem + kEpiOff1 + (warp - 2) * 2 * kEpiBuf;
+    uint32_t nbox = 0;
     int local = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
@@ -375,15 +416,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
+      const int row0 = tc.mb * BM1 + q * 32;
       if (p.swiglu)
-        epilogue_swiglu(p, taddr, tc.mb * BM1 + q * 32 + lane, tc.g, tc.nb * out_bn);
+        epilogue_swiglu(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, stage, nbox);
       else
-        epilogue_rows(p, taddr, tc.mb * BM1 + q * 32 + lane, tc.g, tc.nb * out_bn);
+        epilogue_rows(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, out_bn, stage, nbox);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
     if (!ok && lane == 0) report_timeout(p.err, abort_flag);
+    if (lane == 0) bulk_wait_all();  // this warp's TMA stores are complete before the CTA exits
   }
 
   tc_fence_before();
@@ -400,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================================
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-                     const GemmArgs p) {
+                     const __grid_constant__ CUtensorMap omap, const GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff2);  // the leader's copy is the one used
@@ -440,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&amap);
     tma_prefetch_desc(&bmap);
+    tma_prefetch_desc(&omap);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, kTmemCols);
@@ -547,6 +591,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
     const uint32_t tempty_leader = mapa_shared(smem_u32(&tempty[0]), 0);
+    uint8_t* stage = smem + kEpiOff2 + (warp - 2) * 2 * kEpiBuf;
+    uint32_t nbox = 0;
     int local = 0;
     bool ok = true;
     for (int t = pair; t < tiles; t += n_pairs, ++local) {
@@ -558,16 +604,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
-      const int row = tc.mb * BM2 + int(rank) * 128 + q * 32 + lane;
+      const int row0 = tc.mb * BM2 + int(rank) * 128 + q * 32;
       if (p.swiglu)
-        epilogue_swiglu(p, taddr, row, tc.g, tc.nb * out_bn);
+        epilogue_swiglu(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, stage, nbox);
       else
-        epilogue_rows(p, taddr, row, tc.g, tc.nb * out_bn);
+        epilogue_rows(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, out_bn, stage, nbox);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader + uint32_t(acc * sizeof(uint64_t)));
     }
     if (!ok && lane == 0) report_timeout(p.err, abort_flag);
+    if (lane == 0) bulk_wait_all();  // this warp's TMA stores are complete before the CTA exits
   }
 
   // Exit handshake: neither CTA leaves while the other may still signal its
@@ -625,7 +672,10 @@ CUresult make_a_map(CUtensorMap* map, const GemmOperand& A, const GemmArgs& a, u
 cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms,
                         cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.groups <= 0) return cudaSuccess;
-  CUtensorMap amap, bmap;
+  CUtensorMap amap, bmap, omap;
+  if (make_map_out_u16(&omap, a.out, uint64_t(a.N), uint64_t(a.M), uint64_t(a.groups), uint64_t(a.ldo),
+                       uint64_t(a.out_gstride)) != CUDA_SUCCESS)
+    return note_cuda_error("gemm: output tensor map encode", cudaErrorInvalidValue);
   if (a.M >= BM2) {
     // CTA-pair kernel: each CTA loads 128-row halves of both operands.
     if (make_a_map(&amap, A, a, 128) != CUDA_SUCCESS ||
@@ -649,7 +699,7 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, amap, bmap, a);
+    e = cudaLaunchKernelEx(&cfg, gemm_pair_kernel, amap, bmap, omap, a);
     count_launch();
     if (e == cudaSuccess) e = cudaGetLastError();
     return note_cuda_error("gemm (CTA pairs): launch", e);
@@ -663,7 +713,7 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
   const int grid = int(tiles < num_sms ? tiles : num_sms);
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes1);
   if (e != cudaSuccess) return note_cuda_error("gemm: set shared memory size", e);
-  gemm_tc_kernel<<<grid, kThreads, kSmemBytes1, s>>>(amap, bmap, a);
+  gemm_tc_kernel<<<grid, kThreads, kSmemBytes1, s>>>(amap, bmap, omap, a);
   count_launch();
   return note_cuda_error("gemm: launch", cudaGetLastError());
 }

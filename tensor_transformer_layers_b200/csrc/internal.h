@@ -111,6 +111,10 @@ CUresult make_map_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint6
                           uint32_t box0, uint32_t box1, uint64_t d1_stride = 0);
 CUresult make_map_3d_bf16_box(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
                               uint32_t box0, uint32_t box1, uint32_t box2);
+// Output map of the GEMM epilogue's TMA stores: 16-bit {n, m, g} with the
+// given row and group strides (elements), box 64 x 32, 128-byte swizzle.
+CUresult make_map_out_u16(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t g, uint64_t row_stride,
+                          uint64_t group_stride);
 CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
                          uint32_t box1);
 
