@@ -188,3 +188,19 @@ def test_joint_attn_checks():
     st, h = tp.tp_joint_attn_prepare(A, A, A, A, 768, 6, 4, stream=0)
     assert st == S["TP_ERR_HEADS_INDIVISIBLE"] and not h
     assert tp.tp_joint_attn_run(None, A, 64, A, 32, A, A, A, ws, stream=0) == S["TP_ERR_BAD_HANDLE"]
+
+
+def test_header_is_plain_c(tmp_path):
+    # The ABI header must compile as C99 on its own (no C++ constructs outside
+    # the extern "C" guard) and as C++.
+    import shutil
+    import subprocess
+    src = tmp_path / "use.c"
+    src.write_text('#include "tp.h"\nint main(void) { return tp_abi_version() == TP_ABI_VERSION ? 0 : 1; }\n')
+    for cc, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not available")
+        r = subprocess.run([cc, std, "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-x",
+                            "c" if cc == "gcc" else "c++", "-I", os.path.join(ROOT, "include"), str(src)],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
