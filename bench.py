@@ -3,12 +3,12 @@
 
 One step = one pass of the whole layer-pair path over one batch of synthetic
 tokens, with all tp_degree shards on one GPU: slice every shard of W_up,
-b_up and W_down (a1), the colwise FFN-in GEMM with bias + GELU for every shard
-(a2, a3), and the rowwise FFN-out GEMM whose accumulator sums every shard's
-partial plus the bias once (a4).  These are the five C-ABI calls that the
-one-shot ``tp_mlp_pair`` makes, issued one by one so that each kernel's
-duration is measured with CUDA events inside the timed region (a GPU test
-checks that the sequence is bit-identical to ``tp_mlp_pair``).
+b_up and W_down in one launch (a1), the colwise FFN-in GEMM with bias + GELU
+for every shard (a2, a3), and the rowwise FFN-out GEMM whose accumulator sums
+every shard's partial plus the bias once (a4).  These are the three C-ABI
+calls that the one-shot ``tp_mlp_pair`` makes, issued one by one so that each
+kernel's duration is measured with CUDA events inside the timed region (a GPU
+test checks that the sequence is bit-identical to ``tp_mlp_pair``).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                        [--workload flux_mlp|flux_attn|wide_block|flux_reduce|flux_swiglu|
@@ -238,14 +238,11 @@ class MlpWorkload:
              "Y": torch.empty((M, D), dtype=torch.int16, device=dev)}
         ck = tp._check
         self.bufs = b
+        jobs = [(g["W_up"], F, D, tp.TP_COLWISE, b["w_up"]), (g["W_down"], D, F, tp.TP_ROWWISE, b["w_down"]),
+                (g["b_up"], T, Fs, tp.TP_COLWISE, b["b_up"])]
         return [
-            Kernel("slice_w_up", "GB/s", 2.0 * F * D * 2,
-                   lambda: ck(tp.tp_shard_weight_all(g["W_up"], F, D, tp.TP_COLWISE, T, b["w_up"]), "slice W_up")),
-            Kernel("slice_b_up", "GB/s", 2.0 * F * 2,
-                   lambda: ck(tp.tp_shard_weight_all(g["b_up"], T, Fs, tp.TP_COLWISE, T, b["b_up"]), "slice b_up")),
-            Kernel("slice_w_down", "GB/s", 2.0 * D * F * 2,
-                   lambda: ck(tp.tp_shard_weight_all(g["W_down"], D, F, tp.TP_ROWWISE, T, b["w_down"]),
-                              "slice W_down")),
+            Kernel("slice_weights", "GB/s", 2.0 * (F * D + D * F + F) * 2,
+                   lambda: ck(tp.tp_shard_weights_batch(jobs, T), "slice W_up, W_down, b_up")),
             Kernel("colwise_gemm", "TFLOP/s", 2.0 * M * D * F,
                    lambda: ck(tp.tp_colwise_linear(g["X"], M, D, b["w_up"], b["b_up"], Fs, T, 1, tp.TP_OUT_BF16,
                                                    b["H"]), "colwise")),
@@ -617,7 +614,8 @@ class ReduceWorkload(MlpWorkload):
 
 class SwigluWorkload(MlpWorkload):
     """flux_swiglu: the SwiGLU pair with gate and up packed (blocks [1, 1]):
-    packed colwise slicing, the SwiGLU colwise GEMM, the rowwise GEMM."""
+    packed colwise slicing of W_in and b_in with W_out's rowwise slicing in
+    one launch, the SwiGLU colwise GEMM, the rowwise GEMM."""
     key = "flux_swiglu"
     metric = "TP SwiGLU MLP-pair bf16 TFLOP/s on 1 B200"
 
@@ -648,16 +646,12 @@ class SwigluWorkload(MlpWorkload):
              "Y": torch.empty((M, D), dtype=torch.int16, device=dev)}
         ck = tp._check
         self.bufs = b
+        jobs = [(g["W_in"], 2 * F, D, tp.TP_COLWISE, b["w_in"], [1, 1]),
+                (g["W_out"], D, F, tp.TP_ROWWISE, b["w_out"]),
+                (g["b_in"], 1, 2 * F, tp.TP_ROWWISE, b["b_in"], [1, 1])]
         return [
-            Kernel("slice_w_in", "GB/s", 2.0 * 2 * F * D * 2,
-                   lambda: ck(tp.tp_shard_packed_all(g["W_in"], 2 * F, D, tp.TP_COLWISE, [1, 1], T, b["w_in"]),
-                              "slice W_in")),
-            Kernel("slice_b_in", "GB/s", 2.0 * 2 * F * 2,
-                   lambda: ck(tp.tp_shard_packed_all(g["b_in"], 1, 2 * F, tp.TP_ROWWISE, [1, 1], T, b["b_in"]),
-                              "slice b_in")),
-            Kernel("slice_w_out", "GB/s", 2.0 * D * F * 2,
-                   lambda: ck(tp.tp_shard_weight_all(g["W_out"], D, F, tp.TP_ROWWISE, T, b["w_out"]),
-                              "slice W_out")),
+            Kernel("slice_weights", "GB/s", 2.0 * (2 * F * D + D * F + 2 * F) * 2,
+                   lambda: ck(tp.tp_shard_weights_batch(jobs, T), "slice W_in (packed), W_out, b_in (packed)")),
             Kernel("colwise_swiglu", "TFLOP/s", 2.0 * M * D * 2 * F,
                    lambda: ck(tp.tp_colwise_swiglu(g["X"], M, D, b["w_in"], b["b_in"], Fs, T, b["H"]),
                               "colwise swiglu")),

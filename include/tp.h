@@ -137,6 +137,25 @@ tp_status tp_shard_weight(const uint16_t* W, int64_t rows, int64_t cols, int sty
 tp_status tp_shard_weight_all(const uint16_t* W, int64_t rows, int64_t cols, int style,
                               int tp_degree, uint16_t* out, void* stream);
 
+/* Several all-shard slicing jobs in one launch (e.g. W_up, b_up and W_down of
+ * an MLP pair).  jobs[] is HOST memory, 1 <= njobs <= 8 (else BAD_SHAPE).  A
+ * job with blocks == NULL is a tp_shard_weight_all job; with blocks != NULL
+ * it is a tp_shard_packed_all job (blocks[] in host memory, nblocks of them).
+ * Every job is checked as the corresponding single call before anything is
+ * launched.  Each job's output is all T shards stacked in rank order.  A
+ * colwise layer's bias of n elements is the job {b, T, n/T, TP_COLWISE} (or
+ * {b, 1, n, TP_ROWWISE}: the same slices).  One launch for up to 8 plain jobs
+ * or packed blocks in all, one more per further 8. */
+typedef struct {
+  const uint16_t* W;     /* device, [rows x cols] */
+  int64_t rows, cols;
+  int style;             /* TP_COLWISE, TP_ROWWISE (or TP_ROWWISE_SPLIT_INPUT when plain) */
+  uint16_t* out;         /* device, as tp_shard_weight_all's / tp_shard_packed_all's out */
+  const int64_t* blocks; /* NULL, or the packed blocks (host) */
+  int nblocks;
+} tp_shard_job;
+tp_status tp_shard_weights_batch(const tp_shard_job* jobs, int njobs, int tp_degree, void* stream);
+
 /* out[n/T] = b[rank*n/T : (rank+1)*n/T] (a colwise layer's bias).  n/T must be
  * a multiple of 8. */
 tp_status tp_shard_bias(const uint16_t* b, int64_t n, int tp_degree, int rank,

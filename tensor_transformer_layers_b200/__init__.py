@@ -81,6 +81,7 @@ SIGNATURES = {
     "tp_joint_attn_run_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "tp_joint_attn_run": (_I, [_P, _P, _I64, _P, _I64, _P, _P, _P, _SZ, _P]),
     "tp_colwise_linear_rows": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _I, _P, _I64, _P]),
+    "tp_shard_weights_batch": (_I, [_P, _I, _I, _P]),
     "tp_rowwise_linear_sum_rows": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
 }
 
@@ -253,6 +254,28 @@ def tp_mlp_pair_sharded_noalloc(X, M, D, F, W_up_shards, b_up_shards, W_down_sha
     return lib().tp_mlp_pair_sharded_noalloc(_ptr(X), M, D, F, _ptr(W_up_shards), _ptr(b_up_shards),
                                              _ptr(W_down_shards), _ptr(b_down), tp_degree, _ptr(Y),
                                              _stream(stream))
+
+
+class tp_shard_job(ctypes.Structure):
+    """Mirrors tp_shard_job in include/tp.h."""
+    _fields_ = [("W", _P), ("rows", _I64), ("cols", _I64), ("style", _I), ("out", _P),
+                ("blocks", ctypes.POINTER(_I64)), ("nblocks", _I)]
+
+
+def tp_shard_weights_batch(jobs, tp_degree, stream=None) -> int:
+    """jobs: list of (W, rows, cols, style, out) or (W, rows, cols, style, out, blocks);
+    all sliced in one launch (up to 8 plain jobs or packed blocks)."""
+    keep, items = [], []
+    for job in jobs:
+        W, r, c, s, o = job[:5]
+        blocks = job[5] if len(job) > 5 else None
+        arr, n = _blocks(blocks)
+        keep.append(arr)
+        items.append(tp_shard_job(_ptr(W), r, c, s, _ptr(o), ctypes.cast(arr, ctypes.POINTER(_I64)) if arr else None,
+                                  n))
+    table = (tp_shard_job * max(len(items), 1))(*items)
+    return lib().tp_shard_weights_batch(ctypes.cast(table, _P) if items else None, len(items), tp_degree,
+                                        _stream(stream))
 
 
 def _blocks(blocks):

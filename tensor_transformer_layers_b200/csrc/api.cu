@@ -274,32 +274,44 @@ tp_status slice_all_qkv(const uint16_t* Wqkv, int64_t D, int T, uint16_t* out, c
              : TP_ERR_CUDA;
 }
 
-// Packed slicing ("Fused projections").  sizes[] are absolute block sizes
-// along the packed dimension (validated).  rank < 0: all shards, stacked.
-tp_status slice_packed(const uint16_t* W, int64_t rows, int64_t cols, int style, const int64_t* sizes, int nb,
-                       int T, int rank, uint16_t* out, cudaStream_t s) {
+// Packed slicing ("Fused projections") as blocked copies: one SliceJob per
+// packed block, covering every shard (rank < 0) or one shard.  sizes[] are
+// absolute block sizes along the packed dimension (validated).  Returns the
+// number of jobs written to `out_jobs`.
+int packed_jobs(const uint16_t* W, int64_t rows, int64_t cols, int style, const int64_t* sizes, int nb, int T,
+                int rank, uint16_t* out, SliceJob* out_jobs) {
   const int64_t P = style == TP_COLWISE ? rows : cols;
   const int64_t Ps = P / T;  // shard extent along the packed dimension
   int64_t start = 0, off = 0;
   for (int b = 0; b < nb; ++b) {
     const int64_t q = sizes[b] / T;  // this block's share per shard
-    cudaError_t e;
-    if (style == TP_COLWISE) {
-      if (rank >= 0)
-        e = launch_slice_copy(W + (start + rank * q) * cols, out + off * cols, 1, q, cols, cols, 0, 0, s);
-      else
-        e = launch_slice_copy(W + start * cols, out + off * cols, T, q, cols, cols, q * cols, Ps * cols, s);
-    } else {
-      if (rank >= 0)
-        e = launch_slice_copy(W + start + rank * q, out + off, 1, rows, q, cols, 0, 0, s, 1, 0, 0, Ps);
-      else
-        e = launch_slice_copy(W + start, out + off, T, rows, q, cols, q, rows * Ps, s, 1, 0, 0, Ps);
-    }
-    if (e != cudaSuccess) return TP_ERR_CUDA;
+    const int64_t r0 = rank < 0 ? 0 : rank;
+    const int64_t nblk = rank < 0 ? T : 1;
+    if (style == TP_COLWISE)
+      out_jobs[b] = SliceJob{W + (start + r0 * q) * cols, out + off * cols, nblk, q, cols, cols, cols, q * cols,
+                             Ps * cols};
+    else
+      out_jobs[b] = SliceJob{W + start + r0 * q, out + off, nblk, rows, q, cols, Ps, q, rows * Ps};
     start += sizes[b];
     off += q;
   }
+  return nb;
+}
+
+// Launches jobs in groups of kMaxSliceJobs.
+tp_status run_slice_jobs(const SliceJob* jobs, int n, cudaStream_t s) {
+  for (int i = 0; i < n; i += kMaxSliceJobs) {
+    const int k = n - i < kMaxSliceJobs ? n - i : kMaxSliceJobs;
+    if (launch_slice_jobs(jobs + i, k, s) != cudaSuccess) return TP_ERR_CUDA;
+  }
   return TP_OK;
+}
+
+tp_status slice_packed(const uint16_t* W, int64_t rows, int64_t cols, int style, const int64_t* sizes, int nb,
+                       int T, int rank, uint16_t* out, cudaStream_t s) {
+  SliceJob jobs[kMaxPackedBlocks];
+  const int n = packed_jobs(W, rows, cols, style, sizes, nb, T, rank, out, jobs);
+  return run_slice_jobs(jobs, n, s);
 }
 
 // Validates a packed call and turns proportional blocks into absolute sizes.
@@ -594,6 +606,41 @@ tp_status tp_shard_weight_all(const uint16_t* W, int64_t rows, int64_t cols, int
                              : slice_all_rowwise(W, rows, cols, tp_degree, out, as_stream(stream));
 }
 
+tp_status tp_shard_weights_batch(const tp_shard_job* jobs, int njobs, int tp_degree, void* stream) {
+  if (!jobs) return TP_ERR_NULL;
+  if (njobs < 1 || njobs > kMaxSliceJobs) return TP_ERR_BAD_SHAPE;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  SliceJob sj[kMaxSliceJobs * kMaxPackedBlocks];
+  int n = 0;
+  for (int j = 0; j < njobs; ++j) {
+    const tp_shard_job& b = jobs[j];
+    if (b.blocks) {  // packed job
+      int64_t sizes[kMaxPackedBlocks];
+      const tp_status st = check_packed(b.W, b.rows, b.cols, b.style, b.blocks, b.nblocks, tp_degree, b.out, sizes);
+      if (st != TP_OK) return st;
+      n += packed_jobs(b.W, b.rows, b.cols, b.style, sizes, b.nblocks, tp_degree, -1, b.out, sj + n);
+      continue;
+    }
+    int style = b.style == TP_ROWWISE_SPLIT_INPUT ? int(TP_ROWWISE) : b.style;
+    if (!b.W || !b.out) return TP_ERR_NULL;
+    if (style != TP_COLWISE && style != TP_ROWWISE) return TP_ERR_BAD_STYLE;
+    if (b.rows < 1 || b.cols < 1 || b.rows >= kMaxDim || b.cols >= kMaxDim) return TP_ERR_BAD_SHAPE;
+    if (style == TP_COLWISE && b.rows % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+    if (style == TP_ROWWISE && b.cols % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+    if (!al16(b.W) || !al16(b.out) || b.cols % 8 != 0) return TP_ERR_ALIGNMENT;
+    if (style == TP_ROWWISE && (b.cols / tp_degree) % 8 != 0) return TP_ERR_ALIGNMENT;
+    if (style == TP_COLWISE) {  // all colwise shards stacked = the weight's own bytes
+      sj[n++] = SliceJob{b.W, b.out, 1, b.rows, b.cols, b.cols, b.cols, 0, 0};
+    } else {  // block r = columns [r*cs, (r+1)*cs) of every row
+      const int64_t cs = b.cols / tp_degree;
+      sj[n++] = SliceJob{b.W, b.out, tp_degree, b.rows, cs, b.cols, cs, cs, b.rows * cs};
+    }
+  }
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_slice_jobs(sj, n, as_stream(stream));
+}
+
 tp_status tp_shard_bias(const uint16_t* b, int64_t n, int tp_degree, int rank, uint16_t* out, void* stream) {
   if (!b || !out) return TP_ERR_NULL;
   if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
@@ -810,10 +857,13 @@ tp_status tp_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F, const 
   uint16_t* b_up_sh = b_up ? reinterpret_cast<uint16_t*>(w + L.b_up) : nullptr;
   uint16_t* w_down_sh = reinterpret_cast<uint16_t*>(w + L.w_down);
   uint16_t* H = reinterpret_cast<uint16_t*>(w + L.h);
-  // a1: materialise every shard (what each rank would hold after sharded loading).
-  if ((st = slice_all_colwise(W_up, F, D, w_up_sh, s)) != TP_OK) return st;
-  if (b_up && (st = slice_all_colwise(b_up, 1, F, b_up_sh, s)) != TP_OK) return st;
-  if ((st = slice_all_rowwise(W_down, D, F, tp_degree, w_down_sh, s)) != TP_OK) return st;
+  // a1: materialise every shard (what each rank would hold after sharded
+  // loading), W_up, b_up and W_down in one launch.
+  const int64_t Fs = F / tp_degree;
+  SliceJob sj[3] = {{W_up, w_up_sh, 1, F, D, D, D, 0, 0},
+                    {W_down, w_down_sh, tp_degree, D, Fs, F, Fs, Fs, D * Fs},
+                    {b_up, b_up_sh, 1, 1, F, F, F, 0, 0}};  // used only when b_up is given
+  if (launch_slice_jobs(sj, b_up ? 3 : 2, s) != cudaSuccess) return TP_ERR_CUDA;
   // a2..a4
   return mlp_forward(di, X, M, D, F, tp_degree, w_up_sh, b_up_sh, w_down_sh, b_down, H, Y, s);
 }
@@ -841,11 +891,18 @@ tp_status tp_swiglu_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F,
   uint16_t* w_in_sh = reinterpret_cast<uint16_t*>(w + L.w_up);
   uint16_t* b_in_sh = b_in ? reinterpret_cast<uint16_t*>(w + L.b_up) : nullptr;
   uint16_t* w_out_sh = reinterpret_cast<uint16_t*>(w + L.w_down);
-  const int64_t halves[2] = {F, F};  // [gate; up], packed colwise with blocks [1, 1]
-  if ((st = slice_packed(W_in, 2 * F, D, TP_COLWISE, halves, 2, tp_degree, -1, w_in_sh, s)) != TP_OK) return st;
-  if (b_in && (st = slice_packed(b_in, 1, 2 * F, TP_ROWWISE, halves, 2, tp_degree, -1, b_in_sh, s)) != TP_OK)
-    return st;
-  if ((st = slice_all_rowwise(W_out, D, F, tp_degree, w_out_sh, s)) != TP_OK) return st;
+  // [gate; up] packed colwise with blocks [1, 1]: shard r = [gate_r; up_r]
+  // (block b of shard r at rows b*Fs of the shard); its bias likewise; W_out
+  // rowwise.  One launch.
+  const int64_t Fs = F / tp_degree;
+  SliceJob sj[5] = {{W_in, w_in_sh, tp_degree, Fs, D, D, D, Fs * D, 2 * Fs * D},
+                    {W_in + F * D, w_in_sh + Fs * D, tp_degree, Fs, D, D, D, Fs * D, 2 * Fs * D},
+                    {W_out, w_out_sh, tp_degree, D, Fs, F, Fs, Fs, D * Fs}};
+  if (b_in) {
+    sj[3] = SliceJob{b_in, b_in_sh, tp_degree, 1, Fs, Fs, Fs, Fs, 2 * Fs};
+    sj[4] = SliceJob{b_in + F, b_in_sh + Fs, tp_degree, 1, Fs, Fs, Fs, Fs, 2 * Fs};
+  }
+  if (launch_slice_jobs(sj, b_in ? 5 : 3, s) != cudaSuccess) return TP_ERR_CUDA;
   return mlp_forward(di, X, M, D, F, tp_degree, w_in_sh, b_in_sh, w_out_sh, b_out,
                      reinterpret_cast<uint16_t*>(w + L.h), Y, s, true);
 }

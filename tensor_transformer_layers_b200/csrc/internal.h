@@ -22,6 +22,17 @@ cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblock
                               int64_t nblocks2 = 1, int64_t src_bstride2 = 0, int64_t dst_bstride2 = 0,
                               int64_t dst_ld = -1);
 
+// Up to kMaxSliceJobs blocked 2-D copies (same meaning as above, one block
+// index) in one launch.  Element units; cols, the lds, the strides and both
+// pointers multiples of 8 elements / 16 bytes.
+constexpr int kMaxSliceJobs = 8;
+struct SliceJob {
+  const uint16_t* src;
+  uint16_t* dst;
+  int64_t nblocks, rows, cols, src_ld, dst_ld, src_bstride, dst_bstride;
+};
+cudaError_t launch_slice_jobs(const SliceJob* jobs, int njobs, cudaStream_t s);
+
 // ----------------------------------------------------------------------------
 // a8: Y[M x N] = bf16(sum_r parts[r] + bias)
 // ----------------------------------------------------------------------------

@@ -46,7 +46,114 @@ __global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __res
   }
 }
 
+// Several blocked 2-D copies in one launch.  Job j owns CTAs
+// [cta0[j], cta0[j+1]) and walks its flattened (block, row, chunk) index
+// space with them; a job that is one contiguous span per block has rows = 1
+// and a single block needs no division (the branches are uniform per CTA).
+struct SliceJobs {
+  const uint4* src[kMaxSliceJobs];
+  uint4* dst[kMaxSliceJobs];
+  uint32_t nblocks[kMaxSliceJobs], rows[kMaxSliceJobs], c8[kMaxSliceJobs];
+  int64_t src_ld8[kMaxSliceJobs], dst_ld8[kMaxSliceJobs], src_b8[kMaxSliceJobs], dst_b8[kMaxSliceJobs];
+  int cta0[kMaxSliceJobs + 1];
+  int njobs;
+};
+
+__global__ void __launch_bounds__(kThreads) slice_jobs_kernel(const __grid_constant__ SliceJobs J) {
+  int j = 0;
+  while (j + 1 < J.njobs && int(blockIdx.x) >= J.cta0[j + 1]) ++j;
+  const uint32_t nb = J.nblocks[j], rows = J.rows[j], c8 = J.c8[j];
+  const uint32_t per_block = rows * c8;
+  const uint32_t total = nb * per_block;  // < 2^31 (host)
+  const uint32_t stride = uint32_t(J.cta0[j + 1] - J.cta0[j]) * kThreads;
+  const uint4* src = J.src[j];
+  uint4* dst = J.dst[j];
+  for (uint32_t base = (blockIdx.x - uint32_t(J.cta0[j])) * kThreads + threadIdx.x; base < total;
+       base += stride * kUnroll) {
+    uint4 v[kUnroll];
+    int64_t doff[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t i = base + u * stride;
+      if (i < total) {
+        uint32_t b = 0, rem = i;
+        if (nb > 1) {
+          b = i / per_block;
+          rem = i - b * per_block;
+        }
+        uint32_t r = 0, c = rem;
+        if (rows > 1) {
+          r = rem / c8;
+          c = rem - r * c8;
+        }
+        v[u] = __ldcs(src + int64_t(b) * J.src_b8[j] + int64_t(r) * J.src_ld8[j] + c);
+        doff[u] = int64_t(b) * J.dst_b8[j] + int64_t(r) * J.dst_ld8[j] + c;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t i = base + u * stride;
+      if (i < total) __stcs(dst + doff[u], v[u]);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_slice_jobs(const SliceJob* jobs, int njobs, cudaStream_t st) {
+  if (njobs <= 0) return cudaSuccess;
+  if (njobs > kMaxSliceJobs) return note_cuda_error("slice jobs: too many jobs", cudaErrorInvalidValue);
+  SliceJobs J{};
+  int64_t chunks[kMaxSliceJobs], all = 0;
+  bool fits = true;
+  for (int j = 0; j < njobs; ++j) {
+    SliceJob s = jobs[j];
+    if (s.src_ld == s.cols && s.dst_ld == s.cols) {  // contiguous per block: one long row
+      s.cols *= s.rows;
+      s.rows = 1;
+      s.src_ld = s.dst_ld = s.cols;
+    }
+    chunks[j] = s.nblocks * s.rows * (s.cols / 8);
+    if (chunks[j] >= (int64_t(1) << 31) - int64_t(kThreads) * kUnroll * 148 * 16) fits = false;
+    J.src[j] = reinterpret_cast<const uint4*>(s.src);
+    J.dst[j] = reinterpret_cast<uint4*>(s.dst);
+    J.nblocks[j] = uint32_t(s.nblocks);
+    J.rows[j] = uint32_t(s.rows);
+    J.c8[j] = uint32_t(s.cols / 8);
+    J.src_ld8[j] = s.src_ld / 8;
+    J.dst_ld8[j] = s.dst_ld / 8;
+    J.src_b8[j] = s.src_bstride / 8;
+    J.dst_b8[j] = s.dst_bstride / 8;
+    all += chunks[j];
+  }
+  if (!fits) {  // a job too large for 32-bit indexing: one launch per job
+    for (int j = 0; j < njobs; ++j) {
+      const SliceJob& s = jobs[j];
+      cudaError_t e = launch_slice_copy(s.src, s.dst, s.nblocks, s.rows, s.cols, s.src_ld, s.src_bstride,
+                                        s.dst_bstride, st, 1, 0, 0, s.dst_ld);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
+  if (all == 0) return cudaSuccess;
+  // CTAs in proportion to each job's bytes (at least one each), about 16 per SM in all.
+  const int64_t budget = 148 * 16;
+  int cta = 0;
+  for (int j = 0; j < njobs; ++j) {
+    J.cta0[j] = cta;
+    int64_t n = (chunks[j] * budget + all - 1) / all;
+    const int64_t need = (chunks[j] + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
+    if (n > need) n = need;
+    if (n < 1) n = 1;
+    cta += int(n);
+  }
+  J.cta0[njobs] = cta;
+  J.njobs = njobs;
+  slice_jobs_kernel<<<cta, kThreads, 0, st>>>(J);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? e : note_cuda_error("slice jobs: launch", e);
+}
 
 cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblocks, int64_t rows, int64_t cols,
                               int64_t src_ld, int64_t src_bstride, int64_t dst_bstride, cudaStream_t st,

@@ -204,3 +204,20 @@ def test_header_is_plain_c(tmp_path):
                             "c" if cc == "gcc" else "c++", "-I", os.path.join(ROOT, "include"), str(src)],
                            capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_shard_batch_checks():
+    ok = (A, 8, 8, tp.TP_COLWISE, A)
+    assert tp.tp_shard_weights_batch([], 2, stream=0) == S["TP_ERR_NULL"]
+    assert tp.tp_shard_weights_batch([ok] * 9, 2, stream=0) == S["TP_ERR_BAD_SHAPE"]
+    assert tp.tp_shard_weights_batch([ok], 0, stream=0) == S["TP_ERR_BAD_DEGREE"]
+    # a bad job anywhere in the list rejects the whole call before any launch
+    assert tp.tp_shard_weights_batch([ok, (A, 8, 8, 7, A)], 2, stream=0) == S["TP_ERR_BAD_STYLE"]
+    assert tp.tp_shard_weights_batch([ok, (A, 9, 8, tp.TP_COLWISE, A)], 2, stream=0) == S["TP_ERR_INDIVISIBLE"]
+    assert tp.tp_shard_weights_batch([ok, (A, 8, 24, tp.TP_ROWWISE, A)], 2, stream=0) == S["TP_ERR_ALIGNMENT"]
+    assert tp.tp_shard_weights_batch([ok, (0, 8, 8, tp.TP_COLWISE, A)], 2, stream=0) == S["TP_ERR_NULL"]
+    # packed jobs are checked like tp_shard_packed_all
+    assert tp.tp_shard_weights_batch([ok, (A, 36, 8, tp.TP_COLWISE, A, [1, 1, 3])], 2, stream=0) == \
+        S["TP_ERR_BAD_BLOCKS"]
+    assert tp.tp_shard_weights_batch([ok, (A, 18, 8, tp.TP_COLWISE, A, [1, 1, 1, 3, 3])], 3, stream=0) == \
+        S["TP_ERR_INDIVISIBLE"]

@@ -111,8 +111,8 @@ def test_empty_input_writes_nothing(tiny):
 
 
 def test_bench_step_sequence_matches_one_shot(flux):
-    # bench.py times the five calls that tp_mlp_pair makes, one by one; they must
-    # produce exactly the one-shot result.
+    # bench.py times the three calls that tp_mlp_pair makes (one batched slice
+    # launch, two GEMMs), one by one; they must produce exactly the one-shot result.
     c, d, _ = flux
     M, D, F, T = c["M"], c["D"], c["F"], c["T"]
     Fs = F // T
@@ -123,12 +123,12 @@ def test_bench_step_sequence_matches_one_shot(flux):
     H = torch.empty((T, M, Fs), dtype=torch.int16, device="cuda")
     Y = torch.empty((M, D), dtype=torch.int16, device="cuda")
     n0 = tp.tp_kernel_launches()
-    assert tp.tp_shard_weight_all(dd["W_up"], F, D, tp.TP_COLWISE, T, w_up) == 0
-    assert tp.tp_shard_weight_all(dd["b_up"], T, Fs, tp.TP_COLWISE, T, b_up) == 0
-    assert tp.tp_shard_weight_all(dd["W_down"], D, F, tp.TP_ROWWISE, T, w_down) == 0
+    jobs = [(dd["W_up"], F, D, tp.TP_COLWISE, w_up), (dd["W_down"], D, F, tp.TP_ROWWISE, w_down),
+            (dd["b_up"], T, Fs, tp.TP_COLWISE, b_up)]
+    assert tp.tp_shard_weights_batch(jobs, T) == 0
     assert tp.tp_colwise_linear(dd["X"], M, D, w_up, b_up, Fs, T, 1, tp.TP_OUT_BF16, H) == 0
     assert tp.tp_rowwise_linear_sum(H, M, Fs, w_down, D, dd["b_down"], T, Y) == 0
-    assert tp.tp_kernel_launches() - n0 == 5
+    assert tp.tp_kernel_launches() - n0 == 3
     torch.cuda.synchronize()
     one = _run_pair(dd, M, D, F, T)
     assert np.array_equal(from_dev(Y), one)

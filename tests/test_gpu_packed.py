@@ -85,6 +85,33 @@ def test_packed_with_one_block_is_the_plain_slice():
     assert np.array_equal(from_dev(a), from_dev(b))
 
 
+def test_shard_batch_mixed_jobs_bit_exact():
+    # plain colwise, plain rowwise, a bias, packed colwise [1,1,1,3,3] and packed
+    # rowwise [256, 768] in one call: 1 + 1 + 1 + 5 + 2 = 10 copy jobs, two launches.
+    T = 4
+    Wc = syn.normal_bf16((512, 136), 1.0, seed=1, tid=440)
+    Wr = syn.normal_bf16((72, 1024), 1.0, seed=2, tid=441)
+    b = syn.normal_bf16((2048,), 1.0, seed=3, tid=442)
+    Wpc = syn.normal_bf16((9 * 128, 64), 1.0, seed=4, tid=443)
+    Wpr = syn.normal_bf16((40, 1024), 1.0, seed=5, tid=444)
+    outs = [_empty((T, 128, 136)), _empty((T, 72, 256)), _empty((T, 512)), _empty((T, 9 * 32, 64)),
+            _empty((T, 40, 256))]
+    jobs = [(to_dev(Wc), 512, 136, tp.TP_COLWISE, outs[0]), (to_dev(Wr), 72, 1024, tp.TP_ROWWISE, outs[1]),
+            (to_dev(b), T, 512, tp.TP_COLWISE, outs[2]),
+            (to_dev(Wpc), 9 * 128, 64, tp.TP_COLWISE, outs[3], [1, 1, 1, 3, 3]),
+            (to_dev(Wpr), 40, 1024, tp.TP_ROWWISE, outs[4], [256, 768])]
+    n0 = tp.tp_kernel_launches()
+    assert tp.tp_shard_weights_batch(jobs, T) == 0
+    assert tp.tp_kernel_launches() - n0 == 2
+    torch.cuda.synchronize()
+    for r in range(T):
+        assert np.array_equal(from_dev(outs[0][r]), o.slice_colwise(Wc, T, r))
+        assert np.array_equal(from_dev(outs[1][r]), o.slice_rowwise(Wr, T, r))
+        assert np.array_equal(from_dev(outs[2][r]), o.slice_colwise(b, T, r))
+        assert np.array_equal(from_dev(outs[3][r]), o.slice_packed_colwise(Wpc, [1, 1, 1, 3, 3], T, r))
+        assert np.array_equal(from_dev(outs[4][r]), o.slice_packed_rowwise(Wpr, [256, 768], T, r))
+
+
 # --------------------------------------------------------------------------- SwiGLU colwise GEMM
 @pytest.mark.parametrize("M,K,Fs,T,bias", [
     (64, 128, 256, 2, True),     # one-CTA kernel
@@ -197,6 +224,22 @@ def test_flux_swiglu_pair(flux_swiglu):
     c, d, ref = flux_swiglu
     g = _swiglu_pair(_dev(d), c["T"])
     assert_parity(g, ref, "flux swiglu T=4")
+
+
+def test_swiglu_bench_step_matches_one_shot():
+    # bench.py times the SwiGLU pair as its three step calls (one batched slice
+    # launch, the SwiGLU colwise GEMM, the rowwise GEMM); same bits as the one-shot call.
+    import bench
+    wl = bench.SwigluWorkload(dict(kind="swiglu", M=300, D=256, F=1024, T=4, seed=11))
+    d = wl.host_inputs(0)
+    g = {k: to_dev(v) for k, v in d.items()}
+    n0 = tp.tp_kernel_launches()
+    for k in wl.kernels(tp, g, "cuda"):
+        k.fn()
+    assert tp.tp_kernel_launches() - n0 == 3
+    torch.cuda.synchronize()
+    one = _swiglu_pair(g, 4)
+    assert np.array_equal(from_dev(wl.bufs["Y"]), one)
 
 
 def test_swiglu_prepare_run_matches_one_shot(flux_swiglu):
