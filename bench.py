@@ -317,12 +317,12 @@ class AttnWorkload(MlpWorkload):
              "A": torch.empty((M, D), dtype=torch.int16, device=dev)}
         ck = tp._check
 
-        def slice_qkv():
-            ck(tp.tp_shard_qkv_heads_all(g["W_qkv"], D, H, T, b["w_qkv"]), "slice W_qkv")
+        # the head split of W_qkv is packed colwise with blocks [1, 1, 1]; with W_o: one launch
+        jobs = [(g["W_qkv"], 3 * D, D, tp.TP_COLWISE, b["w_qkv"], [1, 1, 1]),
+                (g["W_o"], D, D, tp.TP_ROWWISE, b["w_o"])]
         ks = [
-            Kernel(prefix + "slice_w_qkv", "GB/s", 2.0 * 3 * D * D * 2, slice_qkv),
-            Kernel(prefix + "slice_w_o", "GB/s", 2.0 * D * D * 2,
-                   lambda: ck(tp.tp_shard_weight_all(g["W_o"], D, D, tp.TP_ROWWISE, T, b["w_o"]), "slice W_o")),
+            Kernel(prefix + "slice_weights", "GB/s", 2.0 * 4 * D * D * 2,
+                   lambda: ck(tp.tp_shard_weights_batch(jobs, T), "slice W_qkv, W_o")),
             Kernel(prefix + "qkv_gemm", "TFLOP/s", 2.0 * M * D * 3 * D,
                    lambda: ck(tp.tp_colwise_linear(X, M, D, b["w_qkv"], None, 3 * Ds, T, 0, tp.TP_OUT_F16,
                                                    b["QKV"]), "qkv")),
@@ -374,9 +374,9 @@ class AttnWorkload(MlpWorkload):
 
 
 class JointAttnWorkload(AttnWorkload):
-    """flux_joint_attn: dual-stream joint attention (image and text streams'
-    head-split QKV, one SDPA over 4096 + 512 tokens, per-stream rowwise
-    out-projections)."""
+    """flux_joint_attn: dual-stream joint attention (both streams' weights
+    sliced in one launch, head-split QKV per stream, one SDPA over
+    4096 + 512 tokens, per-stream rowwise out-projections)."""
     key = "flux_joint_attn"
     metric = "TP dual-stream joint-attention TFLOP/s (QKV fp16, bf16 weights) on 1 B200"
 
@@ -416,15 +416,12 @@ class JointAttnWorkload(AttnWorkload):
         ck = tp._check
         qkv_txt = b["QKV"].view(T, M * 3 * Ds)[:, Mi * 3 * Ds:]  # rows [Mi, M) of every shard's block
         o_txt = b["O"].view(T, M * Ds)[:, Mi * Ds:]
+        jobs = [(g["W_qkv_img"], 3 * D, D, tp.TP_COLWISE, b["wq_img"], [1, 1, 1]),
+                (g["W_qkv_txt"], 3 * D, D, tp.TP_COLWISE, b["wq_txt"], [1, 1, 1]),
+                (g["W_o_img"], D, D, tp.TP_ROWWISE, b["wo_img"]), (g["W_o_txt"], D, D, tp.TP_ROWWISE, b["wo_txt"])]
         return [
-            Kernel("slice_w_qkv_img", "GB/s", 2.0 * 3 * D * D * 2,
-                   lambda: ck(tp.tp_shard_qkv_heads_all(g["W_qkv_img"], D, H, T, b["wq_img"]), "slice")),
-            Kernel("slice_w_qkv_txt", "GB/s", 2.0 * 3 * D * D * 2,
-                   lambda: ck(tp.tp_shard_qkv_heads_all(g["W_qkv_txt"], D, H, T, b["wq_txt"]), "slice")),
-            Kernel("slice_w_o_img", "GB/s", 2.0 * D * D * 2,
-                   lambda: ck(tp.tp_shard_weight_all(g["W_o_img"], D, D, tp.TP_ROWWISE, T, b["wo_img"]), "slice")),
-            Kernel("slice_w_o_txt", "GB/s", 2.0 * D * D * 2,
-                   lambda: ck(tp.tp_shard_weight_all(g["W_o_txt"], D, D, tp.TP_ROWWISE, T, b["wo_txt"]), "slice")),
+            Kernel("slice_weights", "GB/s", 2.0 * 8 * D * D * 2,
+                   lambda: ck(tp.tp_shard_weights_batch(jobs, T), "slice both streams' W_qkv, W_o")),
             Kernel("qkv_gemm_img", "TFLOP/s", 2.0 * Mi * D * 3 * D,
                    lambda: ck(tp.tp_colwise_linear_rows(g["X_img"], Mi, D, b["wq_img"], None, 3 * Ds, T, 0,
                                                         tp.TP_OUT_F16, b["QKV"], M), "qkv img")),

@@ -265,6 +265,23 @@ tp_status slice_all_rowwise(const uint16_t* W, int64_t rows, int64_t cols, int T
   return launch_slice_copy(W, out, T, rows, cs, cols, cs, rows * cs, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
+// Job builders for batched slicing (one launch for a layer's weights).
+// All colwise shards of W[rows x cols] stacked: the weight's own bytes.
+SliceJob job_colwise_all(const uint16_t* W, int64_t rows, int64_t cols, uint16_t* out) {
+  return SliceJob{W, out, 1, rows, cols, cols, cols, 0, 0};
+}
+// All rowwise shards: block r = columns [r*cols/T, (r+1)*cols/T) of every row.
+SliceJob job_rowwise_all(const uint16_t* W, int64_t rows, int64_t cols, int T, uint16_t* out) {
+  const int64_t cs = cols / T;
+  return SliceJob{W, out, T, rows, cs, cols, cs, cs, rows * cs};
+}
+// Head split of a fused [Q; K; V] weight (packed colwise, blocks [1, 1, 1]):
+// three jobs, block x of shard r from rows x*D + r*D/T to out rows (3r + x)*D/T.
+void jobs_qkv_all(const uint16_t* Wqkv, int64_t D, int T, uint16_t* out, SliceJob* jobs) {
+  const int64_t rs = D / T;
+  for (int x = 0; x < 3; ++x) jobs[x] = SliceJob{Wqkv + x * D * D, out + x * rs * D, T, rs, D, D, D, rs * D, 3 * rs * D};
+}
+
 tp_status slice_all_qkv(const uint16_t* Wqkv, int64_t D, int T, uint16_t* out, cudaStream_t s) {
   // shard r = [Q_r; K_r; V_r]; X_r = rows [r*D/T, (r+1)*D/T) of block X.  One
   // launch: block (r, x) copies X_r from Wqkv[x*D + r*D/T] to out[(3r + x)*D/T].
@@ -959,9 +976,12 @@ tp_status tp_mlp_prepare(const uint16_t* W_up, const uint16_t* b_up, const uint1
             cudaMalloc(&h->w_down, size_t(D) * F * 2) == cudaSuccess &&
             (!b_up || cudaMalloc(&h->b_up, size_t(F) * 2) == cudaSuccess) &&
             (!b_down || cudaMalloc(&h->b_down, size_t(D) * 2) == cudaSuccess);
-  ok = ok && slice_all_colwise(W_up, F, D, h->w_up, s) == TP_OK &&
-       slice_all_rowwise(W_down, D, F, tp_degree, h->w_down, s) == TP_OK &&
-       (!b_up || slice_all_colwise(b_up, 1, F, h->b_up, s) == TP_OK) &&
+  if (ok) {
+    SliceJob sj[3] = {job_colwise_all(W_up, F, D, h->w_up), job_rowwise_all(W_down, D, F, tp_degree, h->w_down)};
+    if (b_up) sj[2] = job_colwise_all(b_up, 1, F, h->b_up);
+    ok = run_slice_jobs(sj, b_up ? 3 : 2, s) == TP_OK;
+  }
+  ok = ok &&
        (!b_down || cudaMemcpyAsync(h->b_down, b_down, size_t(D) * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess);
   if (!ok) {
     tp_destroy(h);
@@ -1016,8 +1036,10 @@ tp_status tp_attn_block(const uint16_t* X, int64_t M, int64_t D, const uint16_t*
   uint8_t* w = static_cast<uint8_t*>(ws);
   uint16_t* wq = reinterpret_cast<uint16_t*>(w + L.w_qkv);
   uint16_t* wo = reinterpret_cast<uint16_t*>(w + L.w_o);
-  if ((st = slice_all_qkv(W_qkv, D, tp_degree, wq, s)) != TP_OK) return st;
-  if ((st = slice_all_rowwise(W_o, D, D, tp_degree, wo, s)) != TP_OK) return st;
+  SliceJob sj[4];  // W_qkv head split and W_o rowwise, one launch
+  jobs_qkv_all(W_qkv, D, tp_degree, wq, sj);
+  sj[3] = job_rowwise_all(W_o, D, D, tp_degree, wo);
+  if ((st = run_slice_jobs(sj, 4, s)) != TP_OK) return st;
   return attn_forward(di, X, M, D, heads, tp_degree, wq, wo, reinterpret_cast<uint16_t*>(w + L.qkv),
                       reinterpret_cast<uint16_t*>(w + L.o), Y, s);
 }
@@ -1039,8 +1061,12 @@ tp_status tp_attn_prepare(const uint16_t* W_qkv, const uint16_t* W_o, int64_t D,
   h->T = tp_degree;
   bool ok = cudaMalloc(&h->w_qkv, size_t(3) * D * D * 2) == cudaSuccess &&
             cudaMalloc(&h->w_o, size_t(D) * D * 2) == cudaSuccess;
-  ok = ok && slice_all_qkv(W_qkv, D, tp_degree, h->w_qkv, s) == TP_OK &&
-       slice_all_rowwise(W_o, D, D, tp_degree, h->w_o, s) == TP_OK;
+  if (ok) {
+    SliceJob sj[4];
+    jobs_qkv_all(W_qkv, D, tp_degree, h->w_qkv, sj);
+    sj[3] = job_rowwise_all(W_o, D, D, tp_degree, h->w_o);
+    ok = run_slice_jobs(sj, 4, s) == TP_OK;
+  }
   if (!ok) {
     tp_destroy(h);
     return TP_ERR_CUDA;
@@ -1098,10 +1124,12 @@ tp_status tp_joint_attn_block(const uint16_t* X_img, int64_t M_img, const uint16
   cudaStream_t s = as_stream(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
   auto at = [w](size_t off) { return reinterpret_cast<uint16_t*>(w + off); };
-  if ((st = slice_all_qkv(W_qkv_img, D, tp_degree, at(L.w_qkv_img), s)) != TP_OK) return st;
-  if ((st = slice_all_qkv(W_qkv_txt, D, tp_degree, at(L.w_qkv_txt), s)) != TP_OK) return st;
-  if ((st = slice_all_rowwise(W_o_img, D, D, tp_degree, at(L.w_o_img), s)) != TP_OK) return st;
-  if ((st = slice_all_rowwise(W_o_txt, D, D, tp_degree, at(L.w_o_txt), s)) != TP_OK) return st;
+  SliceJob sj[8];  // both streams' head splits and out-projections, one launch
+  jobs_qkv_all(W_qkv_img, D, tp_degree, at(L.w_qkv_img), sj);
+  jobs_qkv_all(W_qkv_txt, D, tp_degree, at(L.w_qkv_txt), sj + 3);
+  sj[6] = job_rowwise_all(W_o_img, D, D, tp_degree, at(L.w_o_img));
+  sj[7] = job_rowwise_all(W_o_txt, D, D, tp_degree, at(L.w_o_txt));
+  if ((st = run_slice_jobs(sj, 8, s)) != TP_OK) return st;
   return joint_attn_forward(di, X_img, M_img, X_txt, M_txt, D, heads, tp_degree, at(L.w_qkv_img), at(L.w_qkv_txt),
                             at(L.w_o_img), at(L.w_o_txt), at(L.qkv), at(L.o), Y_img, Y_txt, s);
 }
@@ -1125,10 +1153,14 @@ tp_status tp_joint_attn_prepare(const uint16_t* W_qkv_img, const uint16_t* W_qkv
   const size_t wq = size_t(3) * D * D * 2, wo = size_t(D) * D * 2;
   bool ok = cudaMalloc(&h->w_qkv_img, wq) == cudaSuccess && cudaMalloc(&h->w_qkv_txt, wq) == cudaSuccess &&
             cudaMalloc(&h->w_o_img, wo) == cudaSuccess && cudaMalloc(&h->w_o_txt, wo) == cudaSuccess;
-  ok = ok && slice_all_qkv(W_qkv_img, D, tp_degree, h->w_qkv_img, s) == TP_OK &&
-       slice_all_qkv(W_qkv_txt, D, tp_degree, h->w_qkv_txt, s) == TP_OK &&
-       slice_all_rowwise(W_o_img, D, D, tp_degree, h->w_o_img, s) == TP_OK &&
-       slice_all_rowwise(W_o_txt, D, D, tp_degree, h->w_o_txt, s) == TP_OK;
+  if (ok) {
+    SliceJob sj[8];
+    jobs_qkv_all(W_qkv_img, D, tp_degree, h->w_qkv_img, sj);
+    jobs_qkv_all(W_qkv_txt, D, tp_degree, h->w_qkv_txt, sj + 3);
+    sj[6] = job_rowwise_all(W_o_img, D, D, tp_degree, h->w_o_img);
+    sj[7] = job_rowwise_all(W_o_txt, D, D, tp_degree, h->w_o_txt);
+    ok = run_slice_jobs(sj, 8, s) == TP_OK;
+  }
   if (!ok) {
     tp_destroy(h);
     return TP_ERR_CUDA;

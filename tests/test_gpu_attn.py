@@ -71,3 +71,21 @@ def test_flux_attention_block():
     torch.cuda.synchronize()
     assert np.array_equal(from_dev(Y2), g)
     layer.close()
+
+
+def test_bench_step_sequence_matches_one_shot():
+    # bench.py times the attention block as four step calls (one batched slice
+    # launch for W_qkv's head split and W_o, the QKV GEMM, the SDPA, the
+    # out-projection); same bits as tp_attn_block.
+    import bench
+    wl = bench.AttnWorkload(dict(kind="attn", M=384, D=512, H=4, T=2, seed=12))
+    d = wl.host_inputs(0)
+    g = {k: to_dev(v) for k, v in d.items()}
+    n0 = tp.tp_kernel_launches()
+    for k in wl.kernels(tp, g, "cuda"):
+        k.fn()
+    assert tp.tp_kernel_launches() - n0 == 4
+    torch.cuda.synchronize()
+    Y = tp.attn_block(g["X"], g["W_qkv"], g["W_o"], 4, 2)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev(wl.bufs["A"]), from_dev(Y))

@@ -98,9 +98,9 @@ def test_flux_joint_sampled_rows_and_prepared(flux_joint):
 
 
 def test_bench_step_sequence_matches_one_shot():
-    # bench.py times the joint block as its nine step-level calls (four slices,
-    # two row-range QKV GEMMs, one SDPA, two row-range out-projections); they
-    # must give exactly the one-shot result.
+    # bench.py times the joint block as its six step-level calls (one batched
+    # slice launch, two row-range QKV GEMMs, one SDPA, two row-range
+    # out-projections); they must give exactly the one-shot result.
     import bench
     wl = bench.JointAttnWorkload(dict(kind="joint", M_img=300, M_txt=77, D=256, H=2, T=2, seed=9))
     d = wl.host_inputs(0)
@@ -108,7 +108,7 @@ def test_bench_step_sequence_matches_one_shot():
     n0 = tp.tp_kernel_launches()
     for k in wl.kernels(tp, g, "cuda"):
         k.fn()
-    assert tp.tp_kernel_launches() - n0 == 9
+    assert tp.tp_kernel_launches() - n0 == 6
     torch.cuda.synchronize()
     gi, gt = _run(g, 300, 77, 2, 2)
     assert np.array_equal(from_dev(wl.bufs["Y_img"]), gi) and np.array_equal(from_dev(wl.bufs["Y_txt"]), gt)
