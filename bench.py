@@ -912,33 +912,65 @@ def run_ours(args, wl, rank, local_rank, world):
                 "peak_source": f"{peak_src}: {'bf16 burst' if dom.unit == 'TFLOP/s' else 'HBM copy'} from {src}",
                 "algorithmic_work_per_launch": dom.work}
 
-    # ---- end to end: the public one-shot call with host buffers copied in and the result copied out.
+    # ---- end to end: the public one-shot call, every step's inputs copied in from pinned host
+    # memory and its result copied back, as a serving loop runs it: step i+1's inputs are staged
+    # (second device buffer, own stream) while step i computes, and the result's copy back runs on
+    # a third stream.  Every copy of every step is inside the timed region.
     y0 = wl.one_shot(tp, g, dev)
     y_host = torch.empty(y0.shape, dtype=y0.dtype).pin_memory()
-    gi = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    gis = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = y_host.numel() * y_host.element_size()
+    s_h2d, s_cmp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        for k in host:
-            gi[k].copy_(host[k], non_blocking=True)
-        y_host.copy_(wl.one_shot(tp, gi, dev), non_blocking=True)
+    def e2e_run(n, start_ev):
+        for s in (s_h2d, s_cmp, s_d2h):
+            s.wait_event(start_ev)
+        used = [None, None]  # compute done with staging buffer b
+        d2h_done = None
+        for i in range(n):
+            b = i & 1
+            if used[b] is not None:
+                s_h2d.wait_event(used[b])  # step i-2 no longer reads this staging buffer
+            with torch.cuda.stream(s_h2d):
+                for k in host:
+                    gis[b][k].copy_(host[k], non_blocking=True)
+                staged = torch.cuda.Event()
+                staged.record(s_h2d)
+            s_cmp.wait_event(staged)
+            if d2h_done is not None:
+                s_cmp.wait_event(d2h_done)  # the previous result has left the output buffer
+            with torch.cuda.stream(s_cmp):
+                y = wl.one_shot(tp, gis[b], dev)
+                used[b] = torch.cuda.Event()
+                used[b].record(s_cmp)
+            s_d2h.wait_event(used[b])
+            with torch.cuda.stream(s_d2h):
+                y_host.copy_(y, non_blocking=True)
+                d2h_done = torch.cuda.Event()
+                d2h_done.record(s_d2h)
+        cur = torch.cuda.current_stream(dev)
+        cur.wait_stream(s_h2d)
+        cur.wait_stream(s_cmp)
+        cur.wait_stream(s_d2h)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    w0 = torch.cuda.Event()
+    w0.record()
+    e2e_run(max(1, args.warmup), w0)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = args.steps
     e0.record()
-    for _ in range(n_e2e):
-        e2e_step()
+    e2e_run(n_e2e, e0)
     e1.record()
     torch.cuda.synchronize()
     e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
     barrier()
     e2e = {"value": wl.work() * world * n_e2e / e2e_s / scale, "unit": wl.unit, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "call": wl.e2e_call}
+           "d2h_bytes_per_step": d2h, "call": wl.e2e_call,
+           "pipelining": "two device staging buffers: step i+1's host-to-device copies overlap step i's compute; "
+                         "device-to-host copies on a third stream; all copies inside the timed region"}
 
     out = {
         "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
