@@ -87,10 +87,20 @@ constexpr uint32_t kIdesc2 = idesc_bf16_f32(BM2, BN2, false);
 static_assert(kTmemCols == 512, "two 256-column accumulators fill TMEM");
 static_assert(kSmemBytes1 <= 227 * 1024 && kSmemBytes2 <= 227 * 1024, "shared memory budget");
 
-__device__ __forceinline__ float gelu_tanh(float x) {
-  // 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))  (Hendrycks & Gimpel, 2016)
-  const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
-  return 0.5f * x * (1.0f + tanh_approx(u));
+// GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
+// (Hendrycks & Gimpel, 2016), on two values at once: the polynomial and the
+// final product in packed fp32 pairs (half the FMA-pipe instructions of the
+// scalar form; the epilogue's arithmetic competes with the MMA issue for the
+// sub-partitions while the next tile's MMAs run), tanh on the MUFU unit.
+__device__ __forceinline__ void gelu_tanh2(float& a, float& b) {
+  const uint64_t x = f32x2(a, b);
+  const uint64_t x2 = mul_f32x2(x, x);
+  const uint64_t inner = fma_f32x2(mul_f32x2(x2, f32x2(0.044715f, 0.044715f)), x, x);  // x + 0.044715 x^3
+  float u0, u1;
+  f32x2_split(mul_f32x2(inner, f32x2(0.7978845608028654f, 0.7978845608028654f)), u0, u1);
+  const uint64_t th = f32x2(tanh_approx(u0), tanh_approx(u1));
+  const uint64_t hx = mul_f32x2(x, f32x2(0.5f, 0.5f));
+  f32x2_split(fma_f32x2(hx, th, hx), a, b);  // 0.5 x + 0.5 x tanh(u)
 }
 
 // SiLU(x) = x * sigmoid(x) = x / (1 + 2^(-x log2 e))  (Elfwing et al., 2018).
@@ -168,20 +178,17 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& p, const CUtensorM
         for (int j = 0; j < 4; ++j) {
           if (col0 + 8 * j < p.N) {
             const uint4 bb = __ldg(bp + j);
-            v[8 * j + 0] += bf16_lo(bb.x);
-            v[8 * j + 1] += bf16_hi(bb.x);
-            v[8 * j + 2] += bf16_lo(bb.y);
-            v[8 * j + 3] += bf16_hi(bb.y);
-            v[8 * j + 4] += bf16_lo(bb.z);
-            v[8 * j + 5] += bf16_hi(bb.z);
-            v[8 * j + 6] += bf16_lo(bb.w);
-            v[8 * j + 7] += bf16_hi(bb.w);
+            const uint32_t w[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+              f32x2_split(add_f32x2(f32x2(v[8 * j + 2 * h], v[8 * j + 2 * h + 1]), f32x2(bf16_lo(w[h]), bf16_hi(w[h]))),
+                          v[8 * j + 2 * h], v[8 * j + 2 * h + 1]);
           }
         }
       }
       if (p.gelu) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+        for (int j = 0; j < 32; j += 2) gelu_tanh2(v[j], v[j + 1]);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
