@@ -221,3 +221,39 @@ def test_shard_batch_checks():
         S["TP_ERR_BAD_BLOCKS"]
     assert tp.tp_shard_weights_batch([ok, (A, 18, 8, tp.TP_COLWISE, A, [1, 1, 1, 3, 3])], 3, stream=0) == \
         S["TP_ERR_INDIVISIBLE"]
+
+
+def test_c_program_links_and_gets_errors(tmp_path):
+    # A plain C program against libtp.so: status strings and argument errors,
+    # which are decided on the host before any CUDA call.
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "tp.h"
+int main(void) {
+  uint16_t* fake = (uint16_t*)(uintptr_t)(1u << 20);
+  int64_t blocks[2] = {1, 4};  /* sum 5 does not divide 36 */
+  if (tp_abi_version() != TP_ABI_VERSION) return 1;
+  if (tp_shard_weight(NULL, 8, 8, TP_COLWISE, 2, 0, fake, NULL) != TP_ERR_NULL) return 2;
+  if (tp_shard_weight(fake, 9, 8, TP_COLWISE, 2, 0, fake, NULL) != TP_ERR_INDIVISIBLE) return 3;
+  if (tp_shard_packed_all(fake, 36, 8, TP_COLWISE, blocks, 2, 2, fake, NULL) != TP_ERR_BAD_BLOCKS) return 4;
+  if (tp_attn_block(fake, 64, 768, fake, fake, 6, 4, fake, fake, 1 << 30, NULL) != TP_ERR_HEADS_INDIVISIBLE) return 5;
+  if (tp_mlp_pair(fake, 0, 128, 512, fake, fake, fake, fake, 2, fake, NULL, 0, NULL) != TP_OK) return 6;
+  if (strcmp(tp_status_string(TP_ERR_NULL), "a required pointer is NULL") != 0) return 7;
+  puts("ok");
+  return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(tp.LIB_PATH)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                        "-L", libdir, "-l:libtp.so", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
