@@ -98,7 +98,8 @@ struct AttnArgs {
   int* err;
 };
 
-cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s);
+// Persistent over work items: at most num_sms CTAs.
+cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, int num_sms, cudaStream_t s);
 
 // One CTA whose bounded wait on an mbarrier that nothing arrives on must run
 // out after limit_ns and set kErrTimeout in *err (watchdog.cu).

@@ -30,6 +30,14 @@ def test_sdpa_step(M, Hs, T):
             assert_rounded_once(g[r][:, j * 128:(j + 1) * 128], o.sdpa(Q, K, V), f"sdpa r={r} j={j}")
 
 
+# More work items (shard, head, 256 query rows) than SMs: the persistent kernel
+# walks several items per CTA (149 items: one CTA takes two; 400 items with
+# ragged query and key blocks; 300 items of two whole query blocks each).
+@pytest.mark.parametrize("M,Hs,T", [(256, 149, 1), (333, 100, 2), (512, 150, 1)])
+def test_sdpa_several_items_per_cta(M, Hs, T):
+    test_sdpa_step(M, Hs, T)
+
+
 def test_sdpa_large_scores_rescale_path():
     # Scores spread over a wide range force the running-max rescale of O.
     M, Hs, T = 512, 1, 1
@@ -43,6 +51,22 @@ def test_sdpa_large_scores_rescale_path():
     torch.cuda.synchronize()
     ref = o.sdpa(q[0][:, :128], q[0][:, 128:256], q[0][:, 256:])
     assert_rounded_once(from_dev(O)[0], ref, "sdpa wide scores")
+
+
+def test_sdpa_huge_scores():
+    # Scores of a few thousand (Q scaled by 64, exact in fp16): the softmax is
+    # nearly one-hot and the kernel's row-max estimate sits furthest from the
+    # true max; the result must still be the rounded exact attention.
+    M = 384
+    QKV = syn.normal_f16((1, M, 3 * 128), 1.0, seed=11, tid=402)
+    q = syn.f16_bits_to_f64(QKV)
+    QKV[0][:, :128] = (q[0][:, :128] * 64.0).astype(np.float16).view(np.uint16)
+    q = syn.f16_bits_to_f64(QKV)
+    O = torch.empty((1, M, 128), dtype=torch.int16, device="cuda")
+    assert tp.tp_sdpa_shards(to_dev(QKV), M, 1, 1, O) == 0
+    torch.cuda.synchronize()
+    ref = o.sdpa(q[0][:, :128], q[0][:, 128:256], q[0][:, 256:])
+    assert_rounded_once(from_dev(O)[0], ref, "sdpa huge scores")
 
 
 @pytest.mark.parametrize("M,heads,T", [(200, 4, 2), (64, 2, 1), (333, 4, 4)])
