@@ -250,7 +250,7 @@ tp_status run_sdpa(DeviceInfo* di, const uint16_t* QKV, int64_t M, int heads, in
   a.out = O;
   a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(TP_HEAD_DIM)));  // log2(e) / sqrt(d)
   a.err = di->err;
-  return launch_attention(map, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return launch_attention(map, a, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 // Slices of whole weights (all T shards), used by the one-shot calls and prepare.

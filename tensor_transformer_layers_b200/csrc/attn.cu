@@ -58,6 +58,13 @@
 namespace tp {
 namespace {
 
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 constexpr int kD = 128;             // head dim
 constexpr int kBQ = 128;            // query rows per tile
 constexpr int kTiles = 2;           // query tiles per CTA
@@ -347,8 +354,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // Row max: 3-input max over four independent chains (64 instructions
         // for 128 scores, a short dependency chain).  The element-wise code
-        // below uses packed fp32 pairs: scalar fp32 arithmetic at this rate on
-        // every sub-partition slows the other tile's concurrent MMAs.
+        // below uses packed fp32 pairs: measured on B200, scalar fp32
+        // add/mul/fma/max issued at this rate by warps on all four SM
+        // sub-partitions slow concurrent tcgen05 MMAs by a third or more (a
+        // 128x128x16 MMA from 64 to ~95-106 cycles), while the packed forms,
+        // MUFU, conversions and integer ALU work at the same rate do not.
         float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
         for (int q = 0; q < (kBKV - 4) / 2; ++q) m4[q & 3] = fmax3(m4[q & 3], s[4 + 2 * q], s[5 + 2 * q]);
@@ -457,15 +467,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
+  int dev = 0, num_sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess && num_sms <= 0) e = cudaErrorInvalidValue;
+  if (e != cudaSuccess) return note_cuda_error("attention: SM count", e);
   // Persistent: one CTA per SM (at most one per work item), each walking the
   // items blockIdx.x, blockIdx.x + gridDim.x, ... so that one item's last
   // blocks and output overlap the next item's Q/K/V loads and first S.
   const int q_blocks = (a.M + kTiles * kBQ - 1) / (kTiles * kBQ);
   const int64_t n_items = int64_t(q_blocks) * a.T * a.Hs;
   const int64_t grid = n_items < num_sms ? n_items : num_sms;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return note_cuda_error("attention: set shared memory size", e);
   attn_tc_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(qkv_map, a);
   count_launch();

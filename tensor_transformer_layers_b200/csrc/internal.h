@@ -98,8 +98,7 @@ struct AttnArgs {
   int* err;
 };
 
-// Persistent over work items: at most num_sms CTAs.
-cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, int num_sms, cudaStream_t s);
+cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s);
 
 // One CTA whose bounded wait on an mbarrier that nothing arrives on must run
 // out after limit_ns and set kErrTimeout in *err (watchdog.cu).

@@ -394,10 +394,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // Packed fp32 pairs (sm_100): one instruction operates on two fp32 values in a
 // 64-bit register pair, halving the instruction count of element-wise code.
-// Measured on B200: scalar fp32 add/mul/fma/max issued at a high rate by warps
-// on all four SM sub-partitions slow concurrent tcgen05 MMAs by a third or more
-// (a 128x128x16 MMA from 64 to ~95-106 cycles), while the packed forms, MUFU,
-// conversions and integer ALU work at the same element rate do not.
 __device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -422,13 +418,6 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
   return d;
 }
 
-// max(a, b, c) in one instruction (sm_100).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -446,13 +435,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Element-wise max of two bf16 pairs.
-__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 
