@@ -58,6 +58,9 @@
 namespace tp {
 namespace {
 
+// Waits until no TMA store of this thread still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // max(a, b, c) in one instruction (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
@@ -78,7 +81,9 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kQOff = 0;
 constexpr int kKVOff = kTiles * kQBytes;
-constexpr int kBarOff = kKVOff + kStages * kKVBytes;
+constexpr int kOutBuf = 32 * 128;                  // one softmax warp's staging box: 32 rows x 64 bf16
+constexpr int kOutOff = kKVOff + kStages * kKVBytes;  // 8 staging boxes, one per softmax warp
+constexpr int kBarOff = kOutOff + 8 * kOutBuf;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 constexpr uint32_t kColS0 = 0, kColO0 = 256;  // tile t: S at kColS0 + 128 t, O at kColO0 + 128 t
 constexpr uint32_t kIdescS = idesc_f32acc(kBQ, kBKV, false, false);  // fp16 Q, K
@@ -104,7 +109,8 @@ __device__ __forceinline__ AttnItem attn_item(int i, int q_blocks, int Hs) {
 // 320 threads: ten warps, so some SM sub-partitions (16K registers each) hold
 // three of them, which caps a thread at 168 registers.
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap qkv, const AttnArgs p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qkv, const __grid_constant__ CUtensorMap omap,
+                   const AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
@@ -424,36 +430,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_t) waits for that arrival.
       if (ok) ok = mbar_wait(&o_done[t], k & 1, abort_flag);
       if (ok) {
+        // O_t / l in bf16, 64 columns at a time: staged in this warp's box in
+        // the 128-byte swizzle of the output map, then one TMA store (whole
+        // 128-byte lines; rows >= M are clipped, a box wholly below M skipped).
         tc_fence_after();
         const AttnItem it = attn_item(int(blockIdx.x) + k * int(gridDim.x), q_blocks, p.Hs);
-        const int row = it.qb * (kTiles * kBQ) + t * kBQ + (warp & 3) * 32 + lane;
+        const int row0 = it.qb * (kTiles * kBQ) + t * kBQ + (warp & 3) * 32;
         const float inv_l = 1.0f / l_run;
         const uint64_t inv_l2 = f32x2(inv_l, inv_l);
-        uint16_t* orow = p.out + (int64_t(it.shard) * p.M + row) * int64_t(p.Hs * kD) + it.head * kD;
+        uint8_t* stg = smem + kOutOff + warp * kOutBuf;
 #pragma unroll 1
-        for (int c = 0; c < kD / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(c * 32), r);
-          uint32_t w[16];
+        for (int half = 0; half < 2; ++half) {
+          if (lane == 0) bulk_wait_read_0();  // the previous store has read the box
+          __syncwarp();
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r[32];
+            tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(half * 64 + c * 32), r);
+            uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float lo, hi;
-            f32x2_split(mul_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv_l2), lo, hi);
-            w[i] = pack_bf16x2(lo, hi);
+            for (int i = 0; i < 16; ++i) {
+              float lo, hi;
+              f32x2_split(mul_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv_l2), lo, hi);
+              w[i] = pack_bf16x2(lo, hi);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int chunk = c * 4 + q;  // 16-byte chunk of this lane's 128-byte row
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                  make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            }
           }
-          uint4 o[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) o[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-          if (row < p.M) {
-            uint4* op = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) op[i] = o[i];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.M) {
+            tma_store_3d(&omap, stg, it.head * kD + half * 64, row0, it.shard);
+            bulk_commit();
           }
         }
         tc_fence_before();
       }
     }
     if (!ok && lane == 0) report_timeout(p.err, abort_flag);
+    if (lane == 0) bulk_wait_all();  // this warp's TMA stores are complete before the CTA exits
   }
 
   tc_fence_before();
@@ -480,9 +499,14 @@ cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cuda
   const int q_blocks = (a.M + kTiles * kBQ - 1) / (kTiles * kBQ);
   const int64_t n_items = int64_t(q_blocks) * a.T * a.Hs;
   const int64_t grid = n_items < num_sms ? n_items : num_sms;
+  // O [T][M][Hs*128] bf16, written in 64-column x 32-row boxes
+  CUtensorMap omap;
+  if (make_map_out_u16(&omap, a.out, uint64_t(a.Hs) * kD, uint64_t(a.M), uint64_t(a.T), uint64_t(a.Hs) * kD, 0) !=
+      CUDA_SUCCESS)
+    return note_cuda_error("attention: output tensor map encode", cudaErrorInvalidValue);
   e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return note_cuda_error("attention: set shared memory size", e);
-  attn_tc_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(qkv_map, a);
+  attn_tc_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(qkv_map, omap, a);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) {
