@@ -73,7 +73,9 @@ typedef enum {
   TP_ERR_BAD_STYLE = 11,         /* unknown tp_style */
   TP_ERR_BAD_HANDLE = 12,        /* NULL or foreign handle */
   TP_ERR_SCRATCH_LIMIT = 13,     /* problem too large for the no-allocation entry point's fixed scratch */
-  TP_ERR_BAD_BLOCKS = 14         /* packed blocks: count outside 1..64, a block < 1, or sum not dividing the dim */
+  TP_ERR_BAD_BLOCKS = 14,        /* packed blocks: count outside 1..64, a block < 1, or sum not dividing the dim */
+  TP_ERR_RANGE = 15              /* an fp16 activation (e.g. the Q/K/V feeding attention) was outside the fp16
+                                    range or NaN; reported by tp_check_device_error */
 } tp_status;
 
 typedef enum {
@@ -110,8 +112,14 @@ uint64_t tp_kernel_launches(void);
 tp_status tp_debug_watchdog(uint32_t wait_ms, void* stream);
 
 /* Synchronises `stream`, then reports (and clears) the device error word that
- * the kernels' bounded waits set: TP_OK, or TP_ERR_DEVICE_TIMEOUT.  Returns
- * TP_ERR_CUDA if the synchronisation itself fails. */
+ * kernels set: TP_ERR_DEVICE_TIMEOUT if a bounded wait ran out, else
+ * TP_ERR_RANGE if an epilogue that stores fp16 (the Q/K/V of the attention
+ * layers, or tp_colwise_linear with TP_OUT_F16) produced a value whose fp16
+ * rounding is +-inf or NaN (|v| >= 65520, or NaN), else TP_OK.  The kernel
+ * that sets TP_ERR_RANGE still writes its whole output (the affected values
+ * as +-inf or NaN) and the context stays usable; the status says the output
+ * of that call must not be trusted.  Returns TP_ERR_CUDA if the
+ * synchronisation itself fails. */
 tp_status tp_check_device_error(void* stream);
 
 /* ---------------------------------------------------------------------------
@@ -209,7 +217,9 @@ tp_status tp_shard_packed_all(const uint16_t* W, int64_t rows, int64_t cols, int
  * when gelu != 0, identity otherwise.  bf16 operands, fp32 accumulation in
  * tensor memory (tcgen05), one rounding at the end to out_dtype
  * (TP_OUT_BF16, or TP_OUT_F16 as used for the Q/K/V that feed attention;
- * anything else is TP_ERR_BAD_STYLE).
+ * anything else is TP_ERR_BAD_STYLE).  With TP_OUT_F16 a value that rounds
+ * to +-inf (outside the fp16 range) or is NaN sets the range flag that
+ * tp_check_device_error() reports as TP_ERR_RANGE.
  * Requires K % 8 == 0 and N_s % 8 == 0 (ALIGNMENT).  M == 0 is a no-op. */
 tp_status tp_colwise_linear(const uint16_t* X, int64_t M, int64_t K,
                             const uint16_t* W_shards, const uint16_t* b_shards, int64_t N_s,
@@ -313,7 +323,10 @@ tp_status tp_swiglu_mlp_pair(const uint16_t* X, int64_t M, int64_t D, int64_t F,
 
 /* Attention block: Y = bf16( sum_r O_r W_o,r^T ), O_r = per-shard SDPA of the
  * head-split QKV projection X W_qkv,r^T.  X[M x D], W_qkv[3D x D], W_o[D x D],
- * Y[M x D]; D == heads*128; heads % T == 0.  No biases.
+ * Y[M x D]; D == heads*128; heads % T == 0.  No biases.  Q, K and V are held
+ * in fp16: a projection value outside the fp16 range makes the next
+ * tp_check_device_error() return TP_ERR_RANGE (the attention weights P are
+ * at most 2^8 by construction and cannot overflow).
  * Workspace: tp_attn_workspace_bytes(). */
 size_t tp_attn_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree);
 tp_status tp_attn_block(const uint16_t* X, int64_t M, int64_t D,
@@ -390,7 +403,11 @@ void tp_destroy(void* handle);
  * rows do not fit (F > 262144) the call returns TP_ERR_SCRATCH_LIMIT before
  * launching anything.  Other checks as tp_mlp_pair.
  * The first call on a device looks up the array's device address (once per
- * device); make that first call before any stream capture.  Every call shares
+ * device); make that first call before any stream capture.  Under CUDA's
+ * default lazy module loading that first lookup is also when the driver
+ * creates the 64 MiB array on that device, so make the first call at start-up,
+ * before another allocator takes the device's free memory: after it, calls
+ * change the device's free memory by nothing.  Every call shares
  * the one array: calls that overlap on the GPU (different streams, or
  * different host threads on one device) race and corrupt each other's
  * results.  Nothing in the array has to start at zero: a chunk's activations

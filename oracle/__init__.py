@@ -212,8 +212,9 @@ def mlp_unsharded(X, W_up, b_up, W_down, b_down, act=gelu_tanh):
 
 
 def mlp_colwise_shard(X, W_up, b_up, tp_degree, rank, act=gelu_tanh):
-    """H_r = act(X W_up,r^T + b_up,r): shard r's slice of the FFN hidden activations."""
-    return act(linear(X, slice_colwise(W_up, tp_degree, rank), slice_colwise(b_up, tp_degree, rank)))
+    """H_r = act(X W_up,r^T + b_up,r): shard r's slice of the FFN hidden activations (b_up may be None)."""
+    b_r = None if b_up is None else slice_colwise(b_up, tp_degree, rank)
+    return act(linear(X, slice_colwise(W_up, tp_degree, rank), b_r))
 
 
 def mlp_rowwise_partial(H_r, W_down, tp_degree, rank):

@@ -31,7 +31,7 @@ STATUS = {
     4: "TP_ERR_INDIVISIBLE", 5: "TP_ERR_HEADS_INDIVISIBLE", 6: "TP_ERR_BAD_SHAPE",
     7: "TP_ERR_ALIGNMENT", 8: "TP_ERR_WORKSPACE", 9: "TP_ERR_CUDA",
     10: "TP_ERR_DEVICE_TIMEOUT", 11: "TP_ERR_BAD_STYLE", 12: "TP_ERR_BAD_HANDLE",
-    13: "TP_ERR_SCRATCH_LIMIT", 14: "TP_ERR_BAD_BLOCKS",
+    13: "TP_ERR_SCRATCH_LIMIT", 14: "TP_ERR_BAD_BLOCKS", 15: "TP_ERR_RANGE",
 }
 
 _P = ctypes.c_void_p

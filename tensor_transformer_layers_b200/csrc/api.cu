@@ -81,6 +81,14 @@ inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+int mlp_shape_status(int64_t M, int64_t D, int64_t F, int T) {
+  if (T < 1) return TP_ERR_BAD_DEGREE;
+  if (M < 0 || D < 1 || F < 1 || M >= kMaxDim || D >= kMaxDim || F >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (F % T != 0) return TP_ERR_INDIVISIBLE;
+  if (D % 8 != 0 || (F / T) % 8 != 0) return TP_ERR_ALIGNMENT;
+  return TP_OK;
+}
+
 thread_local char g_last_error[512] = "";
 
 cudaError_t note_cuda_error(const char* where, cudaError_t e, const char* detail) {
@@ -361,11 +369,7 @@ tp_status check_packed(const uint16_t* W, int64_t rows, int64_t cols, int style,
 // Shape checks shared by the layer calls.
 // ---------------------------------------------------------------------------
 tp_status check_mlp_shape(int64_t M, int64_t D, int64_t F, int T) {
-  if (T < 1) return TP_ERR_BAD_DEGREE;
-  if (M < 0 || D < 1 || F < 1 || M >= kMaxDim || D >= kMaxDim || F >= kMaxDim) return TP_ERR_BAD_SHAPE;
-  if (F % T != 0) return TP_ERR_INDIVISIBLE;
-  if (D % 8 != 0 || (F / T) % 8 != 0) return TP_ERR_ALIGNMENT;
-  return TP_OK;
+  return tp_status(mlp_shape_status(M, D, F, T));
 }
 
 tp_status check_attn_shape(int64_t M, int64_t D, int heads, int T) {
@@ -553,6 +557,8 @@ const char* tp_status_string(int s) {
     case TP_ERR_BAD_BLOCKS:
       return "packed blocks invalid: count outside 1..64, a block < 1, or their sum does not divide the packed "
              "dimension";
+    case TP_ERR_RANGE:
+      return "an fp16 activation (Q/K/V) was outside the fp16 range or NaN; the call's output is not valid";
     case TP_ERR_SCRATCH_LIMIT:
       return "size exceeds the 64 MiB static scratch of tp_mlp_pair_sharded_noalloc (F * 256 bytes must fit)";
     default: return "unknown status";
@@ -575,7 +581,7 @@ tp_status tp_check_device_error(void* stream) {
   if (v != 0) {
     const int zero = 0;
     if (cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TP_ERR_CUDA;
-    return TP_ERR_DEVICE_TIMEOUT;
+    return (v & kErrTimeout) ? TP_ERR_DEVICE_TIMEOUT : TP_ERR_RANGE;
   }
   return TP_OK;
 }

@@ -91,6 +91,9 @@ constexpr uint32_t kIdescPV = idesc_f32acc(kBQ, kD, false, true);    // fp16 P, 
 constexpr float kRescaleThreshold = 8.0f;                           // log2 units
 
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+// The output staging boxes use the 128-byte swizzle (chunk ^ (row & 7)), which
+// is defined relative to 1024-byte-aligned boxes.
+static_assert(kOutOff % 1024 == 0 && kOutBuf % 1024 == 0, "output staging boxes must be 1024-byte aligned");
 
 // Work item i (query block qb = i % q_blocks of head-slot hs = i / q_blocks,
 // hs = shard * Hs + head); consecutive items share a head's K and V in L2.

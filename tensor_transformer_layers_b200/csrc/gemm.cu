@@ -161,6 +161,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& p, const CUtensorM
   const uint16_t* bias = p.bias ? p.bias + int64_t(g) * p.bias_gstride : nullptr;
   const int n_left = p.N - col_base;
   const int boxes = n_left >= width ? width / 64 : (n_left > 0 ? (n_left + 63) / 64 : 0);  // warp-uniform
+  uint32_t nonfinite = 0;  // fp16 outputs: any half that rounded to +-inf or NaN
   for (int b = 0; b < boxes; ++b) {
     uint8_t* buf = next_buf(stage, nbox, lane);
 #pragma unroll
@@ -198,6 +199,9 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& p, const CUtensorM
           o.y = pack_f16x2(v[8 * j + 2], v[8 * j + 3]);
           o.z = pack_f16x2(v[8 * j + 4], v[8 * j + 5]);
           o.w = pack_f16x2(v[8 * j + 6], v[8 * j + 7]);
+          // Columns past N are never stored; only the stored ones may raise the flag.
+          if (col0 + 8 * j < p.N)
+            nonfinite |= f16x2_nonfinite(o.x) | f16x2_nonfinite(o.y) | f16x2_nonfinite(o.z) | f16x2_nonfinite(o.w);
         } else {
           o.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
           o.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
@@ -209,6 +213,10 @@ __device__ __forceinline__ void epilogue_rows(const GemmArgs& p, const CUtensorM
     }
     store_box(omap, buf, lane, col_base + b * 64, row0, g, p.M);
   }
+  // A value outside the fp16 range became +-inf (or was NaN): record it, so
+  // the caller learns of it instead of receiving silent infinities.  Rows past
+  // M are zero-filled operands, hence finite, and are never stored anyway.
+  if (p.out_f16 && __any_sync(0xffffffffu, nonfinite != 0u) && lane == 0 && p.err) atomicOr(p.err, kErrRange);
 }
 
 // SwiGLU drain of one accumulator: columns [0, 128) hold gate, [128, 256) the

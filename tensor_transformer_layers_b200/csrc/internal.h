@@ -107,6 +107,12 @@ cudaError_t launch_watchdog_probe(int* err, uint64_t limit_ns, cudaStream_t s);
 // Counts kernel launches (api.cu); every launcher calls it once per launch.
 void count_launch();
 
+// Shape checks of an MLP pair (M tokens, hidden D, FFN width F, degree T), as
+// every MLP entry point applies them (api.cu); returns a tp_status value.
+int mlp_shape_status(int64_t M, int64_t D, int64_t F, int T);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 // Records why a CUDA call failed (thread-local; read by tp_last_error_message)
 // and returns `e` so launchers can `return note_cuda_error(...)`.
 cudaError_t note_cuda_error(const char* where, cudaError_t e, const char* detail = nullptr);

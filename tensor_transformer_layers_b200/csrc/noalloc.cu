@@ -27,6 +27,10 @@ constexpr int64_t kChunkAlign = 128;  // GEMM tile height
 
 // The scratch itself.  In host code this name is only a stand-in for the
 // symbol, never a device address: the address comes from cudaGetSymbolAddress.
+// This file holds no kernel, so under CUDA's lazy module loading (the default)
+// the driver creates the array on a device when its address is first looked
+// up there, i.e. inside the first call on that device; with eager loading it
+// exists as soon as the library's modules are loaded.
 static __device__ __align__(256) uint16_t g_noalloc_scratch[kScratchBytes / sizeof(uint16_t)];
 
 std::mutex g_mu;
@@ -46,8 +50,6 @@ tp_status scratch_address(void** out) {
   return TP_OK;
 }
 
-inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace tp
 
@@ -58,14 +60,12 @@ extern "C" tp_status tp_mlp_pair_sharded_noalloc(const uint16_t* X, int64_t M, i
                                                  const uint16_t* W_down_shards, const uint16_t* b_down,
                                                  int tp_degree, uint16_t* Y, void* stream) {
   if (!X || !W_up_shards || !W_down_shards || !Y) return TP_ERR_NULL;
-  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
-  if (M < 0 || D < 1 || F < 1 || M >= (int64_t(1) << 31) || D >= (int64_t(1) << 31) || F >= (int64_t(1) << 31))
-    return TP_ERR_BAD_SHAPE;
-  if (F % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  // The same shape rules as every other MLP entry point (one shared check).
+  const int shape = mlp_shape_status(M, D, F, tp_degree);
+  if (shape != TP_OK) return tp_status(shape);
   const int64_t Fs = F / tp_degree;
-  if (D % 8 != 0 || Fs % 8 != 0) return TP_ERR_ALIGNMENT;
-  if (!al16(X) || !al16(W_up_shards) || !al16(W_down_shards) || !al16(Y) || (b_up_shards && !al16(b_up_shards)) ||
-      (b_down && !al16(b_down)))
+  if (!aligned16(X) || !aligned16(W_up_shards) || !aligned16(W_down_shards) || !aligned16(Y) ||
+      (b_up_shards && !aligned16(b_up_shards)) || (b_down && !aligned16(b_down)))
     return TP_ERR_ALIGNMENT;
   // One token's activations across all shards take 2*F bytes; a chunk must hold
   // at least one 128-row tile of them.

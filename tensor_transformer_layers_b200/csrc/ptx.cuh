@@ -17,8 +17,11 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // many polling rounds (32 try_waits each).
 constexpr uint32_t kWaitMaxRounds = 1u << 21;
 
-// Device error word bits (OR-ed in by any CTA whose wait ran out).
+// Device error word bits: kErrTimeout is OR-ed in by any CTA whose wait ran
+// out; kErrRange by an epilogue that rounded a value to fp16 and got +-inf or
+// NaN (the value was outside the fp16 range, or was not a number).
 constexpr int kErrTimeout = 1;
+constexpr int kErrRange = 2;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -436,6 +439,12 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Nonzero iff either fp16 half of `w` is +-inf or NaN (exponent field all
+// ones).  Integer ALU only.
+__device__ __forceinline__ uint32_t f16x2_nonfinite(uint32_t w) {
+  return __vcmpeq2(w & 0x7C007C00u, 0x7C007C00u);  // 0xFFFF in each half whose exponent is all ones
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }

@@ -1,8 +1,10 @@
 """The full wide block (attention then MLP pair, tp_degree 8, 16384 tokens x
 6144 hidden, 48 heads, FFN 24576) on the GPU.  The oracle computes K and V for
-every token but only a seeded sample of query rows (rows 0 and M-1 always
-included): queries are independent given K and V, so those rows of the full
-output are exact."""
+every token but only a seeded sample of 256 query rows: rows 0 and M-1, one
+row inside every 128-row query tile (so every work item of the persistent
+SDPA, on every CTA and in every wave, has at least one checked row) and
+seeded extra rows.  Queries are independent given K and V, so those rows of
+the full output are exact."""
 import numpy as np
 import pytest
 import torch
@@ -14,7 +16,26 @@ from tests._util import assert_parity, f64, from_dev, to_dev
 
 pytestmark = pytest.mark.gpu
 
-N_ROWS = 48
+N_ROWS = 256
+Q_TILE = 128
+
+
+def sample_rows(M, n_rows, seed):
+    """Rows 0 and M-1, one seeded row in every Q_TILE-row query tile, then
+    seeded distinct extra rows up to n_rows."""
+    rng = np.random.default_rng(seed)
+    rows = {0, M - 1}
+    rows.update(t + int(rng.integers(0, min(Q_TILE, M - t))) for t in range(0, M, Q_TILE))
+    rest = np.setdiff1d(np.arange(M), np.fromiter(rows, dtype=np.int64))
+    rows.update(int(r) for r in rng.choice(rest, max(0, n_rows - len(rows)), replace=False))
+    return np.array(sorted(rows))
+
+
+def test_sample_covers_every_query_tile():
+    M = syn.CONFIGS["wide_block"]["M"]
+    rows = sample_rows(M, N_ROWS, 3)
+    assert len(rows) == N_ROWS and rows[0] == 0 and rows[-1] == M - 1
+    assert set(rows // Q_TILE) == set(range(M // Q_TILE))
 
 
 def test_wide_block_sampled_rows():
@@ -25,13 +46,13 @@ def test_wide_block_sampled_rows():
     A = tp.attn_block(dd["X"], dd["W_qkv"], dd["W_o"], H, T)
     Y = tp.mlp_pair(A, dd["W_up"], dd["b_up"], dd["W_down"], dd["b_down"], T)
     torch.cuda.synchronize()
+    assert tp.tp_check_device_error() == 0
     A_all, Y_all = from_dev(A), from_dev(Y)
     assert np.all(np.isfinite(f64(Y_all)))
     del dd, A, Y
     torch.cuda.empty_cache()
 
-    rng = np.random.default_rng(c["seed"])
-    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, N_ROWS - 2, replace=False)]))
+    rows = sample_rows(M, N_ROWS, c["seed"])
     f = {k: f64(v) for k, v in d.items()}
     A_ref, Y_ref = o.block_rows(f["X"], f["W_qkv"], f["W_o"], H, f["W_up"], f["b_up"], f["W_down"], f["b_down"],
                                 rows, tp_degree=T)

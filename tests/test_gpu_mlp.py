@@ -136,3 +136,31 @@ def test_bench_step_sequence_matches_one_shot(flux):
     for r in (0, T - 1):
         assert np.array_equal(from_dev(w_up[r]), o.slice_colwise(d["W_up"], T, r))
         assert np.array_equal(from_dev(w_down[r]), o.slice_rowwise(d["W_down"], T, r))
+
+
+def test_bench_step_equals_prepared_run(flux):
+    # bench.py's headline step is the two GEMM launches on shards sliced once;
+    # they must be exactly what tp_mlp_run does on a tp_mlp_prepare handle.
+    c, d, _ = flux
+    M, D, F, T = c["M"], c["D"], c["F"], c["T"]
+    Fs = F // T
+    dd = _dev(d)
+    w_up = torch.empty((T, Fs, D), dtype=torch.int16, device="cuda")
+    b_up = torch.empty((T, Fs), dtype=torch.int16, device="cuda")
+    w_down = torch.empty((T, D, Fs), dtype=torch.int16, device="cuda")
+    H = torch.empty((T, M, Fs), dtype=torch.int16, device="cuda")
+    Y = torch.empty((M, D), dtype=torch.int16, device="cuda")
+    jobs = [(dd["W_up"], F, D, tp.TP_COLWISE, w_up), (dd["W_down"], D, F, tp.TP_ROWWISE, w_down),
+            (dd["b_up"], T, Fs, tp.TP_COLWISE, b_up)]
+    assert tp.tp_shard_weights_batch(jobs, T) == 0
+    n0 = tp.tp_kernel_launches()
+    assert tp.tp_colwise_linear(dd["X"], M, D, w_up, b_up, Fs, T, 1, tp.TP_OUT_BF16, H) == 0
+    assert tp.tp_rowwise_linear_sum(H, M, Fs, w_down, D, dd["b_down"], T, Y) == 0
+    assert tp.tp_kernel_launches() - n0 == 2
+    pair = tp.MlpPair(dd["W_up"], dd["b_up"], dd["W_down"], dd["b_down"], T)
+    n0 = tp.tp_kernel_launches()
+    Yr = pair(dd["X"])
+    assert tp.tp_kernel_launches() - n0 == 2
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev(Y), from_dev(Yr))
+    pair.close()
