@@ -1093,6 +1093,122 @@ def run_ours(args, wl, rank, local_rank, world):
     return out
 
 
+def run_tp(args, wl, rank, local_rank, world):
+    """--mode tp: tensor parallelism across processes.  tp_degree = world size;
+    rank r holds only its own shards (cut once, as sharded loading would) and
+    every step runs its partial (tp_*_rank_partial), ONE NCCL AllReduce(sum)
+    of the fp32 [M x D] partial, and the finish (bias once, one bf16 rounding,
+    tp_reduce_partials).  The layer's total work is fixed, so scaling is
+    "strong"; X is replicated (every rank gets the same tokens)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import tensor_transformer_layers_b200 as tp
+    from tensor_transformer_layers_b200.dist import AttnRank, MlpRank
+
+    if wl.key not in ("flux_mlp", "flux_attn"):
+        raise SystemExit("--mode tp runs the flux_mlp or flux_attn workload")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    T = world
+    d = wl.host_inputs(0)
+    host = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16)).pin_memory() for k, v in d.items()}
+    g = {k: v.to(dev) for k, v in host.items()}
+    c = wl.cfg
+    M, D = c["M"], c["D"]
+    if wl.key == "flux_mlp":
+        obj = MlpRank(g["W_up"], g["b_up"], g["W_down"], g["b_down"], T, rank)
+    else:
+        obj = AttnRank(g["W_qkv"], g["W_o"], c["H"], T, rank)
+    part = torch.empty((M, D), dtype=torch.float32, device=dev)
+    Y = torch.empty((M, D), dtype=torch.int16, device=dev)
+    grouped = dist.is_available() and dist.is_initialized()
+
+    def step(ev, X):
+        ev[0].record()
+        obj.partial(X, out=part)
+        ev[1].record()
+        if grouped:
+            dist.all_reduce(part, op=dist.ReduceOp.SUM)
+        ev[2].record()
+        obj.finish(part, out=Y)
+        ev[3].record()
+
+    new_events = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]  # noqa: E731
+    for _ in range(args.warmup):
+        step(new_events(), g["X"])
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    evs = [new_events() for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = tp.tp_kernel_launches()
+    sampler.start()
+    for i in range(args.steps):
+        step(evs[i], g["X"])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    launches = tp.tp_kernel_launches() - launches0
+    barrier()
+    assert tp.tp_check_device_error() == 0
+    parts_ms = [[ev[j].elapsed_time(ev[j + 1]) for ev in evs] for j in range(3)]
+    local_s = sum(ev[0].elapsed_time(ev[3]) for ev in evs) / 1e3
+    max_s = max_over_ranks(local_s)
+    value = wl.work() * args.steps / max_s / 1e12
+
+    peaks, peak_src = load_peaks()
+    tc_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ar_bytes = 2.0 * (T - 1) / T * M * D * 4  # ring AllReduce bus bytes of the fp32 partial
+    fin_bytes = M * D * 4 + M * D * 2 + D * 2
+    ms = [statistics.mean(x) for x in parts_ms]
+    tot = sum(ms)
+    kinfo = {
+        "rank_partial": {"ms": round(ms[0], 5), "share": round(ms[0] / tot, 4), "unit": "TFLOP/s",
+                         "achieved": round(wl.work() / T / (ms[0] / 1e3) / 1e12, 1)},
+        "allreduce": {"ms": round(ms[1], 5), "share": round(ms[1] / tot, 4), "unit": "GB/s",
+                      "achieved": round(ar_bytes / (ms[1] / 1e3) / 1e9, 1) if ms[1] > 0 and T > 1 else None,
+                      "bytes": ar_bytes, "note": "NCCL AllReduce(sum) of the fp32 partial; bus bytes 2(T-1)/T x"},
+        "finish": {"ms": round(ms[2], 5), "share": round(ms[2] / tot, 4), "unit": "GB/s",
+                   "achieved": round(fin_bytes / (ms[2] / 1e3) / 1e9, 1)},
+    }
+    kinfo["rank_partial"]["frac"] = round(kinfo["rank_partial"]["achieved"] / tc_peak, 4)
+    kinfo["finish"]["frac"] = round(kinfo["finish"]["achieved"] / hbm_peak, 4)
+    # end to end: X copied in from pinned host memory and Y copied back every step
+    y_host = torch.empty((M, D), dtype=torch.int16).pin_memory()
+    x_dev = torch.empty_like(g["X"])
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        x_dev.copy_(host["X"], non_blocking=True)
+        step(new_events(), x_dev)
+        y_host.copy_(Y, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    barrier()
+    cfg = config_dict(wl, world)
+    cfg["tp_degree"] = T
+    cfg["global_batch_tokens"] = M
+    cfg["parallelism"] = (f"tp{T}: tensor parallelism across {T} process(es), one shard per rank, one NCCL "
+                          f"AllReduce(sum) of the fp32 [M x D] partial per layer, bias once after the sum")
+    return {
+        "metric": wl.metric, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * max_s / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)", "config": cfg,
+        "roofline": {"kernel": "rank_partial", "bound": "tensor", "achieved": kinfo["rank_partial"]["achieved"],
+                     "peak": tc_peak, "unit": "TFLOP/s", "frac": kinfo["rank_partial"]["frac"], "traffic": None,
+                     "peak_source": f"{peak_src}: bf16 burst"},
+        "kernels": kinfo, "clocks": clocks,
+        "e2e": {"value": wl.work() * args.steps / e2e_s / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": host["X"].numel() * 2, "d2h_bytes_per_step": M * D * 2,
+                "call": "rank partial + all_reduce + finish with X copied from pinned host memory, Y copied back"},
+        "gpu_launches": int(launches), "cpu_baseline": None,
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1103,6 +1219,10 @@ def main(argv=None):
                     help="flux_mlp (default: the headline line); the others time the remaining rows")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle leg (cpu_baseline is then null)")
+    ap.add_argument("--mode", choices=["replicas", "tp"], default="replicas",
+                    help="replicas (default): every GPU runs the whole layer (all tp_degree shards) on its own "
+                         "tokens; tp: tensor parallelism across the processes, one shard per rank, one NCCL "
+                         "AllReduce per layer (flux_mlp / flux_attn)")
     args = ap.parse_args(argv)
     rank, local_rank, world = dist_env()
     wl = WORKLOADS[args.workload]()
@@ -1119,6 +1239,8 @@ def main(argv=None):
     try:
         if args.impl == "reference":
             out = run_reference(args, wl, rank, world)
+        elif args.mode == "tp":
+            out = run_tp(args, wl, rank, local_rank, world)
         else:
             out = run_ours(args, wl, rank, local_rank, world)
         if rank == 0 and out is not None:

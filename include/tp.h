@@ -380,6 +380,43 @@ tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, 
                             int64_t M_txt, uint16_t* Y_img, uint16_t* Y_txt, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* ---------------------------------------------------------------------------
+ * One rank's share of a layer under tensor parallelism ACROSS processes (one
+ * process per GPU).  Page "Tensor parallelism", opening paragraph and the
+ * paragraph under the "Colwise and rowwise" table: rank r holds only its own
+ * shards, the colwise projection's output stays sharded on that rank, and the
+ * rowwise projection that follows yields a partial sum; a single AllReduce at
+ * the block boundary adds the partials.
+ *
+ * These calls compute rank r's partial of the layer output in fp32 [M x D],
+ * WITHOUT the rowwise bias.  The caller then sums the partials of all ranks
+ * with one AllReduce(sum) in fp32 (NCCL over NVLink; nothing here
+ * communicates) and finishes on every rank with
+ * tp_reduce_partials(summed, M, D, 1, b_down, Y): the bias added once, after
+ * the sum, and one bf16 rounding.  Summing the T partials of one process on
+ * one GPU with tp_reduce_partials(parts, M, D, T, b_down, Y) gives the same
+ * layer.  The rank index is implicit in the shards passed.
+ *
+ * MLP pair: X [M x D] (replicated); W_up_r [F/T x D] and b_up_r [F/T] (or
+ * NULL) = tp_shard_weight / tp_shard_bias of W_up, b_up for this rank;
+ * W_down_r [D x F/T] = tp_shard_weight(W_down, TP_ROWWISE, rank);
+ * part [M x D] fp32.  Same shape checks as tp_mlp_pair.  Workspace (this
+ * rank's hidden activations H_r, bf16): tp_mlp_rank_workspace_bytes().
+ *
+ * Attention block: X [M x D]; W_qkv_r [3D/T x D] = tp_shard_qkv_heads(W_qkv,
+ * ..., rank); W_o_r [D x D/T] = tp_shard_weight(W_o, D, D, TP_ROWWISE, ...,
+ * rank); part [M x D] fp32.  Same checks as tp_attn_block (Q/K/V in fp16 with
+ * the same TP_ERR_RANGE report).  Workspace: tp_attn_rank_workspace_bytes().
+ * ------------------------------------------------------------------------- */
+size_t tp_mlp_rank_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree);
+tp_status tp_mlp_rank_partial(const uint16_t* X, int64_t M, int64_t D, int64_t F, const uint16_t* W_up_r,
+                              const uint16_t* b_up_r, const uint16_t* W_down_r, int tp_degree, float* part, void* ws,
+                              size_t ws_bytes, void* stream);
+size_t tp_attn_rank_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree);
+tp_status tp_attn_rank_partial(const uint16_t* X, int64_t M, int64_t D, const uint16_t* W_qkv_r,
+                               const uint16_t* W_o_r, int heads, int tp_degree, float* part, void* ws,
+                               size_t ws_bytes, void* stream);
+
 /* Frees a handle from tp_*_prepare (synchronises the device first). NULL is a no-op. */
 void tp_destroy(void* handle);
 

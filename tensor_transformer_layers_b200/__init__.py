@@ -83,6 +83,10 @@ SIGNATURES = {
     "tp_colwise_linear_rows": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _I, _P, _I64, _P]),
     "tp_shard_weights_batch": (_I, [_P, _I, _I, _P]),
     "tp_rowwise_linear_sum_rows": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
+    "tp_mlp_rank_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
+    "tp_mlp_rank_partial": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _SZ, _P]),
+    "tp_attn_rank_workspace_bytes": (_SZ, [_I64, _I64, _I, _I]),
+    "tp_attn_rank_partial": (_I, [_P, _I64, _I64, _P, _P, _I, _I, _P, _P, _SZ, _P]),
 }
 
 _lib = None
@@ -361,6 +365,24 @@ def tp_joint_attn_run(handle, X_img, M_img, X_txt, M_txt, Y_img, Y_txt, ws, ws_b
 
 
 # --------------------------------------------------------------------------- convenience
+def tp_mlp_rank_workspace_bytes(M, D, F, tp_degree) -> int:
+    return lib().tp_mlp_rank_workspace_bytes(M, D, F, tp_degree)
+
+
+def tp_mlp_rank_partial(X, M, D, F, W_up_r, b_up_r, W_down_r, tp_degree, part, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_mlp_rank_partial(_ptr(X), M, D, F, _ptr(W_up_r), _ptr(b_up_r), _ptr(W_down_r), tp_degree,
+                                     _ptr(part), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def tp_attn_rank_workspace_bytes(M, D, heads, tp_degree) -> int:
+    return lib().tp_attn_rank_workspace_bytes(M, D, heads, tp_degree)
+
+
+def tp_attn_rank_partial(X, M, D, W_qkv_r, W_o_r, heads, tp_degree, part, ws, ws_bytes, stream=None) -> int:
+    return lib().tp_attn_rank_partial(_ptr(X), M, D, _ptr(W_qkv_r), _ptr(W_o_r), heads, tp_degree, _ptr(part),
+                                      _ptr(ws), ws_bytes, _stream(stream))
+
+
 def _u16(t: torch.Tensor) -> torch.Tensor:
     """bf16 bit patterns travel as 16-bit tensors; accept bfloat16 or int16/uint16 storage."""
     if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16, torch.float16):

@@ -138,6 +138,17 @@ CUresult make_map_out_u16(CUtensorMap* map, void* base, uint64_t n, uint64_t m, 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+CUresult make_map_out_f32(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t g, uint64_t row_stride,
+                          uint64_t group_stride) {
+  const cuuint64_t dims[3] = {n, m, g};
+  const cuuint64_t strides[2] = {row_stride * 4, (group_stride ? group_stride : row_stride * m) * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
                          uint32_t box1) {
   return make_map_3d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, d0, d1, d2, box0, box1);
@@ -178,7 +189,7 @@ tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, c
 // rowwise: Y = sum_r A[r] . W[r]^T + bias.  a_rows: rows of each shard's A
 // block in memory (0 = M; larger when A is a row range of a taller buffer).
 tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, const uint16_t* W, int64_t N,
-                      const uint16_t* bias, int T, uint16_t* Y, cudaStream_t s, int64_t a_rows = 0) {
+                      const uint16_t* bias, int T, void* Y, cudaStream_t s, int64_t a_rows = 0, bool out_f32 = false) {
   if (M == 0) return TP_OK;
   const GemmOperand Aop{A, uint64_t(Ks), uint64_t(M), uint64_t(T), uint64_t(a_rows)};
   const GemmOperand Bop{W, uint64_t(Ks), uint64_t(N), uint64_t(T)};
@@ -196,6 +207,7 @@ tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, 
   a.bias_gstride = 0;
   a.gelu = 0;
   a.out_f16 = 0;
+  a.out_f32 = out_f32 ? 1 : 0;
   a.err = di->err;
   return launch_gemm(Aop, Bop, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
@@ -530,6 +542,20 @@ JointLayout joint_layout(int64_t M, int64_t D, bool with_weights) {
 tp_status check_joint_shape(int64_t Mi, int64_t Mt, int64_t D, int heads, int T) {
   if (Mi < 0 || Mt < 0) return TP_ERR_BAD_SHAPE;
   return check_attn_shape(Mi + Mt, D, heads, T);
+}
+
+// One rank's workspaces: the MLP's hidden shard H_r [M x F/T] (bf16); the
+// attention's QKV_r [M x 3D/T] (fp16) and O_r [M x D/T] (bf16).
+size_t mlp_rank_ws(int64_t M, int64_t F, int T) { return up256(size_t(M) * (F / T) * 2); }
+struct AttnRankLayout {
+  size_t qkv, o, total;
+};
+AttnRankLayout attn_rank_layout(int64_t M, int64_t D, int T) {
+  AttnRankLayout L{};
+  L.qkv = 0;
+  L.o = up256(size_t(M) * 3 * (D / T) * 2);
+  L.total = L.o + up256(size_t(M) * (D / T) * 2);
+  return L;
 }
 
 }  // namespace
@@ -1193,6 +1219,61 @@ tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, 
   return joint_attn_forward(di, X_img, M_img, X_txt, M_txt, h->D, h->heads, h->T, h->w_qkv_img, h->w_qkv_txt,
                             h->w_o_img, h->w_o_txt, reinterpret_cast<uint16_t*>(w + L.qkv),
                             reinterpret_cast<uint16_t*>(w + L.o), Y_img, Y_txt, as_stream(stream));
+}
+
+// ----------------------------------------------------------------------- one rank's partial (multi-process TP)
+size_t tp_mlp_rank_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree) {
+  if (check_mlp_shape(M, D, F, tp_degree) != TP_OK) return 0;
+  return mlp_rank_ws(M, F, tp_degree);
+}
+
+tp_status tp_mlp_rank_partial(const uint16_t* X, int64_t M, int64_t D, int64_t F, const uint16_t* W_up_r,
+                              const uint16_t* b_up_r, const uint16_t* W_down_r, int tp_degree, float* part, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (!X || !W_up_r || !W_down_r || !part) return TP_ERR_NULL;
+  tp_status st = check_mlp_shape(M, D, F, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(X) || !al16(W_up_r) || !al16(W_down_r) || !al16(part) || (b_up_r && !al16(b_up_r)))
+    return TP_ERR_ALIGNMENT;
+  if (M == 0) return TP_OK;
+  if ((st = check_ws(ws, ws_bytes, mlp_rank_ws(M, F, tp_degree))) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const int64_t Fs = F / tp_degree;
+  uint16_t* H = static_cast<uint16_t*>(ws);
+  // this rank's colwise shard (one group) with bias + GELU, then its rowwise
+  // partial (one K shard) left in fp32 for the cross-rank sum; no bias here
+  if ((st = run_colwise(di, X, M, D, W_up_r, b_up_r, Fs, 1, 1, 0, H, s)) != TP_OK) return st;
+  return run_rowwise(di, H, M, Fs, W_down_r, D, nullptr, 1, part, s, 0, true);
+}
+
+size_t tp_attn_rank_workspace_bytes(int64_t M, int64_t D, int heads, int tp_degree) {
+  if (check_attn_shape(M, D, heads, tp_degree) != TP_OK) return 0;
+  return attn_rank_layout(M, D, tp_degree).total;
+}
+
+tp_status tp_attn_rank_partial(const uint16_t* X, int64_t M, int64_t D, const uint16_t* W_qkv_r,
+                               const uint16_t* W_o_r, int heads, int tp_degree, float* part, void* ws,
+                               size_t ws_bytes, void* stream) {
+  if (!X || !W_qkv_r || !W_o_r || !part) return TP_ERR_NULL;
+  tp_status st = check_attn_shape(M, D, heads, tp_degree);
+  if (st != TP_OK) return st;
+  if (!al16(X) || !al16(W_qkv_r) || !al16(W_o_r) || !al16(part)) return TP_ERR_ALIGNMENT;
+  if (M == 0) return TP_OK;
+  const AttnRankLayout L = attn_rank_layout(M, D, tp_degree);
+  if ((st = check_ws(ws, ws_bytes, L.total)) != TP_OK) return st;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const int64_t Ds = D / tp_degree;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* QKV = reinterpret_cast<uint16_t*>(w + L.qkv);
+  uint16_t* O = reinterpret_cast<uint16_t*>(w + L.o);
+  // this rank's heads only: QKV (fp16), SDPA over heads/T heads, rowwise partial in fp32
+  if ((st = run_colwise(di, X, M, D, W_qkv_r, nullptr, 3 * Ds, 1, 0, 1, QKV, s)) != TP_OK) return st;
+  if ((st = run_sdpa(di, QKV, M, heads / tp_degree, 1, O, s)) != TP_OK) return st;
+  return run_rowwise(di, O, M, Ds, W_o_r, D, nullptr, 1, part, s, 0, true);
 }
 
 void tp_destroy(void* handle) {

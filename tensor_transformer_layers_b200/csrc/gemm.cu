@@ -152,6 +152,51 @@ __device__ __forceinline__ uint8_t* next_buf(uint8_t* stage, uint32_t& nbox, int
   return buf;
 }
 
+// fp32 output (a rank's partial sum before the cross-rank AllReduce): each
+// 64-column chunk goes out as two 32-row x 32-column fp32 boxes (128-byte rows
+// in the output map's 128-byte swizzle); a half wholly past N is skipped.
+__device__ __forceinline__ void epilogue_rows_f32(const GemmArgs& p, const CUtensorMap* omap, uint32_t taddr,
+                                                  int row0, int lane, int g, int col_base, int width, uint8_t* stage,
+                                                  uint32_t& nbox) {
+  const uint16_t* bias = p.bias ? p.bias + int64_t(g) * p.bias_gstride : nullptr;
+  const int n_left = p.N - col_base;
+  const int halves = n_left >= width ? width / 32 : (n_left > 0 ? (n_left + 31) / 32 : 0);  // warp-uniform
+  for (int h = 0; h < halves; ++h) {
+    uint8_t* buf = next_buf(stage, nbox, lane);
+    uint32_t r[32];
+    __syncwarp();
+    tmem_ld32_sync(taddr + uint32_t(h * 32), r);
+    const int col0 = col_base + h * 32;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+    if (bias != nullptr) {
+      const uint4* bp = reinterpret_cast<const uint4*>(bias + col0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (col0 + 8 * j < p.N) {
+          const uint4 bb = __ldg(bp + j);
+          const uint32_t w[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            f32x2_split(add_f32x2(f32x2(v[8 * j + 2 * q], v[8 * j + 2 * q + 1]), f32x2(bf16_lo(w[q]), bf16_hi(w[q]))),
+                        v[8 * j + 2 * q], v[8 * j + 2 * q + 1]);
+        }
+      }
+    }
+    if (p.gelu) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) gelu_tanh2(v[j], v[j + 1]);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      stage16(buf, lane, j,
+              make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]), __float_as_uint(v[4 * j + 2]),
+                         __float_as_uint(v[4 * j + 3])));
+    store_box(omap, buf, lane, col0, row0, g, p.M);
+  }
+}
+
 // Drains `width` columns of a 128-row fp32 accumulator (this warp's 32 lanes,
 // TMEM columns from taddr, output columns from col_base, rows from row0) in
 // 64-column boxes: bias, GELU, rounding, staging, TMA store.
@@ -434,6 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = tc.mb * BM1 + q * 32;
       if (p.swiglu)
         epilogue_swiglu(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, stage, nbox);
+      else if (p.out_f32)
+        epilogue_rows_f32(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, out_bn, stage, nbox);
       else
         epilogue_rows(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, out_bn, stage, nbox);
       tc_fence_before();
@@ -622,6 +669,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = tc.mb * BM2 + int(rank) * 128 + q * 32;
       if (p.swiglu)
         epilogue_swiglu(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, stage, nbox);
+      else if (p.out_f32)
+        epilogue_rows_f32(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, out_bn, stage, nbox);
       else
         epilogue_rows(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, out_bn, stage, nbox);
       tc_fence_before();
@@ -688,9 +737,11 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
                         cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.groups <= 0) return cudaSuccess;
   CUtensorMap amap, bmap, omap;
-  if (make_map_out_u16(&omap, a.out, uint64_t(a.N), uint64_t(a.M), uint64_t(a.groups), uint64_t(a.ldo),
-                       uint64_t(a.out_gstride)) != CUDA_SUCCESS)
-    return note_cuda_error("gemm: output tensor map encode", cudaErrorInvalidValue);
+  const CUresult om = a.out_f32 ? make_map_out_f32(&omap, a.out, uint64_t(a.N), uint64_t(a.M), uint64_t(a.groups),
+                                                   uint64_t(a.ldo), uint64_t(a.out_gstride))
+                                : make_map_out_u16(&omap, a.out, uint64_t(a.N), uint64_t(a.M), uint64_t(a.groups),
+                                                   uint64_t(a.ldo), uint64_t(a.out_gstride));
+  if (om != CUDA_SUCCESS) return note_cuda_error("gemm: output tensor map encode", cudaErrorInvalidValue);
   if (a.M >= BM2) {
     // CTA-pair kernel: each CTA loads 128-row halves of both operands.
     if (make_a_map(&amap, A, a, 128) != CUDA_SUCCESS ||

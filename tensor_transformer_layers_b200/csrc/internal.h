@@ -60,13 +60,14 @@ struct GemmArgs {
   int kshards;           // shards walked by one tile's K loop
   int groups;            // output groups (colwise shards)
   int a_follows_shard;   // 1: A's z coordinate = K-loop shard; 0: z = 0
-  uint16_t* out;         // bf16 output
+  void* out;             // bf16 / fp16 / fp32 output
   int64_t out_gstride;   // elements between groups
   int64_t ldo;           // output row stride (elements)
   const uint16_t* bias;  // bf16 bias or nullptr
   int64_t bias_gstride;  // elements between groups' biases
   int gelu;              // 1: tanh-form GELU after bias
   int out_f16;           // 1: store fp16 instead of bf16
+  int out_f32;           // 1: store the fp32 accumulator values (after bias / GELU) unrounded
   int swiglu;            // 1: SwiGLU epilogue over [gate; up] weight rows (see above)
   int a_split_input;     // 1: A map is {K_s, T, M}, loaded at (k, s, row)
   int64_t up_off;        // SwiGLU: rows from gate_g to up_g in B (and bias elements)
@@ -131,6 +132,9 @@ CUresult make_map_3d_bf16_box(CUtensorMap* map, const void* base, uint64_t d0, u
 // Output map of the GEMM epilogue's TMA stores: 16-bit {n, m, g} with the
 // given row and group strides (elements), box 64 x 32, 128-byte swizzle.
 CUresult make_map_out_u16(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t g, uint64_t row_stride,
+                          uint64_t group_stride);
+// The same for fp32 outputs: box 32 x 32 (128-byte rows), 128-byte swizzle.
+CUresult make_map_out_f32(CUtensorMap* map, void* base, uint64_t n, uint64_t m, uint64_t g, uint64_t row_stride,
                           uint64_t group_stride);
 CUresult make_map_3d_f16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
                          uint32_t box1);

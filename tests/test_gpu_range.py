@@ -18,7 +18,7 @@ from tests._util import assert_parity, f64, from_dev, to_dev
 pytestmark = pytest.mark.gpu
 
 BF16_ONE = 0x3F80
-BF16_65280 = 0x477F  # largest bf16 below 65504: finite in fp16 (0x7BFC)
+BF16_65280 = 0x477F  # largest bf16 below 65504: finite in fp16 (0x7BF8)
 BF16_65536 = 0x4780  # 2^16: rounds to fp16 +inf
 
 
@@ -40,7 +40,7 @@ def _colwise_f16(w_bits):
 def test_fp16_output_just_inside_the_range_is_not_flagged():
     st, out = _colwise_f16(BF16_65280)
     assert tp.STATUS[st] == "TP_OK"
-    assert out[1, 299, 199] == 0x7BFC  # 65280 in fp16
+    assert out[1, 299, 199] == 0x7BF8  # 65280 = 2^15 * (1 + 1016/1024) in fp16
     out[1, 299, 199] = 0
     assert not out.any()
 
