@@ -186,15 +186,10 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 # --------------------------------------------------------------------------- workloads
-def blas_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
-    except Exception:  # noqa: BLE001
-        pass
-    return os.cpu_count() or 1
+def oracle_threads():
+    """Host threads the C++ oracle computes with (OpenMP; all cores by default)."""
+    import oracle as o
+    return o.num_threads()
 
 
 def _f64(d, keys):
@@ -859,7 +854,7 @@ def cpu_baseline(wl, d, budget_s: float = 12.0):
     if wl.key in ("flux_attn", "wide_block", "flux_joint_attn"):
         rows = min(rows, 256)  # the K/V projection of every token dominates; more rows add little
     t, done = wl.oracle_run(d, rows)
-    return {"value": done / t / _scale(wl.unit), "unit": wl.unit, "cores": blas_threads(), "kind": "oracle",
+    return {"value": done / t / _scale(wl.unit), "unit": wl.unit, "cores": oracle_threads(), "kind": "oracle",
             "sample": f"{rows} of {M} token rows of the workload through the fp64 oracle ({wl.oracle_fn}, "
                       f"tp_degree {wl.cfg['T']}), {t:.1f} s; value = work the oracle performed / time"}
 
@@ -886,7 +881,7 @@ def run_reference(args, wl, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_dict(wl, world),
-        "cpu_baseline": {"value": value, "unit": wl.unit, "cores": blas_threads(), "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": wl.unit, "cores": oracle_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": wl.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

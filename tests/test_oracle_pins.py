@@ -356,6 +356,8 @@ def _run_pins():
         "scale": test_sdpa_scale_closed_form,
         "mlp_int": lambda: test_mlp_sharded_equals_unsharded_exactly_on_integers(4),
         "mlp_closed": test_mlp_closed_form_on_integers,
+        "mlp_gelu": lambda: test_mlp_sharded_equals_unsharded_with_gelu(2),
+        "softmax": test_softmax_rows_sum_to_one_and_shift_invariant,
         "zero_q": test_attention_zero_queries_closed_form,
         "locality": test_attention_head_locality,
     }
@@ -372,38 +374,50 @@ def test_pins_pass_unmodified():
     assert _run_pins() == []
 
 
-def _mut_linear_transposed(X, W, b=None):
-    W = np.asarray(W, dtype=np.float64)
-    Y = np.asarray(X, dtype=np.float64) @ (W if W.shape[0] == np.asarray(X).shape[1] else W.T)
-    if b is not None:
-        Y = Y + b
-    return Y
-
-
+# Each planted mistake is a one-place edit of the oracle's C++ source: the
+# test compiles the edited copy into its own library and runs the pins on it.
 MUTANTS = {
-    "bias_per_shard": ("reduce_partials",
-                       lambda parts, bias=None: sum(np.asarray(p, float) for p in parts)
-                       + (0 if bias is None else len(parts) * np.asarray(bias)[None, :])),
-    "bias_dropped": ("linear", lambda X, W, b=None: np.asarray(X, float) @ np.asarray(W, float).T),
-    "transposed": ("linear", _mut_linear_transposed),
-    "colwise_off_by_one": ("slice_colwise",
-                           lambda W, T, r: W[((r + 1) % T) * (W.shape[0] // T):(((r + 1) % T) + 1) * (W.shape[0] // T)].copy()),
-    "rowwise_as_colwise": ("slice_rowwise",
-                           lambda W, T, r: W[:, r::T].copy()),
-    "gelu_coeff": ("gelu_tanh",
-                   lambda x: 0.5 * x * (1 + np.tanh(np.sqrt(2 / np.pi) * (x + 0.04715 * x ** 3)))),
-    "scale_sqrt_missing": ("sdpa",
-                           lambda Q, K, V, scale=None: o.softmax_rows(Q @ K.T) @ V),
-    "qkv_interleaved": ("slice_qkv_heads",
-                        lambda W, heads, T, r: W[r * (W.shape[0] // T):(r + 1) * (W.shape[0] // T)].copy()),
+    "bias_per_shard": ("Y[i * N + j] = bias ? acc + bias[j] : acc;",
+                       "Y[i * N + j] = bias ? acc + T * bias[j] : acc;"),
+    "bias_dropped": ("Y[(g * R + r) * N + j0 + q] = b ? acc[q][r] + b[j0 + q] : acc[q][r];",
+                     "Y[(g * R + r) * N + j0 + q] = acc[q][r];"),
+    "transposed": ("const double wk = w[q][k];", "const double wk = W[k * N + j0 + (q < nj ? q : 0)];"),
+    "colwise_off_by_one": ("std::memcpy(out, W + r * step * cols * es, size_t(step * cols * es));",
+                           "std::memcpy(out, W + ((r + 1) % T) * step * cols * es, size_t(step * cols * es));"),
+    "rowwise_strided": ("std::memcpy(out + i * step * es, W + (i * cols + r * step) * es, size_t(step * es));",
+                        "for (int64_t c = 0; c < step; ++c) "
+                        "std::memcpy(out + (i * step + c) * es, W + (i * cols + r + c * T) * es, size_t(es));"),
+    "gelu_coeff": ("0.044715 * x * x * x", "0.04715 * x * x * x"),
+    "scale_missing": ("for (int64_t t = 0; t < n * Mk; ++t) S[size_t(t)] *= scale;", ""),
+    "qkv_interleaved": ("return slice_packed_colwise(W, rows, D, es, blocks, 3, T, r, out);",
+                        "return slice_colwise(W, rows, D, es, T, r, out);"),
+    "activation_skipped": ("  apply_act(H, M * (F / T), act);\n  return kOk;", "  return kOk;"),
+    "softmax_unnormalised": ("for (int64_t j = 0; j < cols; ++j) p[j] /= l;", ""),
 }
 
 
+@pytest.fixture(scope="module")
+def mutant_libs(tmp_path_factory):
+    """Every mutant compiled once (in parallel) from an edited copy of oracle.cpp."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from oracle import build as ob
+    src = open(ob.SRC).read()
+    out = tmp_path_factory.mktemp("oracle_mutants")
+
+    def one(item):
+        name, (old, new) = item
+        assert src.count(old) == 1, f"mutant {name}: the edited text must occur exactly once"
+        return name, ob.compile_source(src.replace(old, new), str(out / f"lib_{name}.so"))
+
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        return dict(ex.map(one, MUTANTS.items()))
+
+
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_have_teeth(name, monkeypatch):
-    attr, fn = MUTANTS[name]
-    monkeypatch.setattr(o, attr, fn)
-    assert _run_pins() != [], f"planted mistake {name!r} was not caught by any pin"
+def test_pins_have_teeth(name, mutant_libs):
+    with o.using_library(mutant_libs[name]):
+        assert _run_pins() != [], f"planted mistake {name!r} was not caught by any pin"
 
 
 # ---------------------------------------------------------------------------
