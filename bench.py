@@ -550,6 +550,134 @@ class JointAttnWorkload(AttnWorkload):
                 "global_batch_tokens": (c["M_img"] + c["M_txt"]) * world}
 
 
+class RingAttnWorkload(AttnWorkload):
+    """flux_ring_attn: Ring attention ("Context parallelism" page) over the
+    flux_attn tokens, R = 4 ranks emulated on one GPU.  Q/K/V (24 heads x 128,
+    fp16, the projections a flux_attn block makes) are split into R token
+    blocks.  Step s: every rank r attends its queries to the key/value block
+    it holds then, rank (r - s) mod R's -- one tp_sdpa_block_stats launch over
+    all ranks, the blocks laid out twice so that the rotation is a pointer
+    offset (on R GPUs it is the NCCL send/recv of the block) -- and a final
+    tp_attn_merge per step combines the R results.  Work: the SDPA's 4 M^2 D."""
+    key = "flux_ring_attn"
+    metric = "Ring-attention (context parallel, 4 ranks on 1 GPU) TFLOP/s on 1 B200"
+    R = 4
+
+    def host_inputs(self, rank):
+        import synthetic as syn
+        c = self.cfg
+        return {"QKV": syn.normal_f16((c["M"], 3 * c["D"]), 1.0, seed=c["seed"] + rank, tid=420)}
+
+    def work(self):
+        M, D = self.cfg["M"], self.cfg["D"]
+        return 4.0 * M * M * D
+
+    def kernels(self, tp, g, dev):
+        import torch
+        c = self.cfg
+        M, D, H, R = c["M"], c["D"], c["H"], self.R
+        Ms = M // R
+        qkv = g["QKV"].view(R, Ms, 3 * D)
+        ring = torch.cat([qkv, qkv]).contiguous()  # blocks 0..R-1 twice: step s starts at block R - s
+        b = {"ring": ring, "O": torch.empty((R, R, Ms, D), dtype=torch.float32, device=dev),
+             "L": torch.empty((R, R, H, Ms), dtype=torch.float32, device=dev),
+             "Y": torch.empty((R, Ms, D), dtype=torch.int16, device=dev)}
+        self.bufs = b
+        ck = tp._check
+        blk = Ms * 3 * D  # elements per token block
+        ks = []
+        for st in range(R):
+            ks.append(Kernel(f"ring_step{st}", "TFLOP/s", 4.0 * M * Ms * D,
+                             lambda st=st: ck(tp.tp_sdpa_block_stats(qkv, Ms, ring.data_ptr() + 2 * (R - st) * blk,
+                                                                     Ms, H * R, R, b["O"][st], b["L"][st]),
+                                              f"ring step {st}")))
+        ks.append(Kernel("merge", "GB/s", R * (M * D * 4 + H * M * 4) + M * D * 2,
+                         lambda: ck(tp.tp_attn_merge(b["O"], b["L"], R, Ms, H * R, R, b["Y"]), "merge")))
+        return ks
+
+    def one_shot(self, tp, gi, dev):
+        """Every step's kernels on the staged inputs `gi` (buffers from torch's caching allocator)."""
+        for k in self.kernels(tp, gi, dev):
+            k.fn()
+        return self.bufs["Y"]
+
+    e2e_call = "tp_sdpa_block_stats per ring step and tp_attn_merge, Q/K/V copied from pinned host memory, O back"
+
+    def oracle_run(self, d, rows):
+        import oracle as o
+        import synthetic as syn
+        c = self.cfg
+        M, D, H = c["M"], c["D"], c["H"]
+        q = syn.f16_bits_to_f64(d["QKV"])
+        t0 = time.perf_counter()
+        for h in range(H):
+            o.sdpa(q[:rows, h * 128:(h + 1) * 128], q[:, D + h * 128:D + (h + 1) * 128],
+                   q[:, 2 * D + h * 128:2 * D + (h + 1) * 128])
+        return time.perf_counter() - t0, 4.0 * rows * M * D
+
+    oracle_fn = "sdpa over all keys (the result Ring attention must reach)"
+
+    def config(self, world):
+        c = self.cfg
+        return {"workload": (f"flux_ring_attn: Ring attention over {c['M']} tokens, {self.R} ranks emulated on one "
+                             f"GPU, {c['H']} heads x 128 (fp16 Q/K/V)"), "M": c["M"], "D": c["D"], "heads": c["H"],
+                "ring_degree": self.R, "global_batch_tokens": c["M"] * world}
+
+
+class UlyssesAttnWorkload(RingAttnWorkload):
+    """flux_ulysses_attn: Ulysses attention ("Context parallelism" page) over
+    the flux_attn tokens, U = 4 ranks emulated on one GPU.  Each rank packs
+    its tokens' Q/K/V by destination head group (packed rowwise slicing,
+    blocks [1, 1, 1]; all ranks in one launch), the all-to-all moves the
+    blocks (device copies here, timed as their own entry; NCCL on U GPUs),
+    each rank attends all M tokens of its H/U heads (one launch for all ranks:
+    the ranks are the SDPA's shards), the reverse all-to-all brings the rows
+    home and each rank puts its head groups back in place
+    (tp_unshard_rowwise_all).  Work: the SDPA's 4 M^2 D."""
+    key = "flux_ulysses_attn"
+    metric = "Ulysses-attention (context parallel, 4 ranks on 1 GPU) TFLOP/s on 1 B200"
+    R = 4
+
+    def kernels(self, tp, g, dev):
+        import torch
+        c = self.cfg
+        M, D, H, U = c["M"], c["D"], c["H"], self.R
+        Ms, C = M // U, 3 * D
+        qkv = g["QKV"].view(U, Ms, C)
+        b = {"send": torch.empty((U, U, Ms, C // U), dtype=torch.int16, device=dev),   # [src][dst]
+             "recv": torch.empty((U, U, Ms, C // U), dtype=torch.int16, device=dev),   # [dst][src] = [dst][M][..]
+             "O": torch.empty((U, M, D // U), dtype=torch.int16, device=dev),           # [rank = shard][M][(H/U) 128]
+             "back": torch.empty((U, U, Ms, D // U), dtype=torch.int16, device=dev),   # [dst][src]
+             "Y": torch.empty((U, Ms, D), dtype=torch.int16, device=dev)}
+        self.bufs = b
+        ck = tp._check
+        jobs = [(qkv[s], Ms, C, tp.TP_ROWWISE, b["send"][s], [1, 1, 1]) for s in range(U)]
+
+        def a2a(dst, src):  # the all-to-all: block [i][j] of src lands at [j][i] of dst
+            dst.copy_(src.transpose(0, 1))
+
+        return [
+            Kernel("pack", "GB/s", 2.0 * M * C * 2, lambda: ck(tp.tp_shard_weights_batch(jobs, U), "pack")),
+            Kernel("alltoall_emulated", "GB/s", 2.0 * M * C * 2, lambda: a2a(b["recv"], b["send"])),
+            Kernel("sdpa", "TFLOP/s", 4.0 * M * M * D,
+                   lambda: ck(tp.tp_sdpa_shards(b["recv"], M, H, U, b["O"]), "sdpa")),
+            Kernel("alltoall_back_emulated", "GB/s", 2.0 * M * D * 2,
+                   lambda: a2a(b["back"], b["O"].view(U, U, Ms, D // U))),
+            Kernel("unpack", "GB/s", 2.0 * M * D * 2,
+                   lambda: [ck(tp.tp_unshard_rowwise_all(b["back"][s], Ms, D, U, b["Y"][s]), "unpack")
+                            for s in range(U)]),
+        ]
+
+    e2e_call = ("pack, all-to-all (device copies), tp_sdpa_shards, all-to-all back, tp_unshard_rowwise_all; Q/K/V "
+                "copied from pinned host memory, O back")
+
+    def config(self, world):
+        d = RingAttnWorkload.config(self, world)
+        d["workload"] = d["workload"].replace("flux_ring_attn: Ring", "flux_ulysses_attn: Ulysses")
+        d["ulysses_degree"] = d.pop("ring_degree")
+        return d
+
+
 class BlockWorkload(AttnWorkload):
     """wide_block: attention then MLP pair at tp_degree 8 (every row a1..a7)."""
     key = "wide_block"
@@ -831,7 +959,8 @@ class SplitInputWorkload(MlpWorkload):
 
 
 WORKLOADS = {w.key: w for w in (MlpWorkload, SweepWorkload, AttnWorkload, BlockWorkload, ReduceWorkload,
-                                SwigluWorkload, SplitInputWorkload, JointAttnWorkload)}
+                                SwigluWorkload, SplitInputWorkload, JointAttnWorkload, RingAttnWorkload,
+                                UlyssesAttnWorkload)}
 
 
 def workload_cfg():

@@ -381,6 +381,45 @@ tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, 
                             void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Context parallelism pieces (page "Context parallelism": Ring attention
+ * passes key/value blocks around a ring of ranks, each attending its own
+ * queries to the block it holds; Ulysses attention regroups all tokens x a
+ * subset of heads onto each rank with an all-to-all, attends locally and
+ * regroups back).  These calls are the per-rank compute and layout steps;
+ * the exchanges themselves (ring send/recv, all-to-all) are the caller's
+ * collectives (NCCL over NVLink); nothing here communicates.
+ * ------------------------------------------------------------------------- */
+
+/* One key/value block of Ring attention, for every shard and head:
+ *   O[r][i, 128h:128h+128] = softmax_j(Q_i K_j^T / sqrt(128)) V_j   over the block's keys j,
+ *   lse[r][h][i] = log2 sum_j 2^(log2(e) Q_i K_j^T / sqrt(128))     (log2 units).
+ * Q_qkv: fp16 [T x Mq x 3*Hs*128] (its Q columns are used); KV_qkv: fp16
+ * [T x Mk x 3*Hs*128] (its K and V columns; may be the same buffer as Q_qkv,
+ * or another rank's block), Hs = heads / T.  O: fp32 [T x Mq x Hs*128], O
+ * normalised over this block's keys; lse: fp32 [T x Hs x Mq].  Mk >= 1.
+ * Errors: NULL, BAD_DEGREE, BAD_SHAPE, HEADS_INDIVISIBLE, ALIGNMENT. */
+tp_status tp_sdpa_block_stats(const uint16_t* Q_qkv, int64_t Mq, const uint16_t* KV_qkv, int64_t Mk, int heads,
+                              int tp_degree, float* O, float* lse, void* stream);
+
+/* Merge of nparts (1..64) block results into the attention over all their
+ * keys: O = sum_b 2^(lse_b - L) O_b / sum_b 2^(lse_b - L), L = max_b lse_b,
+ * written in bf16 like tp_sdpa_shards' output; lse_out (or NULL) receives
+ * L + log2 sum_b 2^(lse_b - L), so merges can be chained.  O_parts: fp32
+ * [nparts x T x M x Hs*128]; lse_parts: fp32 [nparts x T x Hs x M]; O: bf16
+ * [T x M x Hs*128]; lse_out: fp32 [T x Hs x M]. */
+tp_status tp_attn_merge(const float* O_parts, const float* lse_parts, int nparts, int64_t M, int heads,
+                        int tp_degree, uint16_t* O, float* lse_out, void* stream);
+
+/* Inverse of tp_shard_weight_all(..., TP_ROWWISE, ...): src [T x rows x cols/T]
+ * (block r) -> out [rows x cols] with block r at columns [r*cols/T, (r+1)*cols/T).
+ * Ulysses attention uses the rowwise / packed-rowwise slicing to group each
+ * rank's heads by destination before the all-to-all, and this call to put
+ * every head group back in place after the reverse all-to-all.  Bit-exact.
+ * cols % T == 0 (INDIVISIBLE); cols/T % 8 == 0 (ALIGNMENT). */
+tp_status tp_unshard_rowwise_all(const uint16_t* src, int64_t rows, int64_t cols, int tp_degree, uint16_t* out,
+                                 void* stream);
+
+/* ---------------------------------------------------------------------------
  * One rank's share of a layer under tensor parallelism ACROSS processes (one
  * process per GPU).  Page "Tensor parallelism", opening paragraph and the
  * paragraph under the "Colwise and rowwise" table: rank r holds only its own

@@ -62,6 +62,7 @@ _SIGS = {
     "oracle_softmax_rows": [_P, _I64, _I64, _P],
     "oracle_sdpa": [_P, _I64, _P, _P, _I64, _I64, _D, _P, _P],
     "oracle_reduce_partials": [_P, _I, _I64, _I64, _P, _P],
+    "oracle_attn_merge": [_P, _P, _I, _I64, _I64, _P, _P],
     "oracle_mlp_colwise_shard": [_P, _I64, _I64, _P, _P, _I64, _I, _I, _I, _P],
     "oracle_mlp_rowwise_partial": [_P, _I64, _P, _I64, _I64, _I, _I, _P],
     "oracle_mlp_sharded_summed": [_P, _I64, _I64, _P, _P, _I64, _P, _P, _I, _I, _P],
@@ -278,6 +279,19 @@ def sdpa(Q, K, V, scale: float | None = None, return_lse: bool = False):
     lse = np.empty(Mq)
     _call("oracle_sdpa", _p(Q), Mq, _p(K), _p(V), Mk, d, float(scale), _p(O), _p(lse))
     return (O, lse) if return_lse else O
+
+
+def attn_merge(O_parts, lse_parts):
+    """Ring attention's combination of per-key-block results ("Context
+    parallelism" page): O_parts [nparts, M, d] (each block's normalised
+    attention output), lse_parts [nparts, M] (natural log-sum-exp of each
+    block's scaled scores) -> (O [M, d], lse [M]) over all the blocks' keys."""
+    Op = np.ascontiguousarray(O_parts, dtype=np.float64)
+    Lp = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    n, M, d = Op.shape
+    O, lse = np.empty((M, d)), np.empty(M)
+    _call("oracle_attn_merge", _p(Op), _p(Lp), n, M, d, _p(O), _p(lse))
+    return O, lse
 
 
 def reduce_partials(parts, bias=None) -> np.ndarray:

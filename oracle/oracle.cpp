@@ -523,6 +523,36 @@ int joint_attn_unsharded(const double* Xi, int64_t Mi, const double* Xt, int64_t
   return kOk;
 }
 
+// ---------------------------------------------------------------------------
+// Context parallelism ("Context parallelism" page).  Ring attention: every
+// rank attends its queries to one key/value block after another as the blocks
+// travel around the ring, and the per-block results are combined.  A block b
+// gives, per query row, O_b (softmax over the block's keys applied to its
+// values) and lse_b = log sum_{j in b} exp(s_j); then
+//   O = sum_b exp(lse_b - L) O_b / sum_b exp(lse_b - L),  L = max_b lse_b,
+//   lse = L + log sum_b exp(lse_b - L),
+// which is softmax over all keys applied to all values (each O_b is its
+// block's weighted mean, exp(lse_b) its block's total weight).
+// O_parts [nparts][M][d], lse_parts [nparts][M] -> O [M][d], lse [M].
+// ---------------------------------------------------------------------------
+void attn_merge(const double* O_parts, const double* lse_parts, int nparts, int64_t M, int64_t d, double* O,
+                double* lse) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < M; ++i) {
+    double L = -INFINITY;
+    for (int b = 0; b < nparts; ++b) L = std::max(L, lse_parts[b * M + i]);
+    double wsum = 0.0;
+    for (int64_t c = 0; c < d; ++c) O[i * d + c] = 0.0;
+    for (int b = 0; b < nparts; ++b) {
+      const double w = std::exp(lse_parts[b * M + i] - L);
+      wsum += w;
+      for (int64_t c = 0; c < d; ++c) O[i * d + c] += w * O_parts[(b * M + i) * d + c];
+    }
+    for (int64_t c = 0; c < d; ++c) O[i * d + c] /= wsum;
+    if (lse) lse[i] = L + std::log(wsum);
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -579,6 +609,12 @@ int oracle_softmax_rows(const double* S, int64_t rows, int64_t cols, double* P) 
 int oracle_sdpa(const double* Q, int64_t Mq, const double* K, const double* V, int64_t Mk, int64_t d, double scale,
                 double* O, double* lse) {
   sdpa_head(Q, d, Mq, K, d, V, d, Mk, d, scale, O, d, lse);
+  return kOk;
+}
+int oracle_attn_merge(const double* O_parts, const double* lse_parts, int nparts, int64_t M, int64_t d, double* O,
+                      double* lse) {
+  if (nparts < 1) return kBadShape;
+  attn_merge(O_parts, lse_parts, nparts, M, d, O, lse);
   return kOk;
 }
 int oracle_reduce_partials(const double* parts, int T, int64_t M, int64_t N, const double* bias, double* Y) {

@@ -83,6 +83,9 @@ SIGNATURES = {
     "tp_colwise_linear_rows": (_I, [_P, _I64, _I64, _P, _P, _I64, _I, _I, _I, _P, _I64, _P]),
     "tp_shard_weights_batch": (_I, [_P, _I, _I, _P]),
     "tp_rowwise_linear_sum_rows": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I, _P, _P]),
+    "tp_sdpa_block_stats": (_I, [_P, _I64, _P, _I64, _I, _I, _P, _P, _P]),
+    "tp_attn_merge": (_I, [_P, _P, _I, _I64, _I, _I, _P, _P, _P]),
+    "tp_unshard_rowwise_all": (_I, [_P, _I64, _I64, _I, _P, _P]),
     "tp_mlp_rank_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "tp_mlp_rank_partial": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "tp_attn_rank_workspace_bytes": (_SZ, [_I64, _I64, _I, _I]),
@@ -365,6 +368,20 @@ def tp_joint_attn_run(handle, X_img, M_img, X_txt, M_txt, Y_img, Y_txt, ws, ws_b
 
 
 # --------------------------------------------------------------------------- convenience
+def tp_sdpa_block_stats(Q_qkv, Mq, KV_qkv, Mk, heads, tp_degree, O, lse, stream=None) -> int:
+    return lib().tp_sdpa_block_stats(_ptr(Q_qkv), Mq, _ptr(KV_qkv), Mk, heads, tp_degree, _ptr(O), _ptr(lse),
+                                     _stream(stream))
+
+
+def tp_attn_merge(O_parts, lse_parts, nparts, M, heads, tp_degree, O, lse_out=None, stream=None) -> int:
+    return lib().tp_attn_merge(_ptr(O_parts), _ptr(lse_parts), nparts, M, heads, tp_degree, _ptr(O), _ptr(lse_out),
+                               _stream(stream))
+
+
+def tp_unshard_rowwise_all(src, rows, cols, tp_degree, out, stream=None) -> int:
+    return lib().tp_unshard_rowwise_all(_ptr(src), rows, cols, tp_degree, _ptr(out), _stream(stream))
+
+
 def tp_mlp_rank_workspace_bytes(M, D, F, tp_degree) -> int:
     return lib().tp_mlp_rank_workspace_bytes(M, D, F, tp_degree)
 

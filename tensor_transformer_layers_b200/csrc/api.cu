@@ -255,22 +255,41 @@ tp_status run_rowwise_split(DeviceInfo* di, const uint16_t* X, int64_t M, int64_
   return launch_gemm(Aop, Bop, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
-tp_status run_sdpa(DeviceInfo* di, const uint16_t* QKV, int64_t M, int heads, int T, uint16_t* O, cudaStream_t s) {
-  if (M == 0) return TP_OK;
-  const int Hs = heads / T;
-  CUtensorMap map;
-  if (make_map_3d_f16(&map, QKV, uint64_t(3) * Hs * TP_HEAD_DIM, uint64_t(M), uint64_t(T), 64, 128) != CUDA_SUCCESS) {
+// Per-shard SDPA.  Queries: the Q columns of Qsrc [T][Mq][3*Hs*128]; keys and
+// values: the K and V columns of KVsrc [T][Mk][3*Hs*128] (the same buffer for
+// ordinary attention).  Output: bf16 O [T][Mq][Hs*128], or in the statistics
+// mode fp32 O and lse [T][Hs][Mq].
+tp_status run_sdpa_qkv(DeviceInfo* di, const uint16_t* Qsrc, int64_t Mq, const uint16_t* KVsrc, int64_t Mk, int Hs,
+                       int T, void* O, bool stats, float* lse, cudaStream_t s) {
+  if (Mq == 0 || Mk == 0) return TP_OK;
+  const uint64_t cols = uint64_t(3) * Hs * TP_HEAD_DIM;
+  AttnMaps m;
+  const CUresult om = stats ? make_map_out_f32(&m.o, O, uint64_t(Hs) * TP_HEAD_DIM, uint64_t(Mq), uint64_t(T),
+                                               uint64_t(Hs) * TP_HEAD_DIM, 0)
+                            : make_map_out_u16(&m.o, O, uint64_t(Hs) * TP_HEAD_DIM, uint64_t(Mq), uint64_t(T),
+                                               uint64_t(Hs) * TP_HEAD_DIM, 0);
+  if (make_map_3d_f16(&m.q, Qsrc, cols, uint64_t(Mq), uint64_t(T), 64, 128) != CUDA_SUCCESS ||
+      make_map_3d_f16(&m.kv, KVsrc, cols, uint64_t(Mk), uint64_t(T), 64, 128) != CUDA_SUCCESS || om != CUDA_SUCCESS) {
     note_cuda_error("attention: tensor map encode", cudaErrorInvalidValue);
     return TP_ERR_CUDA;
   }
-  AttnArgs a;
-  a.M = int(M);
+  AttnArgs a{};
+  a.Mq = int(Mq);
+  a.Mk = int(Mk);
   a.Hs = Hs;
   a.T = T;
-  a.out = O;
+  a.q_col0 = 0;
+  a.k_col0 = Hs * TP_HEAD_DIM;
+  a.v_col0 = 2 * Hs * TP_HEAD_DIM;
+  a.stats = stats ? 1 : 0;
+  a.lse = lse;
   a.scale_log2 = float(1.4426950408889634 / std::sqrt(double(TP_HEAD_DIM)));  // log2(e) / sqrt(d)
   a.err = di->err;
-  return launch_attention(map, a, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return launch_attention(m, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status run_sdpa(DeviceInfo* di, const uint16_t* QKV, int64_t M, int heads, int T, uint16_t* O, cudaStream_t s) {
+  return run_sdpa_qkv(di, QKV, M, QKV, M, heads / T, T, O, false, nullptr, s);
 }
 
 // Slices of whole weights (all T shards), used by the one-shot calls and prepare.
@@ -1219,6 +1238,54 @@ tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, 
   return joint_attn_forward(di, X_img, M_img, X_txt, M_txt, h->D, h->heads, h->T, h->w_qkv_img, h->w_qkv_txt,
                             h->w_o_img, h->w_o_txt, reinterpret_cast<uint16_t*>(w + L.qkv),
                             reinterpret_cast<uint16_t*>(w + L.o), Y_img, Y_txt, as_stream(stream));
+}
+
+// ----------------------------------------------------------------------- context parallelism pieces
+tp_status tp_sdpa_block_stats(const uint16_t* Q_qkv, int64_t Mq, const uint16_t* KV_qkv, int64_t Mk, int heads,
+                              int tp_degree, float* O, float* lse, void* stream) {
+  if (!Q_qkv || !KV_qkv || !O || !lse) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (Mq < 0 || Mk < 1 || heads < 1 || Mq >= kMaxDim || Mk >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (heads % tp_degree != 0) return TP_ERR_HEADS_INDIVISIBLE;
+  if (!al16(Q_qkv) || !al16(KV_qkv) || !al16(O) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return run_sdpa_qkv(di, Q_qkv, Mq, KV_qkv, Mk, heads / tp_degree, tp_degree, O, true, lse, as_stream(stream));
+}
+
+tp_status tp_attn_merge(const float* O_parts, const float* lse_parts, int nparts, int64_t M, int heads,
+                        int tp_degree, uint16_t* O, float* lse_out, void* stream) {
+  if (!O_parts || !lse_parts || !O) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (nparts < 1 || nparts > 64 || M < 0 || heads < 1 || M >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (heads % tp_degree != 0) return TP_ERR_HEADS_INDIVISIBLE;
+  if (!al16(O_parts) || !al16(O) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(lse_out) & 3u) != 0)
+    return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  return launch_attn_merge(O_parts, lse_parts, nparts, M, heads / tp_degree, tp_degree, O, lse_out,
+                           as_stream(stream)) == cudaSuccess
+             ? TP_OK
+             : TP_ERR_CUDA;
+}
+
+tp_status tp_unshard_rowwise_all(const uint16_t* src, int64_t rows, int64_t cols, int tp_degree, uint16_t* out,
+                                 void* stream) {
+  if (!src || !out) return TP_ERR_NULL;
+  if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
+  if (rows < 1 || cols < 1 || rows >= kMaxDim || cols >= kMaxDim) return TP_ERR_BAD_SHAPE;
+  if (cols % tp_degree != 0) return TP_ERR_INDIVISIBLE;
+  const int64_t cs = cols / tp_degree;
+  if (!al16(src) || !al16(out) || cs % 8 != 0) return TP_ERR_ALIGNMENT;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return TP_ERR_CUDA;
+  // block r of src ([rows x cs], contiguous) lands at columns [r*cs, (r+1)*cs) of out
+  return launch_slice_copy(src, out, tp_degree, rows, cs, cs, rows * cs, cs, as_stream(stream), 1, 0, 0, cols) ==
+                 cudaSuccess
+             ? TP_OK
+             : TP_ERR_CUDA;
 }
 
 // ----------------------------------------------------------------------- one rank's partial (multi-process TP)

@@ -5,7 +5,12 @@
 // and rowwise", paragraph on attention), so attention runs independently per
 // (shard, head).  For every head j of shard r:
 //     O = softmax(Q K^T / sqrt(128)) V     (non-causal, no mask)
-// computed with an online softmax over 128-key tiles.
+// computed with an online softmax over 128-key tiles.  The same kernel serves
+// the per-block step of Ring attention ("Context parallelism" page, section
+// on Ring attention): queries and keys/values may come from different token
+// sets (two tensor maps), and in the statistics mode the kernel writes O
+// normalised in fp32 with each row's log-sum-exp, which the merge over key
+// blocks needs (merge.cu).
 //
 // Structure: a work item is (shard, head, 256 query rows) = two 128-row query
 // tiles t = 0, 1.  The kernel is persistent: one CTA per SM walks the items
@@ -112,8 +117,8 @@ __device__ __forceinline__ AttnItem attn_item(int i, int q_blocks, int Hs) {
 // 320 threads: ten warps, so some SM sub-partitions (16K registers each) hold
 // three of them, which caps a thread at 168 registers.
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap qkv, const __grid_constant__ CUtensorMap omap,
-                   const AttnArgs p) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
+                   const __grid_constant__ CUtensorMap omap, const AttnArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarOff);
@@ -130,8 +135,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_kv = (p.M + kBKV - 1) / kBKV;
-  const int q_blocks = (p.M + kTiles * kBQ - 1) / (kTiles * kBQ);
+  const int n_kv = (p.Mk + kBKV - 1) / kBKV;
+  const int q_blocks = (p.Mq + kTiles * kBQ - 1) / (kTiles * kBQ);
   const int n_items = q_blocks * p.T * p.Hs;
   // this CTA's items: blockIdx.x, blockIdx.x + gridDim.x, ...
   const int my_items = blockIdx.x < n_items ? (n_items - 1 - int(blockIdx.x)) / int(gridDim.x) + 1 : 0;
@@ -162,15 +167,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&qkv);
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kvmap);
       bool ok = true;
       int g = 0;           // K/V blocks issued (ring position)
       int qn[2] = {0, 0};  // Q tiles issued per tile slot
       for (int k = 0; k < my_items && ok; ++k) {
         const AttnItem it = attn_item(int(blockIdx.x) + k * int(gridDim.x), q_blocks, p.Hs);
-        const int qcol = it.head * kD;
-        const int kcol = (p.Hs + it.head) * kD;
-        const int vcol = (2 * p.Hs + it.head) * kD;
+        const int qcol = p.q_col0 + it.head * kD;
+        const int kcol = p.k_col0 + it.head * kD;
+        const int vcol = p.v_col0 + it.head * kD;
         // K/V block 0 first (its ring stage frees early), then Q_0 and Q_1 (each
         // free once the previous item's last S_t is done), then the other blocks.
         for (int j = 0; j < n_kv && ok; ++j, ++g) {
@@ -181,10 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* sk = smem + kKVOff + st * kKVBytes;
           mbar_arrive_expect_tx(&kv_full[st], kKVBytes);
-          tma_load_3d(sk, &qkv, &kv_full[st], kcol, j * kBKV, it.shard);
-          tma_load_3d(sk + kBox, &qkv, &kv_full[st], kcol + 64, j * kBKV, it.shard);
-          tma_load_3d(sk + 2 * kBox, &qkv, &kv_full[st], vcol, j * kBKV, it.shard);
-          tma_load_3d(sk + 3 * kBox, &qkv, &kv_full[st], vcol + 64, j * kBKV, it.shard);
+          tma_load_3d(sk, &kvmap, &kv_full[st], kcol, j * kBKV, it.shard);
+          tma_load_3d(sk + kBox, &kvmap, &kv_full[st], kcol + 64, j * kBKV, it.shard);
+          tma_load_3d(sk + 2 * kBox, &kvmap, &kv_full[st], vcol, j * kBKV, it.shard);
+          tma_load_3d(sk + 3 * kBox, &kvmap, &kv_full[st], vcol + 64, j * kBKV, it.shard);
           if (j == 0) {
             for (int t = 0; t < kTiles; ++t) {
               if (!mbar_wait(&q_empty[t], (k & 1) ^ 1u, abort_flag)) {
@@ -194,8 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint8_t* sq = smem + kQOff + t * kQBytes;
               const int row = it.qb * (kTiles * kBQ) + t * kBQ;
               mbar_arrive_expect_tx(&q_full[t], kQBytes);
-              tma_load_3d(sq, &qkv, &q_full[t], qcol, row, it.shard);
-              tma_load_3d(sq + kBox, &qkv, &q_full[t], qcol + 64, row, it.shard);
+              tma_load_3d(sq, &qmap, &q_full[t], qcol, row, it.shard);
+              tma_load_3d(sq + kBox, &qmap, &q_full[t], qcol + 64, row, it.shard);
               ++qn[t];
             }
           }
@@ -356,10 +362,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
         }
         const int kv0 = j * kBKV;
-        if (kv0 + kBKV > p.M) {  // ragged last key tile: keys >= M do not exist
+        if (kv0 + kBKV > p.Mk) {  // ragged last key tile: keys >= Mk do not exist
 #pragma unroll
           for (int i = 0; i < kBKV; ++i)
-            if (kv0 + i >= p.M) s[i] = -INFINITY;
+            if (kv0 + i >= p.Mk) s[i] = -INFINITY;
         }
         // Row max: 3-input max over four independent chains (64 instructions
         // for 128 scores, a short dependency chain).  The element-wise code
@@ -428,48 +434,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[t]);
       }
-      // Epilogue of this item: O_t / l in bf16.  It reads O_t before this warp's
-      // next p_full arrival, and the next item's first P.V (which overwrites
-      // O_t) waits for that arrival.
+      // Epilogue of this item: O_t / l.  It reads O_t before this warp's next
+      // p_full arrival, and the next item's first P.V (which overwrites O_t)
+      // waits for that arrival.
       if (ok) ok = mbar_wait(&o_done[t], k & 1, abort_flag);
       if (ok) {
-        // O_t / l in bf16, 64 columns at a time: staged in this warp's box in
-        // the 128-byte swizzle of the output map, then one TMA store (whole
-        // 128-byte lines; rows >= M are clipped, a box wholly below M skipped).
         tc_fence_after();
         const AttnItem it = attn_item(int(blockIdx.x) + k * int(gridDim.x), q_blocks, p.Hs);
         const int row0 = it.qb * (kTiles * kBQ) + t * kBQ + (warp & 3) * 32;
         const float inv_l = 1.0f / l_run;
         const uint64_t inv_l2 = f32x2(inv_l, inv_l);
         uint8_t* stg = smem + kOutOff + warp * kOutBuf;
+        if (!p.stats) {
+          // O_t / l in bf16, 64 columns at a time: staged in this warp's box
+          // in the 128-byte swizzle of the output map, then one TMA store
+          // (whole 128-byte lines; rows >= Mq are clipped, a box wholly below
+          // Mq skipped).
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          if (lane == 0) bulk_wait_read_0();  // the previous store has read the box
-          __syncwarp();
+          for (int half = 0; half < 2; ++half) {
+            if (lane == 0) bulk_wait_read_0();  // the previous store has read the box
+            __syncwarp();
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 2; ++c) {
+              uint32_t r[32];
+              tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(half * 64 + c * 32), r);
+              uint32_t w[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                float lo, hi;
+                f32x2_split(mul_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv_l2), lo,
+                            hi);
+                w[i] = pack_bf16x2(lo, hi);
+              }
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int chunk = c * 4 + q;  // 16-byte chunk of this lane's 128-byte row
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                    make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && row0 < p.Mq) {
+              tma_store_3d(&omap, stg, it.head * kD + half * 64, row0, it.shard);
+              bulk_commit();
+            }
+          }
+        } else {
+          // Statistics mode: O_t / l in fp32 (32-column boxes of 128-byte
+          // rows) and each row's log-sum-exp of the scaled scores in log2
+          // units, m + log2(l).
+#pragma unroll 1
+          for (int c = 0; c < kD / 32; ++c) {
+            if (lane == 0) bulk_wait_read_0();
+            __syncwarp();
             uint32_t r[32];
-            tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(half * 64 + c * 32), r);
-            uint32_t w[16];
+            tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(c * 32), r);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               float lo, hi;
               f32x2_split(mul_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv_l2), lo, hi);
-              w[i] = pack_bf16x2(lo, hi);
+              r[2 * i] = __float_as_uint(lo);
+              r[2 * i + 1] = __float_as_uint(hi);
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int chunk = c * 4 + q;  // 16-byte chunk of this lane's 128-byte row
-              *reinterpret_cast<uint4*>(stg + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
-                  make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                  make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && row0 < p.Mq) {
+              tma_store_3d(&omap, stg, it.head * kD + c * 32, row0, it.shard);
+              bulk_commit();
             }
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0 && row0 < p.M) {
-            tma_store_3d(&omap, stg, it.head * kD + half * 64, row0, it.shard);
-            bulk_commit();
-          }
+          if (row0 + lane < p.Mq)
+            p.lse[(int64_t(it.shard) * p.Hs + it.head) * p.Mq + row0 + lane] = m_run + log2f(l_run);
         }
         tc_fence_before();
       }
@@ -489,27 +529,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s) {
-  if (a.M <= 0) return cudaSuccess;
-  int dev = 0, num_sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess && num_sms <= 0) e = cudaErrorInvalidValue;
-  if (e != cudaSuccess) return note_cuda_error("attention: SM count", e);
+cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& a, int num_sms, cudaStream_t s) {
+  if (a.Mq <= 0 || a.Mk <= 0) return cudaSuccess;
   // Persistent: one CTA per SM (at most one per work item), each walking the
   // items blockIdx.x, blockIdx.x + gridDim.x, ... so that one item's last
   // blocks and output overlap the next item's Q/K/V loads and first S.
-  const int q_blocks = (a.M + kTiles * kBQ - 1) / (kTiles * kBQ);
+  const int q_blocks = (a.Mq + kTiles * kBQ - 1) / (kTiles * kBQ);
   const int64_t n_items = int64_t(q_blocks) * a.T * a.Hs;
   const int64_t grid = n_items < num_sms ? n_items : num_sms;
-  // O [T][M][Hs*128] bf16, written in 64-column x 32-row boxes
-  CUtensorMap omap;
-  if (make_map_out_u16(&omap, a.out, uint64_t(a.Hs) * kD, uint64_t(a.M), uint64_t(a.T), uint64_t(a.Hs) * kD, 0) !=
-      CUDA_SUCCESS)
-    return note_cuda_error("attention: output tensor map encode", cudaErrorInvalidValue);
-  e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return note_cuda_error("attention: set shared memory size", e);
-  attn_tc_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(qkv_map, omap, a);
+  attn_tc_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(maps.q, maps.kv, maps.o, a);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) {

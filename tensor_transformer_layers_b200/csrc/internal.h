@@ -88,18 +88,35 @@ struct GemmOperand {
 cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms, cudaStream_t s);
 
 // ----------------------------------------------------------------------------
-// a6: per-shard SDPA.  qkv map: 3-D fp16 {3*Hs*128, M, T}, box {64, 128, 1}.
+// a6: per-shard SDPA (attn.cu).  Queries come from the Q columns of one fp16
+// buffer [T][Mq][*], keys and values from the K and V columns of another (or
+// the same) buffer [T][Mk][*]; head h of a shard uses columns q_col0 + 128 h,
+// k_col0 + 128 h and v_col0 + 128 h.  Maps (fp16, 3-D {columns, rows, T},
+// box 64 x 128, 128-byte swizzle): q over the query buffer, kv over the key /
+// value buffer; o: the output map over [T][Mq][Hs*128] (bf16 box 64 x 32, or
+// fp32 box 32 x 32 in the statistics mode).
 // ----------------------------------------------------------------------------
+struct AttnMaps {
+  CUtensorMap q, kv, o;
+};
 struct AttnArgs {
-  int M;            // tokens
-  int Hs;           // heads per shard
-  int T;            // shards
-  uint16_t* out;    // [T x M x Hs*128]
-  float scale_log2; // log2(e)/sqrt(128)
+  int Mq, Mk;        // query rows, key rows
+  int Hs, T;         // heads per shard, shards
+  int q_col0, k_col0, v_col0;
+  int stats;         // 0: O / l in bf16; 1: O / l in fp32 and lse
+  float* lse;        // statistics mode: [T][Hs][Mq] fp32, log2 units (m + log2 l of the scaled scores)
+  float scale_log2;  // log2(e)/sqrt(128)
   int* err;
 };
+cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& a, int num_sms, cudaStream_t s);
 
-cudaError_t launch_attention(const CUtensorMap& qkv_map, const AttnArgs& a, cudaStream_t s);
+// Merge of per-key-block attention results (Ring attention): for every
+// (shard, row, head), O = sum_b 2^(lse_b - L) O_b / sum_b 2^(lse_b - L) with
+// L = max_b lse_b, written in bf16; lse_out (optional) = L + log2 sum_b
+// 2^(lse_b - L).  O_parts [nparts][T][M][Hs*128] fp32, lse_parts
+// [nparts][T][Hs][M] fp32 (log2 units), O [T][M][Hs*128] bf16.
+cudaError_t launch_attn_merge(const float* O_parts, const float* lse_parts, int nparts, int64_t M, int Hs, int T,
+                              uint16_t* O, float* lse_out, cudaStream_t s);
 
 // One CTA whose bounded wait on an mbarrier that nothing arrives on must run
 // out after limit_ns and set kErrTimeout in *err (watchdog.cu).

@@ -1,0 +1,73 @@
+// merge.cu - combines per-key-block attention results (Ring attention,
+// Diffusers "Context parallelism" page, section on Ring attention: each rank
+// attends its queries to the key/value block it holds while the blocks travel
+// around the ring, and the partial results are combined).
+//
+// Block b gives, for one (shard, query row, head), O_b = softmax over its
+// keys applied to its values (normalised, fp32) and lse_b = log2 of the sum of
+// 2^(scaled score) over its keys.  Over all blocks,
+//   O = sum_b 2^(lse_b - L) O_b / sum_b 2^(lse_b - L),   L = max_b lse_b,
+// which is exactly softmax over all keys applied to all values (each O_b is
+// its block's weighted mean; 2^(lse_b) is its block's total weight).
+// HBM-bound: a thread owns 8 consecutive columns of one row and head (two
+// 16-byte fp32 loads per block, one 16-byte bf16 store).
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace tp {
+namespace {
+
+constexpr int kThreads = 256;
+
+__global__ void __launch_bounds__(kThreads)
+    attn_merge_kernel(const float4* __restrict__ O_parts, const float* __restrict__ lse_parts, int nparts, int64_t M,
+                      int Hs, int64_t n8_total, uint4* __restrict__ O, float* __restrict__ lse_out) {
+  const int64_t stride = int64_t(gridDim.x) * kThreads;
+  const int64_t part_stride4 = n8_total * 2;             // float4s per block's O
+  const int64_t lse_stride = n8_total / 16;              // T * Hs * M values per block
+  const int64_t row_groups = int64_t(Hs) * 16;           // 8-column groups per row
+  for (int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x; i < n8_total; i += stride) {
+    const int64_t tr = i / row_groups;                   // t * M + row
+    const int c8 = int(i - tr * row_groups);
+    const int head = c8 >> 4;
+    const int64_t t = tr / M, row = tr - t * M;
+    const int64_t li = (t * Hs + head) * M + row;
+    float L = -INFINITY;
+    for (int b = 0; b < nparts; ++b) L = fmaxf(L, lse_parts[b * lse_stride + li]);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float wsum = 0.f;
+    for (int b = 0; b < nparts; ++b) {
+      const float w = exp2f(lse_parts[b * lse_stride + li] - L);
+      const float4 lo = __ldcs(O_parts + b * part_stride4 + 2 * i);
+      const float4 hi = __ldcs(O_parts + b * part_stride4 + 2 * i + 1);
+      wsum += w;
+      acc[0] += w * lo.x; acc[1] += w * lo.y; acc[2] += w * lo.z; acc[3] += w * lo.w;
+      acc[4] += w * hi.x; acc[5] += w * hi.y; acc[6] += w * hi.z; acc[7] += w * hi.w;
+    }
+    const float inv = 1.0f / wsum;
+    uint4 o;
+    o.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+    o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+    __stcs(O + i, o);
+    if (lse_out != nullptr && (c8 & 15) == 0) lse_out[li] = L + log2f(wsum);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_merge(const float* O_parts, const float* lse_parts, int nparts, int64_t M, int Hs, int T,
+                              uint16_t* O, float* lse_out, cudaStream_t s) {
+  const int64_t n8_total = int64_t(T) * M * Hs * 16;
+  if (n8_total == 0) return cudaSuccess;
+  int64_t blocks = (n8_total + kThreads - 1) / kThreads;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  attn_merge_kernel<<<unsigned(blocks), kThreads, 0, s>>>(reinterpret_cast<const float4*>(O_parts), lse_parts,
+                                                          nparts, M, Hs, n8_total, reinterpret_cast<uint4*>(O),
+                                                          lse_out);
+  count_launch();
+  return note_cuda_error("attention merge: launch", cudaGetLastError());
+}
+
+}  // namespace tp

@@ -38,6 +38,47 @@ def allreduce_layer(partial, finish, group=None):
     return finish(part)
 
 
+def ulysses_attention(qkv_local, pack, attend, unpack, group=None):
+    """Ulysses attention ("Context parallelism" page): U ranks each hold M/U
+    tokens with every head.  ``pack`` groups this rank's [Q | K | V] columns by
+    destination head group ([U, M/U, ...], e.g. tp_shard_packed_all with
+    TP_ROWWISE and blocks [1, 1, 1]); one all-to-all gives every rank all M
+    tokens of its H/U heads (rank order = token order); ``attend`` runs the
+    attention on them ([M, (H/U)*d] out, viewed as [U, M/U, ...]); the
+    reverse all-to-all returns each rank its tokens' rows of every head group,
+    which ``unpack`` puts back in head order (tp_unshard_rowwise_all)."""
+    import torch.distributed as dist
+    send = pack(qkv_local)
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    out = attend(recv)
+    back = torch.empty_like(out)
+    dist.all_to_all_single(back, out, group=group)
+    return unpack(back)
+
+
+def ring_attention(q_local, kv_local, attend_block, merge, group=None):
+    """Ring attention ("Context parallelism" page): R ranks each hold a block
+    of tokens.  R steps: attend this rank's queries to the key/value block it
+    currently holds (``attend_block`` -> (O_b, lse_b), e.g.
+    tp_sdpa_block_stats), then pass the block on to the next rank and take the
+    previous rank's.  ``merge`` combines the R results (tp_attn_merge); their
+    order differs between ranks and does not change the result."""
+    import torch.distributed as dist
+    R, rank = dist.get_world_size(group), dist.get_rank(group)
+    parts = []
+    kv = kv_local
+    for step in range(R):
+        parts.append(attend_block(q_local, kv))
+        if step + 1 < R:
+            nxt = torch.empty_like(kv)
+            ops = [dist.P2POp(dist.isend, kv, (rank + 1) % R, group), dist.P2POp(dist.irecv, nxt, (rank - 1) % R, group)]
+            for req in dist.batch_isend_irecv(ops):
+                req.wait()
+            kv = nxt
+    return merge(parts)
+
+
 class MlpRank:
     """Rank ``rank`` of a ``tp_degree``-way MLP pair: cuts its own shards from
     the full weights once (as sharded loading would), then runs its partial."""

@@ -121,3 +121,99 @@ def test_single_process_needs_no_collective():
     from tensor_transformer_layers_b200.dist import allreduce_layer
     t = torch.arange(4.0)
     assert torch.equal(allreduce_layer(lambda: t.clone(), lambda s: s * 2), t * 2)
+
+
+# ---------------------------------------------------------------------------
+# Context parallelism across processes: Ulysses all-to-all regrouping and the
+# Ring rotation of key/value blocks, two gloo ranks, oracle compute.
+# ---------------------------------------------------------------------------
+
+def _cp_inputs():
+    rng = np.random.default_rng(11)
+    M, H, d = 8, 4, 16
+    return rng.standard_normal((M, 3 * H * d)), H, d
+
+
+def _attend(qkv, n_heads, d):
+    import oracle as o
+    c = n_heads * d
+    return np.concatenate([o.sdpa(qkv[:, h * d:(h + 1) * d], qkv[:, c + h * d:c + (h + 1) * d],
+                                  qkv[:, 2 * c + h * d:2 * c + (h + 1) * d]) for h in range(n_heads)], axis=1)
+
+
+def _cp_rank_main(rank, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(WORLD))
+    import datetime
+
+    import torch.distributed as dist
+
+    import oracle as o
+    from tensor_transformer_layers_b200.dist import ring_attention, ulysses_attention
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD, timeout=datetime.timedelta(seconds=60))
+    try:
+        QKV, H, d = _cp_inputs()
+        U, M = WORLD, QKV.shape[0]
+        Ms = M // U
+        local = torch.from_numpy(QKV[rank * Ms:(rank + 1) * Ms].copy())
+
+        def pack(x):  # by destination head group: packed rowwise, blocks [1, 1, 1]
+            return torch.from_numpy(np.stack([o.slice_packed_rowwise(x.numpy(), [1, 1, 1], U, u) for u in range(U)]))
+
+        def attend(recv):  # [U, Ms, ...] = all tokens, this rank's heads
+            return torch.from_numpy(_attend(recv.reshape(M, -1).numpy(), H // U, d).reshape(U, Ms, -1))
+
+        def unpack(back):  # [U, Ms, (H/U) d] -> [Ms, H d]
+            return torch.cat([back[u] for u in range(U)], dim=1)
+
+        Yu = ulysses_attention(local, pack, attend, unpack)
+
+        def attend_block(q_rows, kv_rows):  # per head: normalised O and natural log-sum-exp
+            q, kv = q_rows.numpy(), kv_rows.numpy()
+            c = H * d
+            res = [o.sdpa(q[:, h * d:(h + 1) * d], kv[:, c + h * d:c + (h + 1) * d],
+                          kv[:, 2 * c + h * d:2 * c + (h + 1) * d], return_lse=True) for h in range(H)]
+            return [r[0] for r in res], [r[1] for r in res]
+
+        def merge(parts):
+            outs = []
+            for h in range(H):
+                Oh, _ = o.attn_merge(np.stack([p[0][h] for p in parts]), np.stack([p[1][h] for p in parts]))
+                outs.append(Oh)
+            return np.concatenate(outs, axis=1)
+
+        Yr = ring_attention(local, local, attend_block, merge)
+        np.save(os.path.join(out_dir, f"ulysses{rank}.npy"), Yu.numpy())
+        np.save(os.path.join(out_dir, f"ring{rank}.npy"), Yr)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.fixture(scope="module")
+def cp_ranks(tmp_path_factory):
+    out = tmp_path_factory.mktemp("cp_ranks")
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_rank_main, args=(r, port, str(out))) for r in range(WORLD)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    return out
+
+
+def test_ulysses_ranks_get_their_tokens_of_the_full_attention(cp_ranks):
+    QKV, H, d = _cp_inputs()
+    full = _attend(QKV, H, d)
+    Ms = QKV.shape[0] // WORLD
+    for r in range(WORLD):
+        assert np.array_equal(np.load(cp_ranks / f"ulysses{r}.npy"), full[r * Ms:(r + 1) * Ms])
+
+
+def test_ring_ranks_get_their_tokens_of_the_full_attention(cp_ranks):
+    QKV, H, d = _cp_inputs()
+    full = _attend(QKV, H, d)
+    Ms = QKV.shape[0] // WORLD
+    for r in range(WORLD):
+        got = np.load(cp_ranks / f"ring{r}.npy")
+        assert np.max(np.abs(got - full[r * Ms:(r + 1) * Ms])) <= 1e-12

@@ -30,9 +30,9 @@ def test_sdpa_step(M, Hs, T):
             assert_rounded_once(g[r][:, j * 128:(j + 1) * 128], o.sdpa(Q, K, V), f"sdpa r={r} j={j}")
 
 
-# More work items (shard, head, 256 query rows) than SMs: the persistent kernel
-# walks several items per CTA (149 items: one CTA takes two; 400 items with
-# ragged query and key blocks; 300 items of two whole query blocks each).
+# More work items (shard, head, 512 query rows) than CTA pairs: the persistent
+# kernel walks several items per pair (149 items over 74 pairs; 200 items with
+# ragged query and key blocks; 150 items of one whole query block each).
 @pytest.mark.parametrize("M,Hs,T", [(256, 149, 1), (333, 100, 2), (512, 150, 1)])
 def test_sdpa_several_items_per_cta(M, Hs, T):
     test_sdpa_step(M, Hs, T)

@@ -608,3 +608,64 @@ def test_joint_sharded_equals_unsharded_and_rows(T):
     assert np.allclose(Ri, Yi[[0, 5]], rtol=1e-12, atol=1e-12) and np.allclose(Rt, Yt[[2]], rtol=1e-12, atol=1e-12)
     with pytest.raises(ValueError):
         o.joint_attn_sharded_summed(Xi, Xt, Wqi, Wqt, Woi, Wot, 2, 4)  # 4 does not divide 2 heads
+
+
+# ---------------------------------------------------------------------------
+# Context parallelism ("Context parallelism" page): Ring attention's merge of
+# per-key-block results and Ulysses attention's head regrouping.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("splits", [[7], [3, 4], [1, 2, 4], [2, 2, 2, 1]])
+def test_ring_merge_of_key_blocks_is_attention_over_all_keys(splits):
+    rng = _rng(60 + len(splits))
+    Mq, d = 5, 16
+    Mk = sum(splits)
+    Q, K, V = rng.standard_normal((Mq, d)), rng.standard_normal((Mk, d)), rng.standard_normal((Mk, d))
+    full, lse_full = o.sdpa(Q, K, V, return_lse=True)
+    parts, lses, j = [], [], 0
+    for n in splits:
+        Ob, lb = o.sdpa(Q, K[j:j + n], V[j:j + n], scale=1 / np.sqrt(d), return_lse=True)
+        parts.append(Ob)
+        lses.append(lb)
+        j += n
+    O, lse = o.attn_merge(np.stack(parts), np.stack(lses))
+    assert np.max(np.abs(O - full)) <= 1e-12 and np.max(np.abs(lse - lse_full)) <= 1e-12
+    # the merge does not depend on the order the blocks arrive in (ranks see them rotated)
+    O2, _ = o.attn_merge(np.stack(parts[::-1]), np.stack(lses[::-1]))
+    assert np.max(np.abs(O2 - full)) <= 1e-12
+
+
+def test_lse_closed_form():
+    # one key per block: lse = s * scale; equal scores: lse = log(Mk) + s
+    Q = np.array([[1.0, 2.0]])
+    K = np.array([[3.0, -1.0], [3.0, -1.0], [3.0, -1.0]])
+    V = np.eye(3, 2)
+    _, lse = o.sdpa(Q, K, V, scale=0.5, return_lse=True)
+    assert abs(lse[0] - (np.log(3.0) + 0.5 * 1.0)) <= 1e-14
+    # a block with much smaller weight barely moves the merge
+    O, _ = o.attn_merge(np.array([[[1.0, 0.0]], [[0.0, 1.0]]]), np.array([[0.0], [np.log(3.0)]]))
+    assert np.allclose(O, [[0.25, 0.75]], atol=1e-15)
+
+
+def test_ulysses_regrouping_is_attention_over_all_tokens():
+    # U ranks hold M/U tokens with all H heads; packing each rank's [Q|K|V] by
+    # destination head group (packed rowwise, blocks [1, 1, 1]), exchanging
+    # (all-to-all), attending all tokens x H/U heads and regrouping back must
+    # give the full attention -- exactly, since every head sees the same data.
+    rng = _rng(70)
+    U, H, d, M = 2, 4, 8, 6
+    QKV = rng.standard_normal((M, 3 * H * d))
+    def attend(qkv, n_heads):
+        c = n_heads * d
+        return np.concatenate([o.sdpa(qkv[:, h * d:(h + 1) * d], qkv[:, c + h * d:c + (h + 1) * d],
+                                      qkv[:, 2 * c + h * d:2 * c + (h + 1) * d]) for h in range(n_heads)], axis=1)
+    full = attend(QKV, H)
+    Ms = M // U
+    send = [[o.slice_packed_rowwise(QKV[s * Ms:(s + 1) * Ms], [1, 1, 1], U, u) for u in range(U)] for s in range(U)]
+    out_blocks = []
+    for u in range(U):  # rank u receives every rank's tokens for head group u, in rank (= token) order
+        O_u = attend(np.concatenate([send[s][u] for s in range(U)]), H // U)
+        out_blocks.append(O_u)
+    got = np.concatenate([np.concatenate([out_blocks[u][s * Ms:(s + 1) * Ms] for u in range(U)], axis=1)
+                          for s in range(U)])
+    assert np.array_equal(got, full)
