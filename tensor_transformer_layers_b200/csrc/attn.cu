@@ -82,6 +82,7 @@ constexpr int kQBytes = 2 * kBox;   // one Q tile: d in two 64-column boxes
 constexpr int kKVBytes = 4 * kBox;  // K tile (2 boxes) + V tile (2 boxes)
 constexpr int kStages = 2;
 constexpr int kThreads = 320;
+
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kQOff = 0;
@@ -116,6 +117,9 @@ __device__ __forceinline__ AttnItem attn_item(int i, int q_blocks, int Hs) {
 
 // 320 threads: ten warps, so some SM sub-partitions (16K registers each) hold
 // three of them, which caps a thread at 168 registers.
+// kStats: the statistics mode (fp32 O and log-sum-exp) is a separate
+// instantiation, so the ordinary kernel carries none of its code.
+template <bool kStats>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
                    const __grid_constant__ CUtensorMap omap, const AttnArgs p) {
@@ -445,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv_l = 1.0f / l_run;
         const uint64_t inv_l2 = f32x2(inv_l, inv_l);
         uint8_t* stg = smem + kOutOff + warp * kOutBuf;
-        if (!p.stats) {
+        if constexpr (!kStats) {
           // O_t / l in bf16, 64 columns at a time: staged in this warp's box
           // in the 128-byte swizzle of the output map, then one TMA store
           // (whole 128-byte lines; rows >= Mq are clipped, a box wholly below
@@ -537,15 +541,16 @@ cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& a, int num_sm
   const int q_blocks = (a.Mq + kTiles * kBQ - 1) / (kTiles * kBQ);
   const int64_t n_items = int64_t(q_blocks) * a.T * a.Hs;
   const int64_t grid = n_items < num_sms ? n_items : num_sms;
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  const auto kernel = a.stats ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return note_cuda_error("attention: set shared memory size", e);
-  attn_tc_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(maps.q, maps.kv, maps.o, a);
+  kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(maps.q, maps.kv, maps.o, a);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     cudaFuncAttributes fa{};
     char detail[160];
-    if (cudaFuncGetAttributes(&fa, attn_tc_kernel) == cudaSuccess)
+    if (cudaFuncGetAttributes(&fa, kernel) == cudaSuccess)
       snprintf(detail, sizeof(detail), "kernel: %d registers/thread, max %d threads/block, %zu B static smem",
                fa.numRegs, fa.maxThreadsPerBlock, fa.sharedSizeBytes);
     else

@@ -370,47 +370,6 @@ __device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, u
       : "memory");
 }
 
-// Pair MMA with A read from tensor memory (each CTA's TMEM supplies its half
-// of A's rows; B from both CTAs' shared memory, N/2 columns each).
-__device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Waits like mbar_wait_for, but with cluster-scope acquire: for barriers that
-// threads of the other CTA of a pair arrive on (their prior writes, e.g. to
-// their own tensor memory, are then visible to this thread).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar_addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const volatile int* abort) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_cluster(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-#pragma unroll 1
-  for (uint32_t round = 0; round < kWaitMaxRounds; ++round) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait_cluster(a, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-  }
-  return false;
-}
-
 // Arrive once on `bar` (same shared offset) in every CTA of `cta_mask` when all
 // pair MMAs issued so far by this thread complete.
 __device__ __forceinline__ void umma_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
@@ -419,21 +378,6 @@ __device__ __forceinline__ void umma_commit_pair_mc(uint64_t* bar, uint16_t cta_
           smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
-}
-
-// ----------------------------------------------------------------------------
-// Register reallocation between warpgroups (all four warps of a warpgroup
-// execute it together).  inc waits until the pool the CTA was launched with
-// has the registers, so the warpgroups' shares must add up to at most the
-// launch's threads x registers per thread.
-// ----------------------------------------------------------------------------
-template <int N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ----------------------------------------------------------------------------
