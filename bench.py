@@ -282,8 +282,8 @@ class MlpWorkload:
         import torch
         c = self.cfg
         self._pair = tp.MlpPair(g["W_up"], g["b_up"], g["W_down"], g["b_down"], c["T"])
-        self._yp = torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev)
-        return ["X"], lambda gi: self._pair(gi["X"], Y=self._yp), (
+        self._yp = [torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev) for _ in range(2)]
+        return ["X"], lambda gi, b: self._pair(gi["X"], Y=self._yp[b]), (
             "MlpPair: tp_mlp_prepare once, tp_mlp_run every step with X copied from pinned host memory and Y "
             "copied back")
 
@@ -358,8 +358,9 @@ class SweepWorkload(MlpWorkload):
         import torch
         c = self.cfg
         self._pairs = [tp.MlpPair(g["W_up"], g["b_up"], g["W_down"], g["b_down"], T) for T in self.degrees]
-        self._yp = [torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev) for _ in self.degrees]
-        return ["X"], lambda gi: tuple(p(gi["X"], Y=y) for p, y in zip(self._pairs, self._yp)), (
+        self._yp = [[torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev) for _ in self.degrees]
+                    for _ in range(2)]
+        return ["X"], lambda gi, b: tuple(p(gi["X"], Y=y) for p, y in zip(self._pairs, self._yp[b])), (
             "MlpPair at tp_degree 1, 2, 4 and 8 (prepared once), each run every step on X copied from pinned host "
             "memory, all four Y copied back")
 
@@ -453,8 +454,8 @@ class AttnWorkload(MlpWorkload):
         import torch
         c = self.cfg
         self._blk = tp.AttnBlock(g["W_qkv"], g["W_o"], c["H"], c["T"])
-        self._yp = torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev)
-        return ["X"], lambda gi: self._blk(gi["X"], Y=self._yp), (
+        self._yp = [torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev) for _ in range(2)]
+        return ["X"], lambda gi, b: self._blk(gi["X"], Y=self._yp[b]), (
             "AttnBlock: tp_attn_prepare once, tp_attn_run every step with X copied from pinned host memory and Y "
             "copied back")
 
@@ -564,7 +565,7 @@ class JointAttnWorkload(AttnWorkload):
     def prepared(self, tp, g, dev):
         c = self.cfg
         self._blk = tp.JointAttnBlock(g["W_qkv_img"], g["W_qkv_txt"], g["W_o_img"], g["W_o_txt"], c["H"], c["T"])
-        return ["X_img", "X_txt"], lambda gi: self._blk(gi["X_img"], gi["X_txt"]), (
+        return ["X_img", "X_txt"], lambda gi, b: self._blk(gi["X_img"], gi["X_txt"]), (
             "JointAttnBlock: tp_joint_attn_prepare once, tp_joint_attn_run every step with both streams' X copied "
             "from pinned host memory and Y_img, Y_txt copied back")
 
@@ -780,8 +781,8 @@ class BlockWorkload(AttnWorkload):
         self._blk = tp.AttnBlock(g["W_qkv"], g["W_o"], c["H"], c["T"])
         self._pair = tp.MlpPair(g["W_up"], g["b_up"], g["W_down"], g["b_down"], c["T"])
         self._ap = torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev)
-        self._yp = torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev)
-        return ["X"], lambda gi: self._pair(self._blk(gi["X"], Y=self._ap), Y=self._yp), (
+        self._yp = [torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev) for _ in range(2)]
+        return ["X"], lambda gi, b: self._pair(self._blk(gi["X"], Y=self._ap), Y=self._yp[b]), (
             "AttnBlock then MlpPair (prepared once), run every step on X copied from pinned host memory, Y copied "
             "back")
 
@@ -929,8 +930,8 @@ class SwigluWorkload(MlpWorkload):
         import torch
         c = self.cfg
         self._pair = tp.MlpPair(g["W_in"], g["b_in"], g["W_out"], g["b_out"], c["T"], activation="swiglu")
-        self._yp = torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev)
-        return ["X"], lambda gi: self._pair(gi["X"], Y=self._yp), (
+        self._yp = [torch.empty((c["M"], c["D"]), dtype=torch.int16, device=dev) for _ in range(2)]
+        return ["X"], lambda gi, b: self._pair(gi["X"], Y=self._yp[b]), (
             "MlpPair(activation='swiglu'): tp_swiglu_prepare once, tp_mlp_run every step with X copied from "
             "pinned host memory and Y copied back")
 
@@ -1041,13 +1042,23 @@ def _scale(unit):
 
 
 # --------------------------------------------------------------------------- CPU oracle legs
-def cpu_baseline(wl, d, budget_s: float = 12.0):
+def _rows_for(wl, d, seconds: float) -> int:
+    """Token rows of the workload the oracle processes in about `seconds`: the
+    per-row cost and the fixed cost (slicing, K/V of every token) from two
+    probe sizes."""
+    M = wl.cfg["M"]
+    wl.oracle_run(d, 8)  # warm
+    t1, _ = wl.oracle_run(d, 16)
+    t2, _ = wl.oracle_run(d, 64)
+    per_row = max((t2 - t1) / 48.0, 1e-7)
+    fixed = max(t1 - 16 * per_row, 0.0)
+    return int(min(M, max(16, (seconds - fixed) / per_row)))
+
+
+def cpu_baseline(wl, d, budget_s: float = 15.0):
     """The oracle as it stands, on a bounded sample of the workload's token rows."""
     M = wl.cfg["M"]
-    probe = 16
-    wl.oracle_run(d, probe)  # warm
-    t, _ = wl.oracle_run(d, probe)
-    rows = int(min(M, max(probe, probe * budget_s / max(t, 1e-6))))
+    rows = _rows_for(wl, d, budget_s)
     if wl.key in ("flux_attn", "wide_block", "flux_joint_attn"):
         rows = min(rows, 256)  # the K/V projection of every token dominates; more rows add little
     t, done = wl.oracle_run(d, rows)
@@ -1061,11 +1072,8 @@ def run_reference(args, wl, rank, world):
         return None  # rank 0 alone runs the CPU reference
     d = wl.host_inputs(0)
     M = wl.cfg["M"]
-    probe = 16
-    wl.oracle_run(d, probe)
-    t, _ = wl.oracle_run(d, probe)
     per_step = max(0.2, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
-    rows = int(min(M, max(8, probe * per_step / max(t, 1e-6))))
+    rows = _rows_for(wl, d, per_step)
     for _ in range(args.warmup):
         wl.oracle_run(d, rows)
     res = [wl.oracle_run(d, rows) for _ in range(args.steps)]
@@ -1196,9 +1204,9 @@ def run_ours(args, wl, rank, local_rank, world):
     # tokens are a step's input); the one-shot call (weights copied and sliced every step) is reported beside it.
     s_h2d, s_cmp, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_measure(keys, fn, call):
+    def e2e_measure(keys, fn, call, single_output):
         gis = [{k: torch.empty_like(host[k], device=dev) for k in keys} for _ in range(2)]
-        y0 = fn(g if keys == list(host) else {k: g[k] for k in keys})
+        y0 = fn(g if keys == list(host) else {k: g[k] for k in keys}, 0)
         ys = y0 if isinstance(y0, tuple) else (y0,)
         y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
         h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
@@ -1208,7 +1216,7 @@ def run_ours(args, wl, rank, local_rank, world):
             for st in (s_h2d, s_cmp, s_d2h):
                 st.wait_event(start_ev)
             used = [None, None]
-            d2h_done = None
+            d2h_done = [None, None]
             for i in range(n):
                 b = i & 1
                 if used[b] is not None:
@@ -1219,18 +1227,20 @@ def run_ours(args, wl, rank, local_rank, world):
                     staged = torch.cuda.Event()
                     staged.record(s_h2d)
                 s_cmp.wait_event(staged)
-                if d2h_done is not None:
-                    s_cmp.wait_event(d2h_done)  # the previous result has left the output buffer
+                if d2h_done[b] is not None:
+                    s_cmp.wait_event(d2h_done[b])  # step i-2's result has left output buffer b
+                if single_output and d2h_done[b ^ 1] is not None:
+                    s_cmp.wait_event(d2h_done[b ^ 1])  # one output buffer: step i-1's result has left it
                 with torch.cuda.stream(s_cmp):
-                    y = fn(gis[b])
+                    y = fn(gis[b], b)
                     used[b] = torch.cuda.Event()
                     used[b].record(s_cmp)
                 s_d2h.wait_event(used[b])
                 with torch.cuda.stream(s_d2h):
                     for yh, yd in zip(y_host, y if isinstance(y, tuple) else (y,)):
                         yh.copy_(yd, non_blocking=True)
-                    d2h_done = torch.cuda.Event()
-                    d2h_done.record(s_d2h)
+                    d2h_done[b] = torch.cuda.Event()
+                    d2h_done[b].record(s_d2h)
             cur = torch.cuda.current_stream(dev)
             cur.wait_stream(s_h2d)
             cur.wait_stream(s_cmp)
@@ -1250,12 +1260,13 @@ def run_ours(args, wl, rank, local_rank, world):
         barrier()
         return {"value": wl.work() * world * args.steps / e2e_s / scale, "unit": wl.unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "call": call,
-                "pipelining": "two device staging buffers: step i+1's host-to-device copies overlap step i's "
-                              "compute; device-to-host copies on a third stream; all copies inside the timed region"}
+                "pipelining": ("two device staging buffers" + ("" if single_output else " and two output buffers") +
+                               ": step i+1's host-to-device copies overlap step i's compute; device-to-host "
+                               "copies on a third stream; all copies inside the timed region")}
 
-    one_shot_e2e = e2e_measure(list(host), lambda gi: wl.one_shot(tp, gi, dev), wl.e2e_call)
+    one_shot_e2e = e2e_measure(list(host), lambda gi, b: wl.one_shot(tp, gi, dev), wl.e2e_call, True)
     prep = wl.prepared(tp, g, dev)
-    e2e = e2e_measure(prep[0], prep[1], prep[2]) if prep is not None else one_shot_e2e
+    e2e = e2e_measure(prep[0], prep[1], prep[2], False) if prep is not None else one_shot_e2e
 
     out = {
         "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,

@@ -111,6 +111,16 @@ uint64_t tp_kernel_launches(void);
  * TP_ERR_DEVICE_TIMEOUT while the CUDA context stays usable. */
 tp_status tp_debug_watchdog(uint32_t wait_ms, void* stream);
 
+/* The tiling the GEMM entry points use on the current device for an output of
+ * M rows x N columns in `groups` groups (colwise: one group per shard;
+ * rowwise sum: one group), `swiglu` != 0 for tp_colwise_swiglu:
+ *   0  CTA pairs (tcgen05 cta_group::2), 256 x 256 tiles (M >= 256)
+ *   1  one CTA per tile, 128 x 256 tiles
+ *   2  one CTA per tile, 128 x 128 tiles (when that fills the SMs in fewer
+ *      rounds of tiles; never for SwiGLU)
+ * A pure query (no launch); -1 if a size is < 1 or no CUDA device is usable. */
+int tp_gemm_tile_plan(int64_t M, int64_t N, int groups, int swiglu);
+
 /* Synchronises `stream`, then reports (and clears) the device error word that
  * kernels set: TP_ERR_DEVICE_TIMEOUT if a bounded wait ran out, else
  * TP_ERR_RANGE if an epilogue that stores fp16 (the Q/K/V of the attention

@@ -46,6 +46,7 @@ SIGNATURES = {
     "tp_last_error_message": (ctypes.c_char_p, []),
     "tp_check_device_error": (_I, [_P]),
     "tp_debug_watchdog": (_I, [ctypes.c_uint32, _P]),
+    "tp_gemm_tile_plan": (_I, [_I64, _I64, _I, _I]),
     "tp_shard_weight": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P]),
     "tp_shard_weight_all": (_I, [_P, _I64, _I64, _I, _I, _P, _P]),
     "tp_kernel_launches": (ctypes.c_uint64, []),
@@ -159,6 +160,13 @@ def tp_check_device_error(stream=None) -> int:
 
 def tp_debug_watchdog(wait_ms, stream=None) -> int:
     return lib().tp_debug_watchdog(wait_ms, _stream(stream))
+
+
+GEMM_PLANS = {0: "pair256x256", 1: "cta128x256", 2: "cta128x128"}
+
+
+def tp_gemm_tile_plan(M, N, groups, swiglu=False) -> int:
+    return lib().tp_gemm_tile_plan(M, N, groups, int(bool(swiglu)))
 
 
 def tp_shard_weight(W, rows, cols, style, tp_degree, rank, out, stream=None) -> int:

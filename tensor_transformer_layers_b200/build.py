@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libtp.so")
-SOURCES = ["api.cu", "gemm.cu", "attn.cu", "merge.cu", "slice.cu", "reduce.cu", "noalloc.cu", "watchdog.cu"]
+SOURCES = ["api.cu", "gemm.cu", "attn.cu", "merge.cu", "slice.cu", "reduce.cu", "noalloc.cu", "watchdog.cu", "plan.cu"]
 HEADERS = ["ptx.cuh", "internal.h", os.path.join("..", "..", "include", "tp.h")]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

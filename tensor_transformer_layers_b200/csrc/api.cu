@@ -894,6 +894,13 @@ tp_status tp_debug_watchdog(uint32_t wait_ms, void* stream) {
              : TP_ERR_CUDA;
 }
 
+int tp_gemm_tile_plan(int64_t M, int64_t N, int groups, int swiglu) {
+  if (M < 1 || N < 1 || groups < 1) return -1;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != TP_OK) return -1;
+  return gemm_tile_plan(M, N, groups, swiglu != 0, di->num_sms);
+}
+
 // ----------------------------------------------------------------------- MLP pair
 size_t tp_mlp_workspace_bytes(int64_t M, int64_t D, int64_t F, int tp_degree) {
   if (check_mlp_shape(M, D, F, tp_degree) != TP_OK) return 0;

@@ -139,7 +139,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_kv = (p.Mk + kBKV - 1) / kBKV;
+  // Ordinary attention reads Q, K and V from one buffer (the Q, K, V heads of
+  // a row side by side): one map and offsets fixed by Hs.  Only the Ring
+  // block (statistics mode) takes keys and values from another token set.
+  const CUtensorMap* kvm = kStats ? &kvmap : &qmap;
+  const int Mk = kStats ? p.Mk : p.Mq;
+  const int n_kv = (Mk + kBKV - 1) / kBKV;
   const int q_blocks = (p.Mq + kTiles * kBQ - 1) / (kTiles * kBQ);
   const int n_items = q_blocks * p.T * p.Hs;
   // this CTA's items: blockIdx.x, blockIdx.x + gridDim.x, ...
@@ -172,15 +177,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&qmap);
-      tma_prefetch_desc(&kvmap);
+      if (kStats) tma_prefetch_desc(&kvmap);
       bool ok = true;
       int g = 0;           // K/V blocks issued (ring position)
       int qn[2] = {0, 0};  // Q tiles issued per tile slot
       for (int k = 0; k < my_items && ok; ++k) {
         const AttnItem it = attn_item(int(blockIdx.x) + k * int(gridDim.x), q_blocks, p.Hs);
-        const int qcol = p.q_col0 + it.head * kD;
-        const int kcol = p.k_col0 + it.head * kD;
-        const int vcol = p.v_col0 + it.head * kD;
+        const int qcol = (kStats ? p.q_col0 : 0) + it.head * kD;
+        const int kcol = (kStats ? p.k_col0 : p.Hs * kD) + it.head * kD;
+        const int vcol = (kStats ? p.v_col0 : 2 * p.Hs * kD) + it.head * kD;
         // K/V block 0 first (its ring stage frees early), then Q_0 and Q_1 (each
         // free once the previous item's last S_t is done), then the other blocks.
         for (int j = 0; j < n_kv && ok; ++j, ++g) {
@@ -191,10 +196,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* sk = smem + kKVOff + st * kKVBytes;
           mbar_arrive_expect_tx(&kv_full[st], kKVBytes);
-          tma_load_3d(sk, &kvmap, &kv_full[st], kcol, j * kBKV, it.shard);
-          tma_load_3d(sk + kBox, &kvmap, &kv_full[st], kcol + 64, j * kBKV, it.shard);
-          tma_load_3d(sk + 2 * kBox, &kvmap, &kv_full[st], vcol, j * kBKV, it.shard);
-          tma_load_3d(sk + 3 * kBox, &kvmap, &kv_full[st], vcol + 64, j * kBKV, it.shard);
+          tma_load_3d(sk, kvm, &kv_full[st], kcol, j * kBKV, it.shard);
+          tma_load_3d(sk + kBox, kvm, &kv_full[st], kcol + 64, j * kBKV, it.shard);
+          tma_load_3d(sk + 2 * kBox, kvm, &kv_full[st], vcol, j * kBKV, it.shard);
+          tma_load_3d(sk + 3 * kBox, kvm, &kv_full[st], vcol + 64, j * kBKV, it.shard);
           if (j == 0) {
             for (int t = 0; t < kTiles; ++t) {
               if (!mbar_wait(&q_empty[t], (k & 1) ^ 1u, abort_flag)) {
@@ -366,10 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
         }
         const int kv0 = j * kBKV;
-        if (kv0 + kBKV > p.Mk) {  // ragged last key tile: keys >= Mk do not exist
+        if (kv0 + kBKV > Mk) {  // ragged last key tile: keys >= Mk do not exist
 #pragma unroll
           for (int i = 0; i < kBKV; ++i)
-            if (kv0 + i >= p.Mk) s[i] = -INFINITY;
+            if (kv0 + i >= Mk) s[i] = -INFINITY;
         }
         // Row max: 3-input max over four independent chains (64 instructions
         // for 128 scores, a short dependency chain).  The element-wise code

@@ -64,15 +64,18 @@ constexpr int kTmemCols = 2 * kAccCols;
 constexpr int kEpiBuf = 32 * 128;
 constexpr int kEpiBytes = 4 * 2 * kEpiBuf;
 
-// single-CTA kernel
-constexpr int BM1 = 128, BN1 = 256;
-constexpr int kStages1 = 4;
+// single-CTA kernels: 128 x BN tiles, BN = 256 (4 stages) or 128 (6 stages)
+constexpr int BM1 = 128;
 constexpr int kABytes1 = BM1 * BK * 2;
-constexpr int kStageBytes1 = kABytes1 + BN1 * BK * 2;
-constexpr int kEpiOff1 = kStages1 * kStageBytes1;
-constexpr int kBarOff1 = kEpiOff1 + kEpiBytes;
-constexpr int kSmemBytes1 = kBarOff1 + 256 + 1024;  // + barriers + 1 KB alignment slack
-constexpr uint32_t kIdesc1 = idesc_bf16_f32(BM1, BN1, false);
+template <int BN>
+struct Cta1 {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStageBytes = kABytes1 + BN * BK * 2;
+  static constexpr int kEpiOff = kStages * kStageBytes;
+  static constexpr int kBarOff = kEpiOff + kEpiBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers + 1 KB alignment slack
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(BM1, BN, false);
+};
 
 // CTA-pair kernel (per CTA: 128 rows of A and 128 rows of B per stage)
 constexpr int BM2 = 256, BN2 = 256;
@@ -85,7 +88,9 @@ constexpr int kSmemBytes2 = kBarOff2 + 512 + 1024;
 constexpr uint32_t kIdesc2 = idesc_bf16_f32(BM2, BN2, false);
 
 static_assert(kTmemCols == 512, "two 256-column accumulators fill TMEM");
-static_assert(kSmemBytes1 <= 227 * 1024 && kSmemBytes2 <= 227 * 1024, "shared memory budget");
+static_assert(Cta1<256>::kSmemBytes <= 227 * 1024 && Cta1<128>::kSmemBytes <= 227 * 1024 &&
+                  kSmemBytes2 <= 227 * 1024,
+              "shared memory budget");
 
 // GELU, tanh form: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))
 // (Hendrycks & Gimpel, 2016), on two values at once: the polynomial and the
@@ -321,12 +326,18 @@ __device__ __forceinline__ void epilogue_swiglu(const GemmArgs& p, const CUtenso
 // ============================================================================
 // Single-CTA kernel
 // ============================================================================
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                    const __grid_constant__ CUtensorMap omap, const GemmArgs p) {
+  using C = Cta1<BN>;
+  constexpr int kStages1 = C::kStages;
+  constexpr int kStageBytes1 = C::kStageBytes;
+  // SwiGLU tiles take two 128-row weight boxes: only the 256-wide tile has room
+  const bool swiglu = BN == 256 && p.swiglu;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff1);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + kStages1;
   uint64_t* tfull = empty + kStages1;
   uint64_t* tempty = tfull + 2;
@@ -336,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int out_bn = p.swiglu ? BN1 / 2 : BN1;  // output columns per tile
+  const int out_bn = swiglu ? BN / 2 : BN;  // output columns per tile
   const int m_tiles = (p.M + BM1 - 1) / BM1;
   const int n_tiles = (p.N + out_bn - 1) / out_bn;
   const int tiles = m_tiles * n_tiles * p.groups;
@@ -391,12 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(sa, &amap, &full[stage], kb * BK, s, tc.mb * BM1);
           else
             tma_load_3d(sa, &amap, &full[stage], kb * BK, tc.mb * BM1, p.a_follows_shard ? s : 0);
-          if (p.swiglu) {  // two 128-row boxes: gate rows, then the matching up rows
+          if (swiglu) {  // two 128-row boxes: gate rows, then the matching up rows
             tma_load_3d(sa + kABytes1, &bmap, &full[stage], kb * BK, tc.nb * 128, tc.g + s);
             tma_load_3d(sa + kABytes1 + 128 * BK * 2, &bmap, &full[stage], kb * BK, int(p.up_off) + tc.nb * 128,
                         tc.g + s);
           } else {
-            tma_load_3d(sa + kABytes1, &bmap, &full[stage], kb * BK, tc.nb * BN1, tc.g + s);
+            tma_load_3d(sa + kABytes1, &bmap, &full[stage], kb * BK, tc.nb * BN, tc.g + s);
           }
           ++issued;
           if (++stage == kStages1) {
@@ -442,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t db = sdesc_sw128(sa + kABytes1, 16, 1024);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)  // advance 16 bf16 = 32 bytes inside the swizzle row
-            umma_ss(d_tmem, da + uint64_t(2 * k), db + uint64_t(2 * k), kIdesc1, (it | k) != 0 ? 1u : 0u);
+            umma_ss(d_tmem, da + uint64_t(2 * k), db + uint64_t(2 * k), C::kIdesc, (it | k) != 0 ? 1u : 0u);
           umma_commit(&empty[stage]);
           if (++stage == kStages1) {
             stage = 0;
@@ -463,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // this warp's TMEM lane quarter
-    uint8_t* stage = smem + kEpiOff1 + (warp - 2) * 2 * kEpiBuf;
+    uint8_t* stage = smem + C::kEpiOff + (warp - 2) * 2 * kEpiBuf;
     uint32_t nbox = 0;
     int local = 0;
     bool ok = true;
@@ -477,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kAccCols);
       const int row0 = tc.mb * BM1 + q * 32;
-      if (p.swiglu)
+      if (swiglu)
         epilogue_swiglu(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, stage, nbox);
       else if (p.out_f32)
         epilogue_rows_f32(p, &omap, taddr, row0, lane, tc.g, tc.nb * out_bn, out_bn, stage, nbox);
@@ -701,7 +712,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 int g_max_pairs[64] = {};
 std::mutex g_pairs_mu;
 
-int max_active_pairs(int num_sms) {
+}  // namespace
+
+int gemm_max_active_pairs(int num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
   std::lock_guard<std::mutex> lock(g_pairs_mu);
@@ -724,6 +737,8 @@ int max_active_pairs(int num_sms) {
   return g_max_pairs[dev];
 }
 
+namespace {
+
 // A's map: {K_s, rows, z}, or {K_s, z, rows} for a split input (memory
 // [rows][z][K_s]), with a box of 64 x box_rows rows either way.
 CUresult make_a_map(CUtensorMap* map, const GemmOperand& A, const GemmArgs& a, uint32_t box_rows) {
@@ -731,19 +746,42 @@ CUresult make_a_map(CUtensorMap* map, const GemmOperand& A, const GemmArgs& a, u
   return make_map_3d_bf16(map, A.base, A.k, A.rows, A.z, BK, box_rows, A.zrows);
 }
 
+// One-CTA kernel with 128 x BN tiles, one CTA per SM at most.
+template <int BN>
+cudaError_t launch_cta1(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, CUtensorMap& amap,
+                        const CUtensorMap& omap, int num_sms, cudaStream_t s) {
+  using C = Cta1<BN>;
+  const bool swiglu = BN == 256 && a.swiglu;
+  if (a.swiglu && !swiglu) return note_cuda_error("gemm: SwiGLU needs 256-column tiles", cudaErrorInvalidValue);
+  const int out_bn = swiglu ? BN / 2 : BN;
+  CUtensorMap bmap;
+  if (make_a_map(&amap, A, a, BM1) != CUDA_SUCCESS ||
+      make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, uint32_t(out_bn), B.zrows) != CUDA_SUCCESS)
+    return note_cuda_error("gemm: tensor map encode", cudaErrorInvalidValue);
+  const int64_t tiles = int64_t((a.M + BM1 - 1) / BM1) * ((a.N + out_bn - 1) / out_bn) * a.groups;
+  const int grid = int(tiles < num_sms ? tiles : num_sms);
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return note_cuda_error("gemm: set shared memory size", e);
+  gemm_tc_kernel<BN><<<grid, kThreads, C::kSmemBytes, s>>>(amap, bmap, omap, a);
+  count_launch();
+  return note_cuda_error("gemm: launch", cudaGetLastError());
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms,
                         cudaStream_t s) {
   if (a.M <= 0 || a.N <= 0 || a.groups <= 0) return cudaSuccess;
-  CUtensorMap amap, bmap, omap;
+  CUtensorMap amap, omap;
   const CUresult om = a.out_f32 ? make_map_out_f32(&omap, a.out, uint64_t(a.N), uint64_t(a.M), uint64_t(a.groups),
                                                    uint64_t(a.ldo), uint64_t(a.out_gstride))
                                 : make_map_out_u16(&omap, a.out, uint64_t(a.N), uint64_t(a.M), uint64_t(a.groups),
                                                    uint64_t(a.ldo), uint64_t(a.out_gstride));
   if (om != CUDA_SUCCESS) return note_cuda_error("gemm: output tensor map encode", cudaErrorInvalidValue);
-  if (a.M >= BM2) {
+  const int plan = gemm_tile_plan(a.M, a.N, a.groups, a.swiglu != 0, num_sms);
+  if (plan == kPlanPair) {
     // CTA-pair kernel: each CTA loads 128-row halves of both operands.
+    CUtensorMap bmap;
     if (make_a_map(&amap, A, a, 128) != CUDA_SUCCESS ||
         make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, 128, B.zrows) != CUDA_SUCCESS)
       return note_cuda_error("gemm (CTA pairs): tensor map encode", cudaErrorInvalidValue);
@@ -751,7 +789,7 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
     if (e != cudaSuccess) return note_cuda_error("gemm (CTA pairs): set shared memory size", e);
     const int out_bn = a.swiglu ? BN2 / 2 : BN2;
     const int64_t tiles = int64_t((a.M + BM2 - 1) / BM2) * ((a.N + out_bn - 1) / out_bn) * a.groups;
-    int pairs = max_active_pairs(num_sms);
+    int pairs = gemm_max_active_pairs(num_sms);
     if (tiles < pairs) pairs = int(tiles);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(2 * pairs));
@@ -770,18 +808,8 @@ cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmAr
     if (e == cudaSuccess) e = cudaGetLastError();
     return note_cuda_error("gemm (CTA pairs): launch", e);
   }
-  if (make_a_map(&amap, A, a, BM1) != CUDA_SUCCESS ||
-      make_map_3d_bf16(&bmap, B.base, B.k, B.rows, B.z, BK, a.swiglu ? BN1 / 2 : BN1, B.zrows) != CUDA_SUCCESS)
-    return note_cuda_error("gemm: tensor map encode", cudaErrorInvalidValue);
-  const int m_tiles = (a.M + BM1 - 1) / BM1;
-  const int n_tiles = (a.N + (a.swiglu ? BN1 / 2 : BN1) - 1) / (a.swiglu ? BN1 / 2 : BN1);
-  const int64_t tiles = int64_t(m_tiles) * n_tiles * a.groups;
-  const int grid = int(tiles < num_sms ? tiles : num_sms);
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes1);
-  if (e != cudaSuccess) return note_cuda_error("gemm: set shared memory size", e);
-  gemm_tc_kernel<<<grid, kThreads, kSmemBytes1, s>>>(amap, bmap, omap, a);
-  count_launch();
-  return note_cuda_error("gemm: launch", cudaGetLastError());
+  return plan == kPlanCta128x128 ? launch_cta1<128>(A, B, a, amap, omap, num_sms, s)
+                                 : launch_cta1<256>(A, B, a, amap, omap, num_sms, s);
 }
 
 }  // namespace tp

@@ -87,6 +87,14 @@ struct GemmOperand {
 
 cudaError_t launch_gemm(const GemmOperand& A, const GemmOperand& B, const GemmArgs& a, int num_sms, cudaStream_t s);
 
+// The tiling launch_gemm picks for M output rows x N columns x groups: CTA
+// pairs with 256 x 256 tiles, or one CTA per tile with 128 x 256 or 128 x 128
+// tiles (the last when it fills the SMs in fewer rounds; never for SwiGLU).
+enum { kPlanPair = 0, kPlanCta128x256 = 1, kPlanCta128x128 = 2 };
+int gemm_tile_plan(int64_t M, int64_t N, int groups, bool swiglu, int num_sms);  // plan.cu
+// CTA pairs of the pair kernel that fit on the current device at once (cached).
+int gemm_max_active_pairs(int num_sms);
+
 // ----------------------------------------------------------------------------
 // a6: per-shard SDPA (attn.cu).  Queries come from the Q columns of one fp16
 // buffer [T][Mq][*], keys and values from the K and V columns of another (or

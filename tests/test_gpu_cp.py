@@ -148,3 +148,49 @@ def test_unshard_inverts_rowwise_slicing():
     assert tp.tp_unshard_rowwise_all(sh, rows, cols, T, back) == 0
     torch.cuda.synchronize()
     assert np.array_equal(from_dev(back), W)
+
+
+def test_flux_scale_ring_and_ulysses():
+    # The flux_attn tokens (4608, 24 heads x 128) over 4 context-parallel ranks,
+    # laid out as the bench runs them: Ring steps over all ranks in one launch
+    # each (rank r holds block (r - s) mod 4 at step s), the merge, and Ulysses
+    # with the ranks as the SDPA's shards.  Sampled rows against the oracle;
+    # Ulysses bit-exact against the single-device attention.
+    M, H, R = 4608, 24, 4
+    D, Ms = H * 128, M // R
+    QKV = syn.normal_f16((M, 3 * D), 1.0, seed=46, tid=415)
+    full = to_dev(QKV)
+    qkv = full.view(R, Ms, 3 * D)
+    ring = torch.cat([qkv, qkv]).contiguous()
+    blk = Ms * 3 * D
+    Ob = torch.empty((R, R, Ms, D), dtype=torch.float32, device="cuda")
+    Lb = torch.empty((R, R, H, Ms), dtype=torch.float32, device="cuda")
+    for s in range(R):
+        kv = ring.data_ptr() + 2 * (R - s) * blk
+        assert tp.tp_sdpa_block_stats(qkv, Ms, kv, Ms, H * R, R, Ob[s], Lb[s]) == 0
+    Y = torch.empty((R, Ms, D), dtype=torch.int16, device="cuda")
+    assert tp.tp_attn_merge(Ob, Lb, R, Ms, H * R, R, Y) == 0
+    ref_dev = torch.empty((M, D), dtype=torch.int16, device="cuda")
+    assert tp.tp_sdpa_shards(full, M, H, 1, ref_dev) == 0
+    # Ulysses: pack by head group, exchange, attend (ranks = shards), exchange back, unpack
+    send = torch.empty((R, R, Ms, 3 * D // R), dtype=torch.int16, device="cuda")
+    jobs = [(qkv[s], Ms, 3 * D, tp.TP_ROWWISE, send[s], [1, 1, 1]) for s in range(R)]
+    assert tp.tp_shard_weights_batch(jobs, R) == 0
+    recv = send.transpose(0, 1).contiguous()
+    O = torch.empty((R, M, D // R), dtype=torch.int16, device="cuda")
+    assert tp.tp_sdpa_shards(recv, M, H, R, O) == 0
+    back = O.view(R, R, Ms, D // R).transpose(0, 1).contiguous()
+    Yu = torch.empty((R, Ms, D), dtype=torch.int16, device="cuda")
+    for s in range(R):
+        assert tp.tp_unshard_rowwise_all(back[s], Ms, D, R, Yu[s]) == 0
+    torch.cuda.synchronize()
+    assert tp.tp_check_device_error() == 0
+    assert np.array_equal(from_dev(Yu).reshape(M, D), from_dev(ref_dev)), "Ulysses regrouping changed bits"
+    rng = np.random.default_rng(46)
+    rows = np.unique(np.r_[0, M - 1, rng.choice(M, 30, replace=False)])
+    q = syn.f16_bits_to_f64(QKV)
+    got = from_dev(Y).reshape(M, D)
+    for j in (0, H - 1):
+        Qj, Kj, Vj = _heads(q, H, j)
+        ref = o.sdpa(Qj[rows], Kj, Vj)
+        assert_rounded_once(got[rows, j * 128:(j + 1) * 128], ref, f"flux Ring head {j}")

@@ -1,5 +1,6 @@
 """Colwise (a2/a3/a5) and rowwise (a4/a7) tcgen05 GEMMs against the oracle,
-including ragged M, N and K tails and tiny sizes."""
+including ragged M, N and K tails and tiny sizes, on each of the three
+tilings (CTA pairs 256x256, one CTA 128x256, one CTA 128x128)."""
 import numpy as np
 import pytest
 import torch
@@ -12,16 +13,33 @@ from tests._util import assert_parity, assert_rounded_once, f64, from_dev, to_de
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("M,K,Ns,T,gelu,bias,f16", [
+PAIR, CTA256, CTA128 = 0, 1, 2  # tp_gemm_tile_plan codes
+
+COLWISE = [
     (64, 128, 256, 2, True, True, False),     # tiny MLP's FFN-in
     (1, 64, 8, 1, False, False, False),
     (129, 72, 264, 3, True, True, False),     # ragged M, N and K tails
     (300, 1024, 512, 4, False, True, False),
     (256, 3072, 2304, 1, False, False, True),  # one QKV shard of the Flux attention block (fp16 out)
     (129, 72, 264, 3, True, True, True),
-    (257, 72, 264, 3, True, True, False),     # CTA-pair kernel: one row into a second 256-row tile
-    (512, 192, 520, 2, False, True, False),   # CTA-pair kernel, ragged N
-])
+    (257, 72, 264, 3, True, True, False),     # one row into a second 256-row block
+    (512, 192, 520, 2, False, True, False),   # ragged N
+    (200, 72, 2568, 4, True, True, False),    # 128x256 tiles: 128x128 tiles would take two rounds
+    (200, 72, 2568, 4, False, False, True),
+    (1025, 72, 2056, 4, True, True, False),   # CTA pairs, ragged M and N, three rounds of tiles
+    (1025, 72, 2056, 4, False, True, True),
+]
+
+
+def test_colwise_cases_cover_every_tiling():
+    plans = {tp.tp_gemm_tile_plan(M, Ns, T) for (M, K, Ns, T, *_) in COLWISE}
+    assert plans == {PAIR, CTA256, CTA128}
+    assert tp.tp_gemm_tile_plan(200, 2568, 4) == CTA256
+    assert tp.tp_gemm_tile_plan(1025, 2056, 4) == PAIR
+    assert tp.tp_gemm_tile_plan(512, 520, 2) == CTA128
+
+
+@pytest.mark.parametrize("M,K,Ns,T,gelu,bias,f16", COLWISE)
 def test_colwise(M, K, Ns, T, gelu, bias, f16):
     X = syn.normal_bf16((M, K), 1.0, seed=M, tid=300)
     W = syn.normal_bf16((T, Ns, K), 1.0 / np.sqrt(K), seed=K, tid=301)
@@ -47,15 +65,33 @@ def test_colwise(M, K, Ns, T, gelu, bias, f16):
             assert_rounded_once(g[r], ref, f"colwise shard {r}")
 
 
-@pytest.mark.parametrize("M,Ks,N,T,bias", [
+ROWWISE = [
     (64, 256, 128, 2, True),           # tiny MLP's FFN-out
     (1, 8, 8, 1, True),
     (129, 72, 264, 3, True),           # ragged
     (300, 512, 520, 4, False),
     (256, 768, 3072, 4, False),        # Flux attention out-projection shards
-    (257, 72, 264, 3, True),           # CTA-pair kernel, ragged everywhere
-    (1024, 1536, 520, 8, True),        # CTA-pair kernel, 8 shards in one K loop
-])
+    (257, 72, 264, 3, True),           # ragged everywhere
+    (1024, 1536, 520, 8, True),        # 8 shards in one K loop
+    (512, 768, 3072, 4, True),         # a 512-token text stream's out-projection: 128x128 tiles
+    (232, 72, 20488, 2, True),         # 128x256 tiles, ragged N
+    (2305, 72, 2056, 8, True),         # CTA pairs, ragged M and N, 8 shards in one K loop
+]
+
+
+def test_rowwise_cases_cover_every_tiling():
+    plans = {tp.tp_gemm_tile_plan(M, N, 1) for (M, Ks, N, T, _) in ROWWISE}
+    assert plans == {PAIR, CTA256, CTA128}
+    assert tp.tp_gemm_tile_plan(512, 3072, 1) == CTA128
+    assert tp.tp_gemm_tile_plan(2305, 2056, 1) == PAIR
+
+
+def test_swiglu_never_takes_128_column_tiles():
+    for M in (1, 64, 200, 256, 512, 4096):
+        assert tp.tp_gemm_tile_plan(M, 1024, 1, swiglu=True) == (PAIR if M >= 256 else CTA256)
+
+
+@pytest.mark.parametrize("M,Ks,N,T,bias", ROWWISE)
 def test_rowwise_sum(M, Ks, N, T, bias):
     A = syn.normal_bf16((T, M, Ks), 1.0, seed=M, tid=310)
     W = syn.normal_bf16((T, N, Ks), 1.0 / np.sqrt(T * Ks), seed=Ks, tid=311)
