@@ -16,7 +16,8 @@ step-level calls are bit-identical to ``tp_mlp_run`` and ``tp_mlp_pair``).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                        [--workload flux_mlp|flux_mlp_sweep|flux_attn|wide_block|flux_reduce|flux_swiglu|
-                                   flux_split_input|flux_joint_attn]
+                                   flux_split_input|flux_joint_attn|flux_ring_attn|flux_ulysses_attn]
+                       [--mode replicas|tp] [--no-cpu-baseline] [--headline-only]
 The default workload (flux_mlp) is the headline line.  The others time the
 remaining rows the same way: flux_mlp_sweep (the same pair at tp_degree 1, 2,
 4 and 8, one kernel set per degree), flux_attn (QKV head split, QKV GEMM, SDPA,
@@ -24,7 +25,12 @@ out-projection), wide_block (attention then MLP pair at tp_degree 8, every
 row), flux_reduce (the standalone partial-sum reduction, GB/s), flux_swiglu
 (the SwiGLU pair: packed gate/up slicing, SwiGLU colwise GEMM, rowwise GEMM)
 flux_split_input (rowwise_split_input on an FFN-out-sized projection) and
-flux_joint_attn (dual-stream joint attention, 4096 image + 512 text tokens).
+flux_joint_attn (dual-stream joint attention, 4096 image + 512 text tokens),
+flux_ring_attn / flux_ulysses_attn (context-parallel attention, ranks emulated
+on one GPU).  A default one-GPU run also times flux_attn, flux_mlp_sweep,
+wide_block and flux_reduce after the headline measurement, with short loops,
+and adds them to the same line as ``other_configs`` (``--headline-only``
+leaves them out).
 Under torchrun (N > 1) every rank runs the same workload on its own tokens
 (independent replicas: the layer pair has no exchange step when all shards of
 a layer live on one GPU), so per-GPU work is fixed ("weak" scaling) and the
@@ -1100,7 +1106,7 @@ def config_dict(wl, world):
 
 
 # --------------------------------------------------------------------------- GPU leg
-def run_ours(args, wl, rank, local_rank, world):
+def run_ours(args, wl, rank, local_rank, world, light=False):
     import numpy as np
     import torch
 
@@ -1264,9 +1270,12 @@ def run_ours(args, wl, rank, local_rank, world):
                                ": step i+1's host-to-device copies overlap step i's compute; device-to-host "
                                "copies on a third stream; all copies inside the timed region")}
 
-    one_shot_e2e = e2e_measure(list(host), lambda gi, b: wl.one_shot(tp, gi, dev), wl.e2e_call, True)
-    prep = wl.prepared(tp, g, dev)
-    e2e = e2e_measure(prep[0], prep[1], prep[2], False) if prep is not None else one_shot_e2e
+    if light:  # a secondary configuration of the default run: kernels and step only, no e2e legs
+        one_shot_e2e, prep, e2e = None, None, None
+    else:
+        one_shot_e2e = e2e_measure(list(host), lambda gi, b: wl.one_shot(tp, gi, dev), wl.e2e_call, True)
+        prep = wl.prepared(tp, g, dev)
+        e2e = e2e_measure(prep[0], prep[1], prep[2], False) if prep is not None else one_shot_e2e
 
     out = {
         "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
@@ -1309,9 +1318,43 @@ def run_ours(args, wl, rank, local_rank, world):
         out["e2e_one_shot"] = one_shot_e2e
     out.update({"roofline": roofline, "kernels": kinfo, "clocks": clocks, "e2e": e2e,
                 "gpu_launches": int(launches), "wall_s_timed_region": round(t_wall, 4), "cpu_baseline": None})
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not light:
         out["cpu_baseline"] = cpu_baseline(wl, d)
     return out
+
+
+# The other configurations, timed after the headline line's own measurement in
+# a default one-GPU run (same process, same box), each with a short loop:
+# (workload, steps, warmup).
+OTHER_CONFIGS = [("flux_attn", 10, 3), ("flux_mlp_sweep", 5, 3), ("wide_block", 3, 3), ("flux_reduce", 20, 3)]
+
+
+def other_configs(args, rank, local_rank):
+    """Compact lines for the other configurations (attention block, tp_degree
+    sweep, wide block, standalone reduction): value, step time, the dominant
+    kernel's roofline fraction and every kernel's rate.  A failure is reported
+    in its entry and does not stop the headline line."""
+    res = {}
+    for key, steps, warmup in OTHER_CONFIGS:
+        a = argparse.Namespace(**vars(args))
+        a.steps, a.warmup, a.no_cpu_baseline = steps, warmup, True
+        try:
+            o = run_ours(a, WORKLOADS[key](), rank, local_rank, 1, light=True)
+        except Exception as e:  # noqa: BLE001 - recorded in the line, the headline stands
+            res[key] = {"error": f"{type(e).__name__}: {e}"}
+            continue
+        r = o["roofline"]
+        res[key] = {"config": o["config"]["workload"], "value": round(o["value"], 1), "unit": o["unit"],
+                    "steps": steps, "warmup": warmup, "ms_per_step": round(o["ms_per_step"], 5),
+                    "roofline": {"kernel": r["kernel"], "achieved": r["achieved"], "peak": r["peak"],
+                                 "unit": r["unit"], "frac": r["frac"]},
+                    "kernels": {n: {"achieved": k["achieved"], "unit": k["unit"], "frac": k["frac"]}
+                                for n, k in o["kernels"].items()},
+                    "clocks": o["clocks"], "gpu_launches": o["gpu_launches"]}
+        for extra in ("per_degree", "frac_of_nominal_dense_bf16"):
+            if extra in o:
+                res[key][extra] = o[extra]
+    return res
 
 
 def run_tp(args, wl, rank, local_rank, world):
@@ -1440,6 +1483,9 @@ def main(argv=None):
                     help="flux_mlp (default: the headline line); the others time the remaining rows")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle leg (cpu_baseline is then null)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="leave out the other configurations that a default one-GPU run times after the "
+                         "headline (other_configs)")
     ap.add_argument("--mode", choices=["replicas", "tp"], default="replicas",
                     help="replicas (default): every GPU runs the whole layer (all tp_degree shards) on its own "
                          "tokens; tp: tensor parallelism across the processes, one shard per rank, one NCCL "
@@ -1464,6 +1510,8 @@ def main(argv=None):
             out = run_tp(args, wl, rank, local_rank, world)
         else:
             out = run_ours(args, wl, rank, local_rank, world)
+            if world == 1 and args.workload == "flux_mlp" and not args.headline_only:
+                out["other_configs"] = other_configs(args, rank, local_rank)
         if rank == 0 and out is not None:
             print(json.dumps(out), flush=True)
     finally:
