@@ -145,16 +145,28 @@ class ClockSampler:
                 return f(self._h)
         return 0
 
+    def _power_w(self):
+        """Instantaneous board power (the plain power reading is a one-second
+        average, too slow for a timed region of a few milliseconds)."""
+        n = self._nvml
+        try:
+            fv = n.nvmlDeviceGetFieldValues(self._h, [n.NVML_FI_DEV_POWER_INSTANT])[0]
+            if fv.nvmlReturn == 0:
+                return float(fv.value.uiVal) / 1000.0
+        except Exception:  # noqa: BLE001 - fall back to the averaged reading
+            pass
+        try:
+            return n.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+        except Exception:  # noqa: BLE001
+            return None
+
     def _run(self):
         n = self._nvml
         while not self._stop.is_set():
             try:
                 clk = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
                 reasons = int(self._reasons())
-                try:
-                    power_w = n.nvmlDeviceGetPowerUsage(self._h) / 1000.0
-                except Exception:  # noqa: BLE001
-                    power_w = None
+                power_w = self._power_w()
                 self.samples.append((clk, reasons, power_w))
             except Exception:  # noqa: BLE001
                 pass
