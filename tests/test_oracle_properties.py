@@ -71,3 +71,45 @@ def test_joint_sharded_equals_unsharded(T, mi, mt, seed):
     Yi, Yt = o.joint_attn_unsharded(Xi, Xt, Wqi, Wqt, Woi, Wot, heads)
     Si, St = o.joint_attn_sharded_summed(Xi, Xt, Wqi, Wqt, Woi, Wot, heads, T)
     assert np.allclose(Yi, Si, rtol=1e-12, atol=1e-12) and np.allclose(Yt, St, rtol=1e-12, atol=1e-12)
+
+
+@settings(max_examples=40, deadline=None)
+@given(T=st.sampled_from([1, 2, 3, 4]), m=st.integers(1, 5), k=st.integers(1, 3), n=st.integers(1, 3),
+       seed=st.integers(0, 2**31 - 1))
+def test_colwise_shards_and_rowwise_partials_compose_the_layer(T, m, k, n, seed):
+    # The two halves of the pair one at a time: each colwise shard is a column
+    # block of the unsharded hidden layer, and the rowwise partials of those
+    # blocks plus the bias once sum to the unsharded output (exact on integers).
+    rng = np.random.default_rng(seed)
+    D, F = k * T, n * T
+    X, W_up, W_down = _ints(rng, (m, D)), _ints(rng, (F, D)), _ints(rng, (D, F))
+    b_up, b_down = _ints(rng, (F,)), _ints(rng, (D,))
+    ident = lambda x: x  # noqa: E731
+    H_full = X @ W_up.T + b_up
+    parts = []
+    for r in range(T):
+        H_r = o.mlp_colwise_shard(X, W_up, b_up, T, r, act=ident)
+        assert np.array_equal(H_r, H_full[:, r * n:(r + 1) * n])
+        parts.append(o.mlp_rowwise_partial(H_r, W_down, T, r))
+    assert np.array_equal(sum(parts) + b_down, o.mlp_unsharded(X, W_up, b_up, W_down, b_down, act=ident))
+
+
+@settings(max_examples=15, deadline=None)
+@given(T=st.sampled_from([1, 2, 4]), m=st.integers(1, 6), seed=st.integers(0, 2**31 - 1))
+def test_attention_shard_outputs_partition_the_heads(T, m, seed):
+    # Head splitting is an exact partition: shard r's attention output is the
+    # column block of its heads in the unsharded per-head output, each head
+    # computed on its own (the attention of a head reads only that head's
+    # Q, K and V columns).
+    heads, dh = 4, 128
+    D = heads * dh
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((m, D)) * 0.05
+    W_qkv = rng.standard_normal((3 * D, D)) * 0.05
+    qkv = X @ W_qkv.T
+    full = np.concatenate([o.sdpa(qkv[:, h * dh:(h + 1) * dh], qkv[:, D + h * dh:D + (h + 1) * dh],
+                                  qkv[:, 2 * D + h * dh:2 * D + (h + 1) * dh]) for h in range(heads)], axis=1)
+    Hs = heads // T
+    for r in range(T):
+        O_r = o.attn_shard_output(X, W_qkv, heads, T, r)
+        np.testing.assert_allclose(O_r, full[:, r * Hs * dh:(r + 1) * Hs * dh], rtol=1e-12, atol=1e-12)
