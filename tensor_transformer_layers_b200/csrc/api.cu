@@ -38,6 +38,12 @@ struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
   int* err = nullptr;  // device address of g_device_error
+  // A second stream and two events, on which the joint-attention layer runs
+  // the text stream's projections beside the image stream's (created at first
+  // use; side_mu keeps one caller's fork/join sequence together).
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex side_mu;
 };
 
 std::mutex g_mu;
@@ -164,7 +170,8 @@ namespace {
 // out_rows: rows of each group's output block (0 = M; larger when `out` is a
 // row range of a taller [T][out_rows][Ns] buffer).
 tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, const uint16_t* W, const uint16_t* b,
-                      int64_t Ns, int T, int gelu, int out_f16, uint16_t* out, cudaStream_t s, int64_t out_rows = 0) {
+                      int64_t Ns, int T, int gelu, int out_f16, uint16_t* out, cudaStream_t s, int64_t out_rows = 0,
+                      int sms = 0) {
   if (M == 0) return TP_OK;
   const GemmOperand A{X, uint64_t(K), uint64_t(M), 1};
   const GemmOperand B{W, uint64_t(K), uint64_t(Ns), uint64_t(T)};
@@ -183,13 +190,14 @@ tp_status run_colwise(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t K, c
   a.gelu = gelu;
   a.out_f16 = out_f16;
   a.err = di->err;
-  return launch_gemm(A, B, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return launch_gemm(A, B, a, sms > 0 ? sms : di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 // rowwise: Y = sum_r A[r] . W[r]^T + bias.  a_rows: rows of each shard's A
 // block in memory (0 = M; larger when A is a row range of a taller buffer).
 tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, const uint16_t* W, int64_t N,
-                      const uint16_t* bias, int T, void* Y, cudaStream_t s, int64_t a_rows = 0, bool out_f32 = false) {
+                      const uint16_t* bias, int T, void* Y, cudaStream_t s, int64_t a_rows = 0, bool out_f32 = false,
+                      int sms = 0) {
   if (M == 0) return TP_OK;
   const GemmOperand Aop{A, uint64_t(Ks), uint64_t(M), uint64_t(T), uint64_t(a_rows)};
   const GemmOperand Bop{W, uint64_t(Ks), uint64_t(N), uint64_t(T)};
@@ -209,7 +217,7 @@ tp_status run_rowwise(DeviceInfo* di, const uint16_t* A, int64_t M, int64_t Ks, 
   a.out_f16 = 0;
   a.out_f32 = out_f32 ? 1 : 0;
   a.err = di->err;
-  return launch_gemm(Aop, Bop, a, di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return launch_gemm(Aop, Bop, a, sms > 0 ? sms : di->num_sms, s) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 // SwiGLU colwise: out[g] = silu(X W_gate,g^T + bg) * (X W_up,g^T + bu), W[g] = [gate; up].
@@ -487,18 +495,75 @@ tp_status attn_forward(DeviceInfo* di, const uint16_t* X, int64_t M, int64_t D, 
 // QKV land in one [T][Mi+Mt][3*Ds] buffer (image rows first), one SDPA runs
 // over the joint tokens, and each stream's rows of O go through its own
 // rowwise out-projection (read in place as a row range of O).
+//
+// The two streams' projections are independent, so when both have tokens the
+// text stream's GEMM runs on a side stream over a share of the SMs in
+// proportion to its rows, beside the image stream's GEMM on the rest: the
+// short text launch no longer runs alone on a partly idle GPU.  Each GEMM's
+// per-element arithmetic does not depend on its SM budget, so the outputs are
+// the same as with the two launches in sequence.
 tp_status joint_attn_forward(DeviceInfo* di, const uint16_t* X_img, int64_t Mi, const uint16_t* X_txt, int64_t Mt,
                              int64_t D, int heads, int T, const uint16_t* wq_img, const uint16_t* wq_txt,
                              const uint16_t* wo_img, const uint16_t* wo_txt, uint16_t* QKV, uint16_t* O,
                              uint16_t* Y_img, uint16_t* Y_txt, cudaStream_t s) {
   const int64_t Ds = D / T, M = Mi + Mt;
-  tp_status st = run_colwise(di, X_img, Mi, D, wq_img, nullptr, 3 * Ds, T, 0, 1, QKV, s, M);
-  if (st != TP_OK) return st;
-  if ((st = run_colwise(di, X_txt, Mt, D, wq_txt, nullptr, 3 * Ds, T, 0, 1, QKV + Mi * 3 * Ds, s, M)) != TP_OK)
+  uint16_t* qkv_txt = QKV + Mi * 3 * Ds;
+  const uint16_t* o_txt = O + Mi * Ds;
+  if (Mi == 0 || Mt == 0 || di->num_sms < 8) {
+    tp_status st = run_colwise(di, X_img, Mi, D, wq_img, nullptr, 3 * Ds, T, 0, 1, QKV, s, M);
+    if (st == TP_OK) st = run_colwise(di, X_txt, Mt, D, wq_txt, nullptr, 3 * Ds, T, 0, 1, qkv_txt, s, M);
+    if (st == TP_OK) st = run_sdpa(di, QKV, M, heads, T, O, s);
+    if (st == TP_OK) st = run_rowwise(di, O, Mi, Ds, wo_img, D, nullptr, T, Y_img, s, M);
+    if (st == TP_OK) st = run_rowwise(di, o_txt, Mt, Ds, wo_txt, D, nullptr, T, Y_txt, s, M);
     return st;
-  if ((st = run_sdpa(di, QKV, M, heads, T, O, s)) != TP_OK) return st;
-  if ((st = run_rowwise(di, O, Mi, Ds, wo_img, D, nullptr, T, Y_img, s, M)) != TP_OK) return st;
-  return run_rowwise(di, O + Mi * Ds, Mt, Ds, wo_txt, D, nullptr, T, Y_txt, s, M);
+  }
+  std::lock_guard<std::mutex> lock(di->side_mu);
+  if (di->side == nullptr) {
+    cudaError_t e = cudaStreamCreateWithFlags(&di->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&di->fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&di->join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      note_cuda_error("joint attention: side stream", e);
+      return TP_ERR_CUDA;
+    }
+  }
+  // SMs for the text stream: its share of the rows, in whole CTA pairs, and
+  // at least one pair on each side.
+  const int pairs = di->num_sms / 2;
+  int txt_pairs = int((int64_t(pairs) * Mt + M / 2) / M);
+  if (txt_pairs < 1) txt_pairs = 1;
+  if (txt_pairs > pairs - 1) txt_pairs = pairs - 1;
+  const int sms_txt = 2 * txt_pairs, sms_img = di->num_sms - sms_txt;
+  // Runs img(s) and txt(side) between a fork of `s` and a join back into it;
+  // the join is enqueued whatever happened, so `s` never runs ahead of work
+  // left on the side stream.
+  auto beside = [&](auto img, auto txt) {
+    cudaError_t e = cudaEventRecord(di->fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(di->side, di->fork, 0);
+    if (e != cudaSuccess) {
+      note_cuda_error("joint attention: fork", e);
+      return TP_ERR_CUDA;
+    }
+    tp_status st = txt();
+    const tp_status si = img();
+    if (st == TP_OK) st = si;
+    e = cudaEventRecord(di->join, di->side);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, di->join, 0);
+    if (e != cudaSuccess) {
+      note_cuda_error("joint attention: join", e);
+      return TP_ERR_CUDA;
+    }
+    return st;
+  };
+  tp_status st = beside(
+      [&] { return run_colwise(di, X_img, Mi, D, wq_img, nullptr, 3 * Ds, T, 0, 1, QKV, s, M, sms_img); },
+      [&] { return run_colwise(di, X_txt, Mt, D, wq_txt, nullptr, 3 * Ds, T, 0, 1, qkv_txt, di->side, M, sms_txt); });
+  if (st == TP_OK) st = run_sdpa(di, QKV, M, heads, T, O, s);
+  if (st == TP_OK)
+    st = beside(
+        [&] { return run_rowwise(di, O, Mi, Ds, wo_img, D, nullptr, T, Y_img, s, M, false, sms_img); },
+        [&] { return run_rowwise(di, o_txt, Mt, Ds, wo_txt, D, nullptr, T, Y_txt, di->side, M, false, sms_txt); });
+  return st;
 }
 
 struct MlpHandle {

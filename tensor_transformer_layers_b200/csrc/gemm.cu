@@ -33,8 +33,10 @@
 //   rowwise_split_input (style table): A is the replicated input and shard s
 //            reads its own K range of it; the A map is {K_s, T, M}, so the
 //            slice of the input is a TMA coordinate, not a copy.
-// * gemm_tc_kernel: one CTA per SM, 128x256 tile, M=128 N=256 K=16 MMAs,
-//   4 stages of 48 KB (A 128x64 + B 256x64).  Used for M < 256.
+// * gemm_tc_kernel<BN>: one CTA per tile, 128xBN tiles, M=128 N=BN K=16
+//   MMAs; BN = 256 with 4 stages of 48 KB (A 128x64 + B 256x64), BN = 128 with
+//   6 stages of 32 KB.  The host plan (plan.cu) picks it for M < 256 and for
+//   problems whose 128x128 tiles fill the SMs in fewer rounds than pairs do.
 // * gemm_pair_kernel: CTA pairs (cluster of 2, tcgen05 cta_group::2), 256x256
 //   tile per pair.  Each CTA loads its 128 rows of A and its 128 rows of B
 //   (32 KB per k-block instead of 48 KB: the B tile is split between the two
@@ -712,13 +714,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 int g_max_pairs[64] = {};
 std::mutex g_pairs_mu;
 
-}  // namespace
-
-int gemm_max_active_pairs(int num_sms) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
+// Pair clusters of the pair kernel that fit on device `dev` at once (cached).
+int device_max_pairs(int dev) {
   std::lock_guard<std::mutex> lock(g_pairs_mu);
   if (g_max_pairs[dev] == 0) {
+    int num_sms = 0;
+    if (cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || num_sms < 2)
+      num_sms = 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(num_sms & ~1));
     cfg.blockDim = dim3(kThreads);
@@ -735,6 +737,16 @@ int gemm_max_active_pairs(int num_sms) {
     g_max_pairs[dev] = n;
   }
   return g_max_pairs[dev];
+}
+
+}  // namespace
+
+int gemm_max_active_pairs(int num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
+  const int pairs = device_max_pairs(dev);
+  // a launch given part of the SMs (beside another kernel) stays within them
+  return pairs < num_sms / 2 ? pairs : (num_sms / 2 > 0 ? num_sms / 2 : 1);
 }
 
 namespace {

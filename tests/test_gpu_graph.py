@@ -69,3 +69,33 @@ def test_one_shot_swiglu_replays_in_a_graph():
     eager = tp.swiglu_mlp_pair(s["X"], s["W_in"], s["b_in"], s["W_out"], s["b_out"], T)
     torch.cuda.synchronize()
     assert np.array_equal(from_dev(Y), from_dev(eager))
+
+
+def test_prepared_joint_attention_replays_in_a_graph():
+    # The joint layer forks its text-stream projections onto a side stream and
+    # joins them back; inside a capture that becomes two branches of the graph.
+    Mi, Mt, D, H, T = 300, 77, 256, 2, 2
+    d = {k: to_dev(v) for k, v in syn.joint_attn_inputs(Mi, Mt, D, seed=25).items()}
+    layer = tp.JointAttnBlock(d["W_qkv_img"], d["W_qkv_txt"], d["W_o_img"], d["W_o_txt"], H, T)
+    Xi, Xt = d["X_img"].clone(), d["X_txt"].clone()
+    Yi = torch.empty((Mi, D), dtype=torch.int16, device="cuda")
+    Yt = torch.empty((Mt, D), dtype=torch.int16, device="cuda")
+    nb = tp.tp_joint_attn_run_workspace_bytes(Mi, Mt, D, H, T)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+
+    def run():
+        stream = torch.cuda.current_stream().cuda_stream
+        assert tp.tp_joint_attn_run(layer.handle, Xi, Mi, Xt, Mt, Yi, Yt, ws, nb, stream) == 0
+
+    g = _capture(run)
+    for seed in (26, 27):
+        Xi.copy_(to_dev(syn.normal_bf16((Mi, D), 1.0, seed=seed, tid=0)))
+        Xt.copy_(to_dev(syn.normal_bf16((Mt, D), 1.0, seed=seed, tid=1)))
+        g.replay()
+        torch.cuda.synchronize()
+        ei, et = layer(Xi, Xt)
+        torch.cuda.synchronize()
+        assert np.array_equal(from_dev(Yi), from_dev(ei)) and np.array_equal(from_dev(Yt), from_dev(et))
+    del g
+    layer.close()
+    assert tp.tp_check_device_error() == 0

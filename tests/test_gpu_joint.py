@@ -98,17 +98,22 @@ def test_flux_joint_sampled_rows_and_prepared(flux_joint):
 
 
 def test_bench_step_sequence_matches_one_shot():
-    # bench.py times the joint block as its six step-level calls (one batched
-    # slice launch, two row-range QKV GEMMs, one SDPA, two row-range
-    # out-projections); they must give exactly the one-shot result.
+    # bench.py times the joint block as one call of the prepared layer (which
+    # runs the two streams' projections side by side: five launches) and, for
+    # the per-kernel breakdown, as its six step-level calls (one batched slice
+    # launch, two row-range QKV GEMMs, one SDPA, two row-range
+    # out-projections); both must give exactly the one-shot result.
     import bench
     wl = bench.JointAttnWorkload(dict(kind="joint", M_img=300, M_txt=77, D=256, H=2, T=2, seed=9))
     d = wl.host_inputs(0)
     g = {k: to_dev(v) for k, v in d.items()}
+    kernels = wl.kernels(tp, g, "cuda")
+    assert [k.name for k in kernels if k.composite] == ["joint_layer"]
     n0 = tp.tp_kernel_launches()
-    for k in wl.kernels(tp, g, "cuda"):
+    for k in kernels:
         k.fn()
-    assert tp.tp_kernel_launches() - n0 == 6
+    assert tp.tp_kernel_launches() - n0 == 5 + 6
     torch.cuda.synchronize()
     gi, gt = _run(g, 300, 77, 2, 2)
     assert np.array_equal(from_dev(wl.bufs["Y_img"]), gi) and np.array_equal(from_dev(wl.bufs["Y_txt"]), gt)
+    assert np.array_equal(from_dev(wl.bufs["Yj_img"]), gi) and np.array_equal(from_dev(wl.bufs["Yj_txt"]), gt)
