@@ -27,10 +27,9 @@ row), flux_reduce (the standalone partial-sum reduction, GB/s), flux_swiglu
 flux_split_input (rowwise_split_input on an FFN-out-sized projection) and
 flux_joint_attn (dual-stream joint attention, 4096 image + 512 text tokens),
 flux_ring_attn / flux_ulysses_attn (context-parallel attention, ranks emulated
-on one GPU).  A default one-GPU run also times flux_attn, flux_mlp_sweep,
-wide_block and flux_reduce after the headline measurement, with short loops,
-and adds them to the same line as ``other_configs`` (``--headline-only``
-leaves them out).
+on one GPU).  A default one-GPU run also times every other workload after
+the headline measurement, with short loops, and adds them to the same line
+as ``other_configs`` (``--headline-only`` leaves them out).
 Under torchrun (N > 1) every rank runs the same workload on its own tokens
 (independent replicas: the layer pair has no exchange step when all shards of
 a layer live on one GPU), so per-GPU work is fixed ("weak" scaling) and the
@@ -1379,14 +1378,18 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
 # The other configurations, timed after the headline line's own measurement in
 # a default one-GPU run (same process, same box), each with a short loop:
 # (workload, steps, warmup).
-OTHER_CONFIGS = [("flux_attn", 10, 3), ("flux_mlp_sweep", 5, 3), ("wide_block", 3, 3), ("flux_reduce", 20, 3)]
+OTHER_CONFIGS = [("flux_attn", 10, 3), ("flux_mlp_sweep", 5, 3), ("wide_block", 3, 3), ("flux_reduce", 20, 3),
+                 ("flux_swiglu", 10, 3), ("flux_split_input", 10, 3), ("flux_joint_attn", 10, 3),
+                 ("flux_ring_attn", 10, 3), ("flux_ulysses_attn", 10, 3)]
 
 
 def other_configs(args, rank, local_rank):
-    """Compact lines for the other configurations (attention block, tp_degree
-    sweep, wide block, standalone reduction): value, step time, the dominant
-    kernel's roofline fraction and every kernel's rate.  A failure is reported
-    in its entry and does not stop the headline line."""
+    """Compact lines for the other configurations and rows (attention block,
+    tp_degree sweep, wide block, standalone reduction, SwiGLU pair,
+    rowwise_split_input, joint attention, Ring and Ulysses attention): value,
+    step time, the dominant kernel's roofline fraction and every kernel's
+    rate.  A failure is reported in its entry and does not stop the headline
+    line."""
     res = {}
     for key, steps, warmup in OTHER_CONFIGS:
         a = argparse.Namespace(**vars(args))
@@ -1404,7 +1407,7 @@ def other_configs(args, rank, local_rank):
                     "kernels": {n: {"achieved": k["achieved"], "unit": k["unit"], "frac": k["frac"]}
                                 for n, k in o["kernels"].items()},
                     "clocks": o["clocks"], "gpu_launches": o["gpu_launches"]}
-        for extra in ("per_degree", "frac_of_nominal_dense_bf16"):
+        for extra in ("per_degree", "frac_of_nominal_dense_bf16", "value_with_emulated_exchange"):
             if extra in o:
                 res[key][extra] = o[extra]
     return res
