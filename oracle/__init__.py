@@ -34,7 +34,6 @@ from __future__ import annotations
 
 import contextlib
 import ctypes
-import os
 
 import numpy as np
 
