@@ -33,6 +33,7 @@ def _inputs(Mi, Mt, D, heads, seed):
     (200, 77, 256, 2, 2),     # ragged both streams
     (128, 128, 512, 4, 4),
     (300, 5, 384, 3, 1),      # a handful of text tokens
+    (513, 1, 256, 2, 2),      # one text token beside a ragged image stream
 ])
 def test_joint_small(Mi, Mt, D, heads, T):
     d, dd = _inputs(Mi, Mt, D, heads, seed=Mi + Mt)
@@ -117,3 +118,40 @@ def test_bench_step_sequence_matches_one_shot():
     gi, gt = _run(g, 300, 77, 2, 2)
     assert np.array_equal(from_dev(wl.bufs["Y_img"]), gi) and np.array_equal(from_dev(wl.bufs["Y_txt"]), gt)
     assert np.array_equal(from_dev(wl.bufs["Yj_img"]), gi) and np.array_equal(from_dev(wl.bufs["Yj_txt"]), gt)
+
+
+def test_joint_layers_from_two_host_threads():
+    # Two threads, each on its own stream, call the joint layer (which forks
+    # onto the device's side stream) at the same time; each result must equal
+    # the single-threaded one.
+    import threading
+    Mi, Mt, D, heads, T = 300, 77, 256, 2, 2
+    runs = []
+    for seed in (31, 32):
+        d, dd = _inputs(Mi, Mt, D, heads, seed=seed)
+        runs.append((dd, _run(dd, Mi, Mt, heads, T)))
+    errors, results = [], [None, None]
+
+    def worker(i):
+        try:
+            dd = runs[i][0]
+            st = torch.cuda.Stream()
+            with torch.cuda.stream(st):
+                for _ in range(3):
+                    Yi, Yt = tp.joint_attn_block(dd["X_img"], dd["X_txt"], dd["W_qkv_img"], dd["W_qkv_txt"],
+                                                 dd["W_o_img"], dd["W_o_txt"], heads, T, stream=st)
+            st.synchronize()
+            results[i] = (from_dev(Yi), from_dev(Yt))
+        except Exception as e:  # noqa: BLE001 - reported below
+            errors.append(e)
+
+    ts = [threading.Thread(target=worker, args=(i,)) for i in range(2)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join(timeout=120)
+    assert not errors, errors
+    for i in range(2):
+        assert np.array_equal(results[i][0], runs[i][1][0]) and np.array_equal(results[i][1], runs[i][1][1])
+    assert tp.tp_check_device_error() == 0
+
