@@ -113,7 +113,6 @@ class ClockSampler:
         self.period = period
         self.samples = []
         self.max_mhz = None
-        self.power_limit_w = None
         self._stop = threading.Event()
         self._thread = None
         self._h = None
@@ -129,10 +128,6 @@ class ClockSampler:
             self._nvml = pynvml
             self._h = pynvml.nvmlDeviceGetHandleByIndex(idx)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-            try:
-                self.power_limit_w = pynvml.nvmlDeviceGetEnforcedPowerLimit(self._h) / 1000.0
-            except Exception:  # noqa: BLE001 - reported as null
-                self.power_limit_w = None
         except Exception:  # noqa: BLE001 - no NVML: report no clocks
             self._h = None
 
@@ -144,29 +139,11 @@ class ClockSampler:
                 return f(self._h)
         return 0
 
-    def _power_w(self):
-        """Instantaneous board power (the plain power reading is a one-second
-        average, too slow for a timed region of a few milliseconds)."""
-        n = self._nvml
-        try:
-            fv = n.nvmlDeviceGetFieldValues(self._h, [n.NVML_FI_DEV_POWER_INSTANT])[0]
-            if fv.nvmlReturn == 0:
-                return float(fv.value.uiVal) / 1000.0
-        except Exception:  # noqa: BLE001 - fall back to the averaged reading
-            pass
-        try:
-            return n.nvmlDeviceGetPowerUsage(self._h) / 1000.0
-        except Exception:  # noqa: BLE001
-            return None
-
     def _run(self):
         n = self._nvml
         while not self._stop.is_set():
             try:
-                clk = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
-                reasons = int(self._reasons())
-                power_w = self._power_w()
-                self.samples.append((clk, reasons, power_w))
+                self.samples.append((n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM), int(self._reasons())))
             except Exception:  # noqa: BLE001
                 pass
             time.sleep(self.period)
@@ -184,15 +161,11 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
         mhz = [s[0] for s in self.samples]
         bits = 0
-        for _, r, _ in self.samples:
+        for _, r in self.samples:
             bits |= r
         reasons = [name for b, name in REASON_BITS.items() if bits & b and name != "gpu_idle"]
-        watts = [s[2] for s in self.samples if s[2] is not None]
-        # Board power beside the clock: a clock below max with the power at the
-        # enforced limit is the power cap, whether or not its reason bit was seen.
         return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
-                "samples": len(mhz), "power_w": round(statistics.median(watts), 1) if watts else None,
-                "power_max_w": round(max(watts), 1) if watts else None, "power_limit_w": self.power_limit_w}
+                "samples": len(mhz)}
 
 
 def source_sha(*names) -> str:
