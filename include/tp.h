@@ -376,6 +376,12 @@ tp_status tp_attn_run(void* handle, const uint16_t* X, int64_t M, uint16_t* Y,
  * (its X and Y may then be NULL; M_txt == 0 gives tp_attn_block's result on
  * the image stream).  Both streams' Q/K/V go into one buffer and one SDPA
  * launch; each out-projection reads its stream's rows of O in place.
+ * Scheduling: when both streams have tokens, each text-stream projection runs
+ * on a stream the library owns (one per device), forked from `stream` and
+ * joined back into it with events, beside the image stream's projection on
+ * the remaining SMs; the results are the same bits as in sequence, the call
+ * can be captured into a CUDA graph, and calls from several host threads are
+ * serialized on that internal stream.
  * Workspace: tp_joint_attn_workspace_bytes(). */
 size_t tp_joint_attn_workspace_bytes(int64_t M_img, int64_t M_txt, int64_t D, int heads, int tp_degree);
 tp_status tp_joint_attn_block(const uint16_t* X_img, int64_t M_img, const uint16_t* X_txt, int64_t M_txt,
