@@ -10,7 +10,8 @@
 // which is exactly softmax over all keys applied to all values (each O_b is
 // its block's weighted mean; 2^(lse_b) is its block's total weight).
 // HBM-bound: a thread owns 8 consecutive columns of one row and head (two
-// 16-byte fp32 loads per block, one 16-byte bf16 store).
+// 16-byte fp32 loads per block, one 16-byte bf16 store); for up to 8 blocks
+// all of a group's loads are in flight before the sum.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -19,9 +20,14 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// kNP > 0: the block count is a compile-time constant, so every block's loads
+// of one column group are issued before the weighted sum (all of them in
+// flight at once); kNP == 0 walks a run-time count one block at a time.
+template <int kNP>
 __global__ void __launch_bounds__(kThreads)
     attn_merge_kernel(const float4* __restrict__ O_parts, const float* __restrict__ lse_parts, int nparts, int64_t M,
                       int Hs, int64_t n8_total, uint4* __restrict__ O, float* __restrict__ lse_out) {
+  const int np = kNP > 0 ? kNP : nparts;
   const int64_t stride = int64_t(gridDim.x) * kThreads;
   const int64_t part_stride4 = n8_total * 2;             // float4s per block's O
   const int64_t lse_stride = n8_total / 16;              // T * Hs * M values per block
@@ -32,17 +38,36 @@ __global__ void __launch_bounds__(kThreads)
     const int head = c8 >> 4;
     const int64_t t = tr / M, row = tr - t * M;
     const int64_t li = (t * Hs + head) * M + row;
-    float L = -INFINITY;
-    for (int b = 0; b < nparts; ++b) L = fmaxf(L, lse_parts[b * lse_stride + li]);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float wsum = 0.f;
-    for (int b = 0; b < nparts; ++b) {
-      const float w = exp2f(lse_parts[b * lse_stride + li] - L);
-      const float4 lo = __ldcs(O_parts + b * part_stride4 + 2 * i);
-      const float4 hi = __ldcs(O_parts + b * part_stride4 + 2 * i + 1);
-      wsum += w;
-      acc[0] += w * lo.x; acc[1] += w * lo.y; acc[2] += w * lo.z; acc[3] += w * lo.w;
-      acc[4] += w * hi.x; acc[5] += w * hi.y; acc[6] += w * hi.z; acc[7] += w * hi.w;
+    float wsum = 0.f, L = -INFINITY;
+    if constexpr (kNP > 0) {
+      float lse[kNP];
+      float4 lo[kNP], hi[kNP];
+#pragma unroll
+      for (int b = 0; b < kNP; ++b) {
+        lse[b] = lse_parts[b * lse_stride + li];
+        lo[b] = __ldcs(O_parts + b * part_stride4 + 2 * i);
+        hi[b] = __ldcs(O_parts + b * part_stride4 + 2 * i + 1);
+      }
+#pragma unroll
+      for (int b = 0; b < kNP; ++b) L = fmaxf(L, lse[b]);
+#pragma unroll
+      for (int b = 0; b < kNP; ++b) {
+        const float w = exp2f(lse[b] - L);
+        wsum += w;
+        acc[0] += w * lo[b].x; acc[1] += w * lo[b].y; acc[2] += w * lo[b].z; acc[3] += w * lo[b].w;
+        acc[4] += w * hi[b].x; acc[5] += w * hi[b].y; acc[6] += w * hi[b].z; acc[7] += w * hi[b].w;
+      }
+    } else {
+      for (int b = 0; b < np; ++b) L = fmaxf(L, lse_parts[b * lse_stride + li]);
+      for (int b = 0; b < np; ++b) {
+        const float w = exp2f(lse_parts[b * lse_stride + li] - L);
+        const float4 lo = __ldcs(O_parts + b * part_stride4 + 2 * i);
+        const float4 hi = __ldcs(O_parts + b * part_stride4 + 2 * i + 1);
+        wsum += w;
+        acc[0] += w * lo.x; acc[1] += w * lo.y; acc[2] += w * lo.z; acc[3] += w * lo.w;
+        acc[4] += w * hi.x; acc[5] += w * hi.y; acc[6] += w * hi.z; acc[7] += w * hi.w;
+      }
     }
     const float inv = 1.0f / wsum;
     uint4 o;
@@ -63,9 +88,13 @@ cudaError_t launch_attn_merge(const float* O_parts, const float* lse_parts, int 
   if (n8_total == 0) return cudaSuccess;
   int64_t blocks = (n8_total + kThreads - 1) / kThreads;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  attn_merge_kernel<<<unsigned(blocks), kThreads, 0, s>>>(reinterpret_cast<const float4*>(O_parts), lse_parts,
-                                                          nparts, M, Hs, n8_total, reinterpret_cast<uint4*>(O),
-                                                          lse_out);
+  using Kernel = void (*)(const float4*, const float*, int, int64_t, int, int64_t, uint4*, float*);
+  constexpr Kernel by_count[9] = {attn_merge_kernel<0>, attn_merge_kernel<1>, attn_merge_kernel<2>,
+                                  attn_merge_kernel<3>, attn_merge_kernel<4>, attn_merge_kernel<5>,
+                                  attn_merge_kernel<6>, attn_merge_kernel<7>, attn_merge_kernel<8>};
+  const Kernel kernel = nparts <= 8 ? by_count[nparts] : attn_merge_kernel<0>;
+  kernel<<<unsigned(blocks), kThreads, 0, s>>>(reinterpret_cast<const float4*>(O_parts), lse_parts, nparts, M, Hs,
+                                               n8_total, reinterpret_cast<uint4*>(O), lse_out);
   count_launch();
   return note_cuda_error("attention merge: launch", cudaGetLastError());
 }
