@@ -1220,6 +1220,15 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
             kinfo[k.name]["breakdown"] = True
         if k.composite:
             kinfo[k.name]["composite"] = True
+    # Attention's second bound: the exponentials (Mq * Mk * heads = FLOP / (4 * head dim 128)) against the MUFU
+    # rate, 16 ex2 per clock per SM (the CUDA programming guide's arithmetic-throughput table).
+    sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+    mufu_peak = 16.0 * sm_count * float(clocks.get("sm_max_mhz") or 1965) * 1e6
+    for k in kernels:
+        if k.unit == "TFLOP/s" and ("sdpa" in k.name or k.name.startswith("ring_step")):
+            rate = k.work / (4.0 * 128) / (kinfo[k.name]["ms"] / 1e3)
+            kinfo[k.name]["exp_per_s"] = float(f"{rate:.4g}")
+            kinfo[k.name]["exp_frac_of_mufu"] = round(rate / mufu_peak, 4)
     dom = max((k for k in kernels if not (k.load or k.exchange or k.composite)), key=lambda k: kinfo[k.name]["ms"])
     src = "MEASURED_PEAKS.json" if peak_src == "measured" else "the recipe's fallback"
     roofline = {"kernel": dom.name, "bound": "tensor" if dom.unit == "TFLOP/s" else "hbm",
@@ -1227,6 +1236,10 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
                 "unit": dom.unit, "frac": kinfo[dom.name]["frac"], "traffic": recorded_traffic(dom.name, wl.key),
                 "peak_source": f"{peak_src}: {'bf16 burst' if dom.unit == 'TFLOP/s' else 'HBM copy'} from {src}",
                 "algorithmic_work_per_launch": dom.work}
+    if "exp_frac_of_mufu" in kinfo[dom.name]:
+        roofline["mufu"] = {"exp_per_s": kinfo[dom.name]["exp_per_s"], "peak_exp_per_s": float(f"{mufu_peak:.4g}"),
+                            "frac": kinfo[dom.name]["exp_frac_of_mufu"],
+                            "peak_basis": f"16 ex2 per clock per SM x {sm_count} SMs x max SM clock"}
 
     # ---- end to end through the public API, every step's inputs copied in from pinned host memory and its
     # result copied back, as a serving loop runs it: step i+1's inputs are staged (second device buffer, own
