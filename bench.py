@@ -1290,20 +1290,41 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
             cur.wait_stream(s_cmp)
             cur.wait_stream(s_d2h)
 
-        w0 = torch.cuda.Event()
-        w0.record()
-        run(max(1, args.warmup), w0)
-        torch.cuda.synchronize()
-        barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        run(args.steps, e0)
-        e1.record()
-        torch.cuda.synchronize()
-        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3)
-        barrier()
+        def copies_only(n, start_ev):  # the same copies with no compute: the host link's own time
+            for st in (s_h2d, s_d2h):
+                st.wait_event(start_ev)
+            for i in range(n):
+                with torch.cuda.stream(s_h2d):
+                    for k in keys:
+                        gis[i & 1][k].copy_(host[k], non_blocking=True)
+                with torch.cuda.stream(s_d2h):
+                    for yh, yd in zip(y_host, ys):
+                        yh.copy_(yd, non_blocking=True)
+            cur = torch.cuda.current_stream(dev)
+            cur.wait_stream(s_h2d)
+            cur.wait_stream(s_d2h)
+
+        def timed(fn):
+            w0 = torch.cuda.Event()
+            w0.record()
+            fn(max(1, args.warmup), w0)
+            torch.cuda.synchronize()
+            barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn(args.steps, e0)
+            e1.record()
+            torch.cuda.synchronize()
+            t = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+            barrier()
+            return t
+
+        e2e_s = timed(run)
+        copy_s = timed(copies_only)
         return {"value": wl.work() * world * args.steps / e2e_s / scale, "unit": wl.unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "call": call,
+                "copy_only_ms_per_step": round(1e3 * copy_s / args.steps, 4),
+                "frac_of_copy_bound": round(copy_s / e2e_s, 3),
                 "pipelining": ("two device staging buffers" + ("" if single_output else " and two output buffers") +
                                ": step i+1's host-to-device copies overlap step i's compute; device-to-host "
                                "copies on a third stream; all copies inside the timed region")}
