@@ -1411,9 +1411,12 @@ def other_configs(args, rank, local_rank):
                     "steps": steps, "warmup": warmup, "ms_per_step": round(o["ms_per_step"], 5),
                     "roofline": {"kernel": r["kernel"], "achieved": r["achieved"], "peak": r["peak"],
                                  "unit": r["unit"], "frac": r["frac"]},
-                    "kernels": {n: {"achieved": k["achieved"], "unit": k["unit"], "frac": k["frac"]}
+                    "kernels": {n: {"achieved": k["achieved"], "unit": k["unit"], "frac": k["frac"],
+                                    **({"exp_frac_of_mufu": k["exp_frac_of_mufu"]} if "exp_frac_of_mufu" in k else {})}
                                 for n, k in o["kernels"].items()},
                     "clocks": o["clocks"], "gpu_launches": o["gpu_launches"]}
+        if "mufu" in r:
+            res[key]["roofline"]["mufu_frac"] = r["mufu"]["frac"]
         for extra in ("per_degree", "frac_of_nominal_dense_bf16", "value_with_emulated_exchange"):
             if extra in o:
                 res[key][extra] = o[extra]
