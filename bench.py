@@ -653,7 +653,7 @@ class RingAttnWorkload(AttnWorkload):
         Ms = M // R
         qkv = g["QKV"].view(R, Ms, 3 * D)
         ring = torch.cat([qkv, qkv]).contiguous()  # blocks 0..R-1 twice: step s starts at block R - s
-        b = {"ring": ring, "O": torch.empty((R, R, Ms, D), dtype=torch.float32, device=dev),
+        b = {"ring": ring, "O": torch.empty((R, R, Ms, D), dtype=torch.float16, device=dev),
              "L": torch.empty((R, R, H, Ms), dtype=torch.float32, device=dev),
              "Y": torch.empty((R, Ms, D), dtype=torch.int16, device=dev)}
         self.bufs = b
@@ -665,7 +665,7 @@ class RingAttnWorkload(AttnWorkload):
                              lambda st=st: ck(tp.tp_sdpa_block_stats(qkv, Ms, ring.data_ptr() + 2 * (R - st) * blk,
                                                                      Ms, H * R, R, b["O"][st], b["L"][st]),
                                               f"ring step {st}")))
-        ks.append(Kernel("merge", "GB/s", R * (M * D * 4 + H * M * 4) + M * D * 2,
+        ks.append(Kernel("merge", "GB/s", R * (M * D * 2 + H * M * 4) + M * D * 2,
                          lambda: ck(tp.tp_attn_merge(b["O"], b["L"], R, Ms, H * R, R, b["Y"]), "merge")))
         return ks
 
@@ -1542,8 +1542,8 @@ def run_tp(args, wl, rank, local_rank, world):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="flux_mlp",
                     help="flux_mlp (default: the headline line); the others time the remaining rows")

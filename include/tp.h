@@ -411,19 +411,22 @@ tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, 
  *   lse[r][h][i] = log2 sum_j 2^(log2(e) Q_i K_j^T / sqrt(128))     (log2 units).
  * Q_qkv: fp16 [T x Mq x 3*Hs*128] (its Q columns are used); KV_qkv: fp16
  * [T x Mk x 3*Hs*128] (its K and V columns; may be the same buffer as Q_qkv,
- * or another rank's block), Hs = heads / T.  O: fp32 [T x Mq x Hs*128], O
- * normalised over this block's keys; lse: fp32 [T x Hs x Mq].  Mk >= 1.
+ * or another rank's block), Hs = heads / T.  O: fp16 [T x Mq x Hs*128], O
+ * normalised over this block's keys (a convex combination of fp16 rows of V,
+ * so always in fp16 range; rounded once, 2^-11 relative); lse: fp32
+ * [T x Hs x Mq].  Mk >= 1.
  * Errors: NULL, BAD_DEGREE, BAD_SHAPE, HEADS_INDIVISIBLE, ALIGNMENT. */
 tp_status tp_sdpa_block_stats(const uint16_t* Q_qkv, int64_t Mq, const uint16_t* KV_qkv, int64_t Mk, int heads,
-                              int tp_degree, float* O, float* lse, void* stream);
+                              int tp_degree, uint16_t* O, float* lse, void* stream);
 
 /* Merge of nparts (1..64) block results into the attention over all their
  * keys: O = sum_b 2^(lse_b - L) O_b / sum_b 2^(lse_b - L), L = max_b lse_b,
  * written in bf16 like tp_sdpa_shards' output; lse_out (or NULL) receives
- * L + log2 sum_b 2^(lse_b - L), so merges can be chained.  O_parts: fp32
- * [nparts x T x M x Hs*128]; lse_parts: fp32 [nparts x T x Hs x M]; O: bf16
- * [T x M x Hs*128]; lse_out: fp32 [T x Hs x M]. */
-tp_status tp_attn_merge(const float* O_parts, const float* lse_parts, int nparts, int64_t M, int heads,
+ * L + log2 sum_b 2^(lse_b - L).  O_parts: fp16 [nparts x T x M x Hs*128]
+ * (tp_sdpa_block_stats' output), summed in fp32; lse_parts: fp32
+ * [nparts x T x Hs x M]; O: bf16 [T x M x Hs*128]; lse_out: fp32
+ * [T x Hs x M]. */
+tp_status tp_attn_merge(const uint16_t* O_parts, const float* lse_parts, int nparts, int64_t M, int heads,
                         int tp_degree, uint16_t* O, float* lse_out, void* stream);
 
 /* Inverse of tp_shard_weight_all(..., TP_ROWWISE, ...): src [T x rows x cols/T]

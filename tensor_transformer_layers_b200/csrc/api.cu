@@ -266,16 +266,14 @@ tp_status run_rowwise_split(DeviceInfo* di, const uint16_t* X, int64_t M, int64_
 // Per-shard SDPA.  Queries: the Q columns of Qsrc [T][Mq][3*Hs*128]; keys and
 // values: the K and V columns of KVsrc [T][Mk][3*Hs*128] (the same buffer for
 // ordinary attention).  Output: bf16 O [T][Mq][Hs*128], or in the statistics
-// mode fp32 O and lse [T][Hs][Mq].
+// mode fp16 O and fp32 lse [T][Hs][Mq].
 tp_status run_sdpa_qkv(DeviceInfo* di, const uint16_t* Qsrc, int64_t Mq, const uint16_t* KVsrc, int64_t Mk, int Hs,
                        int T, void* O, bool stats, float* lse, cudaStream_t s) {
   if (Mq == 0 || Mk == 0) return TP_OK;
   const uint64_t cols = uint64_t(3) * Hs * TP_HEAD_DIM;
   AttnMaps m;
-  const CUresult om = stats ? make_map_out_f32(&m.o, O, uint64_t(Hs) * TP_HEAD_DIM, uint64_t(Mq), uint64_t(T),
-                                               uint64_t(Hs) * TP_HEAD_DIM, 0)
-                            : make_map_out_u16(&m.o, O, uint64_t(Hs) * TP_HEAD_DIM, uint64_t(Mq), uint64_t(T),
-                                               uint64_t(Hs) * TP_HEAD_DIM, 0);
+  const CUresult om =
+      make_map_out_u16(&m.o, O, uint64_t(Hs) * TP_HEAD_DIM, uint64_t(Mq), uint64_t(T), uint64_t(Hs) * TP_HEAD_DIM, 0);
   if (make_map_3d_f16(&m.q, Qsrc, cols, uint64_t(Mq), uint64_t(T), 64, 128) != CUDA_SUCCESS ||
       make_map_3d_f16(&m.kv, KVsrc, cols, uint64_t(Mk), uint64_t(T), 64, 128) != CUDA_SUCCESS || om != CUDA_SUCCESS) {
     note_cuda_error("attention: tensor map encode", cudaErrorInvalidValue);
@@ -1314,7 +1312,7 @@ tp_status tp_joint_attn_run(void* handle, const uint16_t* X_img, int64_t M_img, 
 
 // ----------------------------------------------------------------------- context parallelism pieces
 tp_status tp_sdpa_block_stats(const uint16_t* Q_qkv, int64_t Mq, const uint16_t* KV_qkv, int64_t Mk, int heads,
-                              int tp_degree, float* O, float* lse, void* stream) {
+                              int tp_degree, uint16_t* O, float* lse, void* stream) {
   if (!Q_qkv || !KV_qkv || !O || !lse) return TP_ERR_NULL;
   if (tp_degree < 1) return TP_ERR_BAD_DEGREE;
   if (Mq < 0 || Mk < 1 || heads < 1 || Mq >= kMaxDim || Mk >= kMaxDim) return TP_ERR_BAD_SHAPE;
@@ -1326,7 +1324,7 @@ tp_status tp_sdpa_block_stats(const uint16_t* Q_qkv, int64_t Mq, const uint16_t*
   return run_sdpa_qkv(di, Q_qkv, Mq, KV_qkv, Mk, heads / tp_degree, tp_degree, O, true, lse, as_stream(stream));
 }
 
-tp_status tp_attn_merge(const float* O_parts, const float* lse_parts, int nparts, int64_t M, int heads,
+tp_status tp_attn_merge(const uint16_t* O_parts, const float* lse_parts, int nparts, int64_t M, int heads,
                         int tp_degree, uint16_t* O, float* lse_out, void* stream) {
   if (!O_parts || !lse_parts || !O) return TP_ERR_NULL;
   if (tp_degree < 1) return TP_ERR_BAD_DEGREE;

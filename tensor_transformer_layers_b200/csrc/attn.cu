@@ -9,8 +9,8 @@
 // the per-block step of Ring attention ("Context parallelism" page, section
 // on Ring attention): queries and keys/values may come from different token
 // sets (two tensor maps), and in the statistics mode the kernel writes O
-// normalised in fp32 with each row's log-sum-exp, which the merge over key
-// blocks needs (merge.cu).
+// normalised over the block's keys, in fp16, with each row's log-sum-exp in
+// fp32, which the merge over key blocks needs (merge.cu).
 //
 // Structure: a work item is (shard, head, 256 query rows) = two 128-row query
 // tiles t = 0, 1.  The kernel is persistent: one CTA per SM walks the items
@@ -51,7 +51,10 @@
 // fp16 limit, and P <= 2^8 by the rescale rule), because bf16's 8-bit
 // significand at these two points alone costs more than the stated max-error
 // budget of the block.  S, the row statistics and O accumulate in fp32; O is
-// written in bf16 for the out-projection.
+// written in bf16 for the out-projection.  A Ring block's O is written in
+// fp16: each row is a convex combination of fp16 rows of V, so it stays in
+// fp16's range, and its rounding (2^-11 relative) is a quarter of the bf16
+// rounding the merged output takes once.
 // Every mbarrier wait is bounded (ptx.cuh); a timeout drains and exits.
 #include <cuda_bf16.h>
 
@@ -117,7 +120,7 @@ __device__ __forceinline__ AttnItem attn_item(int i, int q_blocks, int Hs) {
 
 // 320 threads: ten warps, so some SM sub-partitions (16K registers each) hold
 // three of them, which caps a thread at 168 registers.
-// kStats: the statistics mode (fp32 O and log-sum-exp) is a separate
+// kStats: the statistics mode (fp16 O and log-sum-exp) is a separate
 // instantiation, so the ordinary kernel carries none of its code.
 template <bool kStats>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -454,69 +457,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float inv_l = 1.0f / l_run;
         const uint64_t inv_l2 = f32x2(inv_l, inv_l);
         uint8_t* stg = smem + kOutOff + warp * kOutBuf;
-        if constexpr (!kStats) {
-          // O_t / l in bf16, 64 columns at a time: staged in this warp's box
-          // in the 128-byte swizzle of the output map, then one TMA store
-          // (whole 128-byte lines; rows >= Mq are clipped, a box wholly below
-          // Mq skipped).
+        // O_t / l, 64 columns at a time (bf16; fp16 in the statistics mode),
+        // staged in this warp's box in the 128-byte swizzle of the output
+        // map, then one TMA store (whole 128-byte lines; rows >= Mq are
+        // clipped, a box wholly below Mq skipped).
 #pragma unroll 1
-          for (int half = 0; half < 2; ++half) {
-            if (lane == 0) bulk_wait_read_0();  // the previous store has read the box
-            __syncwarp();
+        for (int half = 0; half < 2; ++half) {
+          if (lane == 0) bulk_wait_read_0();  // the previous store has read the box
+          __syncwarp();
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-              uint32_t r[32];
-              tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(half * 64 + c * 32), r);
-              uint32_t w[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                float lo, hi;
-                f32x2_split(mul_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv_l2), lo,
-                            hi);
-                w[i] = pack_bf16x2(lo, hi);
-              }
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int chunk = c * 4 + q;  // 16-byte chunk of this lane's 128-byte row
-                *reinterpret_cast<uint4*>(stg + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
-                    make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-              }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && row0 < p.Mq) {
-              tma_store_3d(&omap, stg, it.head * kD + half * 64, row0, it.shard);
-              bulk_commit();
-            }
-          }
-        } else {
-          // Statistics mode: O_t / l in fp32 (32-column boxes of 128-byte
-          // rows) and each row's log-sum-exp of the scaled scores in log2
-          // units, m + log2(l).
-#pragma unroll 1
-          for (int c = 0; c < kD / 32; ++c) {
-            if (lane == 0) bulk_wait_read_0();
-            __syncwarp();
+          for (int c = 0; c < 2; ++c) {
             uint32_t r[32];
-            tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(c * 32), r);
+            tmem_ld32_sync(tmem_base + lane_off + colO + uint32_t(half * 64 + c * 32), r);
+            uint32_t w[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               float lo, hi;
-              f32x2_split(mul_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv_l2), lo, hi);
-              r[2 * i] = __float_as_uint(lo);
-              r[2 * i + 1] = __float_as_uint(hi);
+              f32x2_split(mul_f32x2(f32x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv_l2), lo,
+                          hi);
+              w[i] = kStats ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
             }
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-                  make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && row0 < p.Mq) {
-              tma_store_3d(&omap, stg, it.head * kD + c * 32, row0, it.shard);
-              bulk_commit();
+            for (int q = 0; q < 4; ++q) {
+              const int chunk = c * 4 + q;  // 16-byte chunk of this lane's 128-byte row
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                  make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
             }
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.Mq) {
+            tma_store_3d(&omap, stg, it.head * kD + half * 64, row0, it.shard);
+            bulk_commit();
+          }
+        }
+        // Statistics mode: each row's log-sum-exp of the scaled scores in log2
+        // units, m + log2(l).
+        if constexpr (kStats) {
           if (row0 + lane < p.Mq)
             p.lse[(int64_t(it.shard) * p.Hs + it.head) * p.Mq + row0 + lane] = m_run + log2f(l_run);
         }

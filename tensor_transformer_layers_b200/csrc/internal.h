@@ -121,9 +121,9 @@ cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& a, int num_sm
 // Merge of per-key-block attention results (Ring attention): for every
 // (shard, row, head), O = sum_b 2^(lse_b - L) O_b / sum_b 2^(lse_b - L) with
 // L = max_b lse_b, written in bf16; lse_out (optional) = L + log2 sum_b
-// 2^(lse_b - L).  O_parts [nparts][T][M][Hs*128] fp32, lse_parts
+// 2^(lse_b - L).  O_parts [nparts][T][M][Hs*128] fp16, lse_parts
 // [nparts][T][Hs][M] fp32 (log2 units), O [T][M][Hs*128] bf16.
-cudaError_t launch_attn_merge(const float* O_parts, const float* lse_parts, int nparts, int64_t M, int Hs, int T,
+cudaError_t launch_attn_merge(const uint16_t* O_parts, const float* lse_parts, int nparts, int64_t M, int Hs, int T,
                               uint16_t* O, float* lse_out, cudaStream_t s);
 
 // One CTA whose bounded wait on an mbarrier that nothing arrives on must run

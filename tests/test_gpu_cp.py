@@ -40,7 +40,7 @@ def test_block_stats(Mq, Mk, Hs, T):
     cols = 3 * Hs * 128
     Qb = syn.normal_f16((T, Mq, cols), 1.0, seed=Mq, tid=410)
     KVb = syn.normal_f16((T, Mk, cols), 1.0, seed=Mk, tid=411)
-    O = torch.empty((T, Mq, Hs * 128), dtype=torch.float32, device="cuda")
+    O = torch.empty((T, Mq, Hs * 128), dtype=torch.float16, device="cuda")
     lse = torch.empty((T, Hs, Mq), dtype=torch.float32, device="cuda")
     assert tp.tp_sdpa_block_stats(to_dev(Qb), Mq, to_dev(KVb), Mk, Hs * T, T, O, lse) == 0
     torch.cuda.synchronize()
@@ -62,7 +62,7 @@ def test_ring_blocks_merge_to_full_attention(M, splits, Hs):
     cols = 3 * Hs * 128
     QKV = syn.normal_f16((1, M, cols), 1.0, seed=M + 1, tid=412)
     full = to_dev(QKV)
-    parts_O = torch.empty((len(splits), 1, M, Hs * 128), dtype=torch.float32, device="cuda")
+    parts_O = torch.empty((len(splits), 1, M, Hs * 128), dtype=torch.float16, device="cuda")
     parts_L = torch.empty((len(splits), 1, Hs, M), dtype=torch.float32, device="cuda")
     j0 = 0
     for b, n in enumerate(splits):
@@ -163,7 +163,7 @@ def test_flux_scale_ring_and_ulysses():
     qkv = full.view(R, Ms, 3 * D)
     ring = torch.cat([qkv, qkv]).contiguous()
     blk = Ms * 3 * D
-    Ob = torch.empty((R, R, Ms, D), dtype=torch.float32, device="cuda")
+    Ob = torch.empty((R, R, Ms, D), dtype=torch.float16, device="cuda")
     Lb = torch.empty((R, R, H, Ms), dtype=torch.float32, device="cuda")
     for s in range(R):
         kv = ring.data_ptr() + 2 * (R - s) * blk
