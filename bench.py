@@ -277,6 +277,23 @@ class MlpWorkload:
                               "rowwise")),
         ]
 
+    def context(self, g, dev):
+        """The same pair through torch (cuBLAS GEMMs with the bias in their epilogue, GELU as its own
+        kernel): a timed context row only, outside the library and the value."""
+        import torch
+        import torch.nn.functional as tF
+        M, D, F = self.cfg["M"], self.cfg["D"], self.cfg["F"]
+        X, Wu, bu = g["X"].view(torch.bfloat16), g["W_up"].view(torch.bfloat16), g["b_up"].view(torch.bfloat16)
+        Wd, bd = g["W_down"].view(torch.bfloat16), g["b_down"].view(torch.bfloat16)
+        c = {"P": torch.empty((M, F), dtype=torch.bfloat16, device=dev),
+             "H": torch.empty((M, F), dtype=torch.bfloat16, device=dev),
+             "Y": torch.empty((M, D), dtype=torch.bfloat16, device=dev)}
+        return [("cublas_up_gemm_bias", "TFLOP/s", 2.0 * M * D * F, lambda: torch.addmm(bu, X, Wu.t(), out=c["P"])),
+                ("torch_gelu_tanh", "GB/s", 2.0 * M * F * 2,
+                 lambda: c["H"].copy_(tF.gelu(c["P"], approximate="tanh"))),
+                ("cublas_down_gemm_bias", "TFLOP/s", 2.0 * M * F * D,
+                 lambda: torch.addmm(bd, c["H"], Wd.t(), out=c["Y"]))]
+
     def one_shot(self, tp, gi, dev):
         """The public one-shot call on device inputs `gi`; returns the output tensor."""
         import torch
@@ -1329,6 +1346,31 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
                                ": step i+1's host-to-device copies overlap step i's compute; device-to-host "
                                "copies on a third stream; all copies inside the timed region")}
 
+    # ---- context row: the same layer through torch / cuBLAS on the same inputs, timed the same way (not the
+    # library, not in value)
+    context = None
+    if not light and hasattr(wl, "context"):
+        ctx = wl.context(g, dev)
+        for _ in range(max(3, args.warmup)):
+            for _, _, _, fn in ctx:
+                fn()
+        torch.cuda.synchronize()
+        cev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ctx) + 1)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            cev[i][0].record()
+            for j, (_, _, _, fn) in enumerate(ctx):
+                fn()
+                cev[i][j + 1].record()
+        torch.cuda.synchronize()
+        context = {"note": "torch / cuBLAS on the same shapes and inputs, timed like the kernels above; outside "
+                           "the library and the value"}
+        for j, (name, unit, work, _) in enumerate(ctx):
+            ms = statistics.mean(cev[i][j].elapsed_time(cev[i][j + 1]) for i in range(args.steps))
+            context[name] = {"ms": round(ms, 5), "unit": unit, "achieved": round(work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9), 1)}
+        tot = sum(context[n]["ms"] for n, _, _, _ in ctx)
+        context["step_ms"] = round(tot, 5)
+        context["value"] = round(wl.work() / (tot / 1e3) / 1e12, 1)
+
     if light:  # a secondary configuration of the default run: kernels and step only, no e2e legs
         one_shot_e2e, prep, e2e = None, None, None
     else:
@@ -1375,6 +1417,8 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
         out["per_degree"] = per_group
     if prep is not None:
         out["e2e_one_shot"] = one_shot_e2e
+    if context is not None:
+        out["context_torch"] = context
     out.update({"roofline": roofline, "kernels": kinfo, "clocks": clocks, "e2e": e2e,
                 "gpu_launches": int(launches), "wall_s_timed_region": round(t_wall, 4), "cpu_baseline": None})
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not light:
