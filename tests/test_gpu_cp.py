@@ -89,6 +89,35 @@ def test_ring_blocks_merge_to_full_attention(M, splits, Hs):
         2 ** -7 * np.max(np.maximum(a, b)) + 1e-3)
 
 
+def test_block_results_near_the_fp16_limit():
+    # A block's O is a convex combination of V rows, so V values near the fp16
+    # maximum (here up to ~6e4) stay finite in the fp16 block results and in
+    # the merge; each block's O is within one fp16 rounding of the oracle's.
+    Mq, Mk, Hs = 130, 300, 1
+    qkv = syn.f16_bits_to_f64(syn.normal_f16((1, Mk, 3 * 128), 1.0, seed=77, tid=416))
+    qkv[:, :, 256:] *= 15000.0  # V: |V| up to ~6e4 (values past 65504 clipped below)
+    qkv[:, :, 256:] = np.clip(qkv[:, :, 256:], -65000.0, 65000.0)
+    bits = torch.from_numpy(qkv.astype(np.float16)).view(torch.int16).numpy()
+    full = to_dev(bits)
+    q = syn.f16_bits_to_f64(bits)[0]
+    parts_O = torch.empty((2, 1, Mq, 128), dtype=torch.float16, device="cuda")
+    parts_L = torch.empty((2, 1, 1, Mq), dtype=torch.float32, device="cuda")
+    for b, (j0, n) in enumerate(((0, 170), (170, 130))):
+        kv = full[:, j0:j0 + n].contiguous()
+        assert tp.tp_sdpa_block_stats(full[:, :Mq].contiguous(), Mq, kv, n, 1, 1, parts_O[b], parts_L[b]) == 0
+    O = torch.empty((1, Mq, 128), dtype=torch.int16, device="cuda")
+    assert tp.tp_attn_merge(parts_O, parts_L, 2, Mq, 1, 1, O) == 0
+    torch.cuda.synchronize()
+    assert tp.tp_check_device_error() == 0
+    Q = q[:Mq, :128]
+    for b, (j0, n) in enumerate(((0, 170), (170, 130))):
+        Ob = parts_O[b, 0].float().cpu().numpy().astype(np.float64)
+        assert np.all(np.isfinite(Ob)), "fp16 block result overflowed"
+        ref = o.sdpa(Q, q[j0:j0 + n, 128:256], q[j0:j0 + n, 256:])
+        assert np.max(np.abs(Ob - ref) - 2.0 ** -9 * np.abs(ref)) <= 1e-3 * np.sqrt(np.mean(ref ** 2)), f"block {b}"
+    assert_rounded_once(from_dev(O)[0], o.sdpa(Q, q[:, 128:256], q[:, 256:]), "merge near the fp16 limit")
+
+
 def test_merge_rejects_bad_part_counts():
     x = torch.zeros(64, dtype=torch.float32, device="cuda")
     y = torch.zeros(64, dtype=torch.int16, device="cuda")
