@@ -176,6 +176,12 @@ def source_sha(*names) -> str:
     return h.hexdigest()[:16]
 
 
+def has_context_row(wl) -> bool:
+    """Whether the workload's line carries the torch / cuBLAS context row: the headline MLP pair only (the
+    other workloads subclass it but are other layers)."""
+    return type(wl).__name__ == "MlpWorkload"
+
+
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source (else None)."""
@@ -1349,7 +1355,7 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
     # ---- context row: the same layer through torch / cuBLAS on the same inputs, timed the same way (not the
     # library, not in value)
     context = None
-    if not light and hasattr(wl, "context"):
+    if not light and has_context_row(wl):
         ctx = wl.context(g, dev)
         for _ in range(max(3, args.warmup)):
             for _, _, _, fn in ctx:

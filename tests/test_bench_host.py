@@ -76,3 +76,10 @@ def test_reference_arm_json_line():
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["metric"] == bench.METRIC
+
+
+def test_context_row_only_on_the_headline_pair():
+    # The torch / cuBLAS context row is built from the MLP pair's weights: every
+    # other workload (all subclasses of it) must skip it.
+    import bench
+    assert [k for k, W in bench.WORKLOADS.items() if bench.has_context_row(W())] == ["flux_mlp"]
