@@ -162,8 +162,8 @@ tp_status tp_shard_weight_all(const uint16_t* W, int64_t rows, int64_t cols, int
  * Every job is checked as the corresponding single call before anything is
  * launched.  Each job's output is all T shards stacked in rank order.  A
  * colwise layer's bias of n elements is the job {b, T, n/T, TP_COLWISE} (or
- * {b, 1, n, TP_ROWWISE}: the same slices).  One launch for up to 8 plain jobs
- * or packed blocks in all, one more per further 8. */
+ * {b, 1, n, TP_ROWWISE}: the same slices).  One launch for up to 16 plain
+ * jobs or packed blocks in all, one more per further 16. */
 typedef struct {
   const uint16_t* W;     /* device, [rows x cols] */
   int64_t rows, cols;

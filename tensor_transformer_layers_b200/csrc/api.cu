@@ -360,10 +360,10 @@ int packed_jobs(const uint16_t* W, int64_t rows, int64_t cols, int style, const 
   return nb;
 }
 
-// Launches jobs in groups of kMaxSliceJobs.
+// Launches jobs in groups of kSliceJobsPerLaunch.
 tp_status run_slice_jobs(const SliceJob* jobs, int n, cudaStream_t s) {
-  for (int i = 0; i < n; i += kMaxSliceJobs) {
-    const int k = n - i < kMaxSliceJobs ? n - i : kMaxSliceJobs;
+  for (int i = 0; i < n; i += kSliceJobsPerLaunch) {
+    const int k = n - i < kSliceJobsPerLaunch ? n - i : kSliceJobsPerLaunch;
     if (launch_slice_jobs(jobs + i, k, s) != cudaSuccess) return TP_ERR_CUDA;
   }
   return TP_OK;

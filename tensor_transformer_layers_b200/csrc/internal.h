@@ -22,10 +22,13 @@ cudaError_t launch_slice_copy(const uint16_t* src, uint16_t* dst, int64_t nblock
                               int64_t nblocks2 = 1, int64_t src_bstride2 = 0, int64_t dst_bstride2 = 0,
                               int64_t dst_ld = -1);
 
-// Up to kMaxSliceJobs blocked 2-D copies (same meaning as above, one block
-// index) in one launch.  Element units; cols, the lds, the strides and both
-// pointers multiples of 8 elements / 16 bytes.
+// Blocked 2-D copies (same meaning as above, one block index), up to
+// kSliceJobsPerLaunch in one launch.  Element units; cols, the lds, the
+// strides and both pointers multiples of 8 elements / 16 bytes.
+// kMaxSliceJobs bounds the jobs of one tp_shard_weights_batch call (each may
+// expand into several copies: one per packed block).
 constexpr int kMaxSliceJobs = 8;
+constexpr int kSliceJobsPerLaunch = 16;
 struct SliceJob {
   const uint16_t* src;
   uint16_t* dst;

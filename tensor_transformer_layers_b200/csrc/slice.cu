@@ -51,11 +51,11 @@ __global__ void __launch_bounds__(kThreads) slice_copy_kernel(const uint4* __res
 // space with them; a job that is one contiguous span per block has rows = 1
 // and a single block needs no division (the branches are uniform per CTA).
 struct SliceJobs {
-  const uint4* src[kMaxSliceJobs];
-  uint4* dst[kMaxSliceJobs];
-  uint32_t nblocks[kMaxSliceJobs], rows[kMaxSliceJobs], c8[kMaxSliceJobs];
-  int64_t src_ld8[kMaxSliceJobs], dst_ld8[kMaxSliceJobs], src_b8[kMaxSliceJobs], dst_b8[kMaxSliceJobs];
-  int cta0[kMaxSliceJobs + 1];
+  const uint4* src[kSliceJobsPerLaunch];
+  uint4* dst[kSliceJobsPerLaunch];
+  uint32_t nblocks[kSliceJobsPerLaunch], rows[kSliceJobsPerLaunch], c8[kSliceJobsPerLaunch];
+  int64_t src_ld8[kSliceJobsPerLaunch], dst_ld8[kSliceJobsPerLaunch], src_b8[kSliceJobsPerLaunch], dst_b8[kSliceJobsPerLaunch];
+  int cta0[kSliceJobsPerLaunch + 1];
   int njobs;
 };
 
@@ -102,9 +102,9 @@ __global__ void __launch_bounds__(kThreads) slice_jobs_kernel(const __grid_const
 
 cudaError_t launch_slice_jobs(const SliceJob* jobs, int njobs, cudaStream_t st) {
   if (njobs <= 0) return cudaSuccess;
-  if (njobs > kMaxSliceJobs) return note_cuda_error("slice jobs: too many jobs", cudaErrorInvalidValue);
+  if (njobs > kSliceJobsPerLaunch) return note_cuda_error("slice jobs: too many jobs", cudaErrorInvalidValue);
   SliceJobs J{};
-  int64_t chunks[kMaxSliceJobs], all = 0;
+  int64_t chunks[kSliceJobsPerLaunch], all = 0;
   bool fits = true;
   for (int j = 0; j < njobs; ++j) {
     SliceJob s = jobs[j];
