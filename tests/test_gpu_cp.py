@@ -56,7 +56,10 @@ def test_block_stats(Mq, Mk, Hs, T):
             assert np.max(np.abs(Lg[r][j] - ref_lse / LN2)) <= 2e-3, "log-sum-exp (log2 units)"
 
 
-@pytest.mark.parametrize("M,splits,Hs", [(640, [256, 256, 128], 2), (1000, [300, 1, 699], 1), (512, [512], 1)])
+# up to 8 blocks the merge is instantiated per block count; 10 and 12 blocks
+# take the run-time-count path
+@pytest.mark.parametrize("M,splits,Hs", [(640, [256, 256, 128], 2), (1000, [300, 1, 699], 1), (512, [512], 1),
+                                         (640, [64] * 10, 1), (700, [50, 70, 30, 100, 40, 60, 80, 20, 90, 10, 70, 80], 2)])
 def test_ring_blocks_merge_to_full_attention(M, splits, Hs):
     # One "rank" holds all M queries; the keys arrive in blocks, as on a ring.
     cols = 3 * Hs * 128
