@@ -53,8 +53,8 @@
 // budget of the block.  S, the row statistics and O accumulate in fp32; O is
 // written in bf16 for the out-projection.  A Ring block's O is written in
 // fp16: each row is a convex combination of fp16 rows of V, so it stays in
-// fp16's range, and its rounding (2^-11 relative) is a quarter of the bf16
-// rounding the merged output takes once.
+// fp16's range, and its rounding (at most 2^-11 relative) is an eighth of
+// the bf16 rounding (2^-8) the merged output takes once.
 // Every mbarrier wait is bounded (ptx.cuh); a timeout drains and exits.
 #include <cuda_bf16.h>
 
