@@ -17,7 +17,7 @@ step-level calls are bit-identical to ``tp_mlp_run`` and ``tp_mlp_pair``).
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                        [--workload flux_mlp|flux_mlp_sweep|flux_attn|wide_block|flux_reduce|flux_swiglu|
                                    flux_split_input|flux_joint_attn|flux_ring_attn|flux_ulysses_attn]
-                       [--mode replicas|tp] [--no-cpu-baseline] [--headline-only]
+                       [--mode replicas|tp] [--no-cpu-baseline] [--headline-only] [--context-torch]
 The default workload (flux_mlp) is the headline line.  The others time the
 remaining rows the same way: flux_mlp_sweep (the same pair at tp_degree 1, 2,
 4 and 8, one kernel set per degree), flux_attn (QKV head split, QKV GEMM, SDPA,
@@ -1355,7 +1355,7 @@ def run_ours(args, wl, rank, local_rank, world, light=False):
     # ---- context row: the same layer through torch / cuBLAS on the same inputs, timed the same way (not the
     # library, not in value)
     context = None
-    if not light and has_context_row(wl):
+    if not light and getattr(args, "context_torch", False) and has_context_row(wl):
         ctx = wl.context(g, dev)
         for _ in range(max(3, args.warmup)):
             for _, _, _, fn in ctx:
@@ -1602,6 +1602,9 @@ def main(argv=None):
     ap.add_argument("--headline-only", action="store_true",
                     help="leave out the other configurations that a default one-GPU run times after the "
                          "headline (other_configs)")
+    ap.add_argument("--context-torch", action="store_true",
+                    help="also time the same MLP pair through torch / cuBLAS (context_torch: a context row outside "
+                         "the library and the value; flux_mlp only)")
     ap.add_argument("--mode", choices=["replicas", "tp"], default="replicas",
                     help="replicas (default): every GPU runs the whole layer (all tp_degree shards) on its own "
                          "tokens; tp: tensor parallelism across the processes, one shard per rank, one NCCL "
